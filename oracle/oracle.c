@@ -1,0 +1,456 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU reference for the mask-free spatially
+ * adaptive DiT attention path (SAFE-DiT's PCSP / exact mask elision / SRSU +
+ * CAR / SW-CFG, and AccelAes' SkipSparse query-subset attention).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file: only the test suite, the smoke check and the benchmark's CPU
+ * baseline leg do.  It shares no code, header, table or helper with the CUDA
+ * library; the two meet only at the seeded synthetic inputs.
+ *
+ * Every value is read as double (bf16/fp16/fp32 inputs are widened exactly by
+ * the caller) and every result is computed in double, in the order the
+ * definition states.  No blocking, fusion or reordering beyond that.
+ *
+ * Sources (cited per function):
+ *   [P1] "기술 요약: SAFE-DiT" (gist.science/ko/paper/2606.29360):
+ *        문제 정의; 방법론 items 1-4.
+ *   [P4] "SAFE-DiT: Semantics-Aware Fast-path Execution for High-Resolution
+ *        Diffusion Transformers" (gist.science/it/paper/2606.29360):
+ *        Riepilogo Tecnico, Metodologia items 1-4 (same content as P1).
+ *   [P3] AccelAes technical summary (gist.science/ko/paper/2603.12575):
+ *        2. 방법론, B.1 AesMask and B.2 SkipSparse.
+ *
+ * Readings where the pages are silent:
+ *   - softmax scale is a caller argument (1/sqrt(d) by default upstream);
+ *   - scores are summed over heads, positions and calls (sum, not mean);
+ *   - |S| = k is a caller argument; ties at the threshold go to the lower
+ *     token index; S and C are both returned in ascending index order;
+ *   - s_i is the min-max normalised score (0 when all scores are equal);
+ *   - CFG combine is eps_u + gamma_i * (eps_c - eps_u);
+ *   - a bool mask entry True means "attend" (additive 0), False means -inf;
+ *   - a row whose every key is masked is an error (the softmax is undefined).
+ *
+ * Return codes: 0 = ok, -1 = invalid argument, -2 = index out of range or
+ * duplicated, -3 = a row with no admissible key, -4 = NaN score.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define OR_OK 0
+#define OR_EINVAL (-1)
+#define OR_EINDEX (-2)
+#define OR_EMASKED (-3)
+#define OR_ENAN (-4)
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* C1  Image->text cross-attention probabilities for one batch entry.
+ *
+ * [P1 방법론 2 / P4 Metodologia 2]: during a short warm-up the model gathers
+ * the attention weights that image tokens give to the text content tokens.
+ * [P3 B.1 step 3]: the attention weights from image tokens to the selected
+ * text tokens are aggregated into an affinity map.
+ * [P1 방법론 1 "보존" / P4 "Preservazione"]: the text-padding mask is a
+ * semantic mask and is kept, so a padding key receives weight exactly 0.
+ *
+ * For every head h and image token i:
+ *   l_ij = scale * sum_c q[h][i][c] * k[h][j][c]    over valid text keys j
+ *   P[h][i][j] = exp(l_ij - max_j' l_ij') / sum_j'' exp(l_ij'' - max)
+ *   P[h][i][j] = 0 for padding keys (assigned, never exponentiated).
+ * q: [H][N][d], k: [H][L][d], key_valid: [L] (nonzero = valid), P: [H][N][L].
+ */
+int oracle_cross_attn_probs(int64_t H, int64_t N, int64_t L, int64_t d,
+                            const double *q, const double *k,
+                            const uint8_t *key_valid, double scale,
+                            double *P) {
+  if (H < 0 || N < 0 || L <= 0 || d <= 0 || !q || !k || !key_valid || !P)
+    return OR_EINVAL;
+  int64_t n_valid = 0;
+  for (int64_t j = 0; j < L; ++j) n_valid += key_valid[j] != 0;
+  if (n_valid == 0 && H * N > 0) return OR_EMASKED;
+  int64_t total = H * N;
+#pragma omp parallel for schedule(static)
+  for (int64_t hi = 0; hi < total; ++hi) {
+    int64_t h = hi / N, i = hi % N;
+    const double *qi = q + (h * N + i) * d;
+    double *Pi = P + (h * N + i) * L;
+    double m = -INFINITY;
+    for (int64_t j = 0; j < L; ++j) {
+      if (!key_valid[j]) continue;
+      const double *kj = k + (h * L + j) * d;
+      double dot = 0.0;
+      for (int64_t c = 0; c < d; ++c) dot += qi[c] * kj[c];
+      Pi[j] = scale * dot; /* logit, overwritten below */
+      if (Pi[j] > m) m = Pi[j];
+    }
+    double denom = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+      if (!key_valid[j]) continue;
+      Pi[j] = exp(Pi[j] - m);
+      denom += Pi[j];
+    }
+    for (int64_t j = 0; j < L; ++j) Pi[j] = key_valid[j] ? Pi[j] / denom : 0.0;
+  }
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* C2  Sensitivity score aggregation.
+ *
+ * [P1 방법론 2 / P4 Metodologia 2]: weights from image tokens to the text
+ * *content* tokens are aggregated over the warm-up.  [P3 B.1 step 3]: the
+ * attention given to the selected tokens is aggregated per image token.
+ *
+ *   score[i] += sum_h sum_{j : content[j]} P[h][i][j]
+ * summed in double, h outer and j inner.  P: [H][N][L].
+ */
+int oracle_partition_accumulate(int64_t H, int64_t N, int64_t L,
+                                const double *P, const uint8_t *content,
+                                double *score) {
+  if (H < 0 || N < 0 || L < 0 || !P || !content || !score) return OR_EINVAL;
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < N; ++i) {
+    double acc = 0.0;
+    for (int64_t h = 0; h < H; ++h) {
+      const double *row = P + (h * N + i) * L;
+      for (int64_t j = 0; j < L; ++j)
+        if (content[j]) acc += row[j];
+    }
+    score[i] += acc;
+  }
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* C3 + C4  Partition into the sensitive set S and the context set C, and the
+ * sensitivity score s_i.
+ *
+ * [P1 방법론 2 / P4 Metodologia 2]: image tokens are split into S and C, and
+ * the split is then fixed for the trajectory.  [P3 B.1 step 4]: a percentile
+ * threshold marks the important region; with |S| = k this is the top k.
+ * [P1 방법론 4 / P4 Metodologia 4]: the PCSP sensitivity score s_i drives the
+ * per-token guidance, so it lies in [0, 1]; here the min-max normalised score.
+ *
+ * Token i is in S iff its rank is below k, where
+ *   rank_i = #{ j : score_j > score_i  or (score_j == score_i and j < i) },
+ * i.e. order by score descending, ties to the lower index.  Written as an
+ * all-pairs count on purpose (O(N^2)): no sort, obviously the definition.
+ * idx_s: [k] ascending; idx_c: [N-k] ascending;
+ * s[i] = (score_i - min) / (max - min) in double, rounded to float; 0 if
+ * max == min.
+ */
+int oracle_partition_select(int64_t N, int64_t k, const double *score,
+                            int32_t *idx_s, int32_t *idx_c, float *s) {
+  if (N < 0 || k < 0 || k > N || !score) return OR_EINVAL;
+  for (int64_t i = 0; i < N; ++i)
+    if (isnan(score[i])) return OR_ENAN;
+  uint8_t *in_s = (uint8_t *)calloc((size_t)(N > 0 ? N : 1), 1);
+  if (!in_s) return OR_EINVAL;
+#pragma omp parallel for schedule(dynamic, 64)
+  for (int64_t i = 0; i < N; ++i) {
+    int64_t rank = 0;
+    for (int64_t j = 0; j < N; ++j)
+      if (score[j] > score[i] || (score[j] == score[i] && j < i)) ++rank;
+    in_s[i] = rank < k;
+  }
+  int64_t ns = 0, nc = 0;
+  for (int64_t i = 0; i < N; ++i) {
+    if (in_s[i]) {
+      if (idx_s) idx_s[ns] = (int32_t)i;
+      ++ns;
+    } else {
+      if (idx_c) idx_c[nc] = (int32_t)i;
+      ++nc;
+    }
+  }
+  free(in_s);
+  if (s && N > 0) {
+    double lo = score[0], hi = score[0];
+    for (int64_t i = 1; i < N; ++i) {
+      if (score[i] < lo) lo = score[i];
+      if (score[i] > hi) hi = score[i];
+    }
+    for (int64_t i = 0; i < N; ++i)
+      s[i] = (hi == lo) ? 0.0f : (float)((score[i] - lo) / (hi - lo));
+  }
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* C5  Exact mask-elision criterion.
+ *
+ * [P1 방법론 1 / P4 Metodologia 1]: an additive mask m is removable when its
+ * effect on the logits is only a per-row constant shift L_{i,:} + c_i, which
+ * softmax normalisation cancels.  [P1 문제 정의, 방법론 1]: an "all-valid"
+ * image self-attention mask is the case to remove; text-padding, causal and
+ * non-uniform bias masks are semantic and kept.
+ *
+ * Row r is removable iff every entry equals entry 0 under IEEE == (so +0 and
+ * -0 agree and NaN never does) and entry 0 is finite (a row of -inf is a
+ * fully masked row, not a shift).  mask: [rows][cols]; row_flag (nullable):
+ * [rows], 1 = removable.  Returns the AND over rows (1 = the whole mask may
+ * be dropped), or a negative error code.
+ */
+int oracle_mask_row_constant(int64_t rows, int64_t cols, const double *mask,
+                             uint8_t *row_flag) {
+  if (rows < 0 || cols <= 0 || !mask) return OR_EINVAL;
+  int verdict = 1;
+  for (int64_t r = 0; r < rows; ++r) {
+    const double *m = mask + r * cols;
+    int ok = isfinite(m[0]) ? 1 : 0;
+    for (int64_t j = 1; j < cols && ok; ++j)
+      if (!(m[j] == m[0])) ok = 0;
+    if (row_flag) row_flag[r] = (uint8_t)ok;
+    verdict &= ok;
+  }
+  return verdict;
+}
+
+/* Boolean masks take part through their additive meaning: an entry that
+ * allows attention is the additive value 0, one that forbids it is -inf
+ * (the boolean attention-mask convention of PyTorch SDPA, the stack the
+ * SAFE-DiT pages evaluate on [P1 실험 결과]).  The criterion is then C5. */
+int oracle_mask_row_constant_bool(int64_t rows, int64_t cols,
+                                  const uint8_t *mask, uint8_t *row_flag) {
+  if (rows < 0 || cols <= 0 || !mask) return OR_EINVAL;
+  double *add = (double *)malloc(sizeof(double) * (size_t)cols);
+  if (!add) return OR_EINVAL;
+  int verdict = 1;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t j = 0; j < cols; ++j)
+      add[j] = mask[r * cols + j] ? 0.0 : -INFINITY;
+    uint8_t f = 0;
+    int v = oracle_mask_row_constant(1, cols, add, &f);
+    if (row_flag) row_flag[r] = f;
+    verdict &= v;
+  }
+  free(add);
+  return verdict;
+}
+
+/* ------------------------------------------------------------------------ */
+/* C6a  Subset attention (SRSU), one (batch, head) slice, row by row.
+ *
+ * [P1 방법론 3 / P4 Metodologia 3]: on non-anchor steps only the query rows of
+ * the sensitive set are updated, and those queries still attend to the global
+ * key/value set (fresh sensitive states plus cached context states).
+ * [P3 B.2]: queries only for focus tokens, keys and values from the whole
+ * image.  [P1 방법론 1]: kept semantic masks enter as additive terms.
+ *
+ * For r in [0, n_idx), i = idx[r] (or i = r when idx is NULL):
+ *   l_j = scale * q_i . k_j + pad[j] + bias_rows[r][j]      for j in [0, N)
+ *   m = max_j l_j;  p_j = exp(l_j - m)  (p_j = 0 where l_j = -inf)
+ *   out[r] = sum_j p_j v_j / sum_j p_j
+ * q: [Nq][d]; k, v: [N][d]; pad: [N] or NULL; bias_rows: [n_idx][N] (the bias
+ * rows of the requested queries) or NULL; out: [n_idx][d].
+ */
+int oracle_attn_subset(int64_t Nq, int64_t N, int64_t d, const double *q,
+                       const double *k, const double *v, const int32_t *idx,
+                       int64_t n_idx, const double *pad,
+                       const double *bias_rows, double scale, double *out) {
+  if (Nq < 0 || N <= 0 || d <= 0 || n_idx < 0 || !q || !k || !v || !out)
+    return OR_EINVAL;
+  for (int64_t r = 0; r < n_idx; ++r) {
+    int64_t i = idx ? idx[r] : r;
+    if (i < 0 || i >= Nq) return OR_EINDEX;
+  }
+  int err = OR_OK;
+#pragma omp parallel
+  {
+    double *l = (double *)malloc(sizeof(double) * (size_t)N);
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t r = 0; r < n_idx; ++r) {
+      int64_t i = idx ? idx[r] : r;
+      const double *qi = q + i * d;
+      double m = -INFINITY;
+      for (int64_t j = 0; j < N; ++j) {
+        double dot = 0.0;
+        for (int64_t c = 0; c < d; ++c) dot += qi[c] * k[j * d + c];
+        l[j] = scale * dot;
+        if (pad) l[j] += pad[j];
+        if (bias_rows) l[j] += bias_rows[r * N + j];
+        if (l[j] > m) m = l[j];
+      }
+      double *o = out + r * d;
+      for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+      if (m == -INFINITY) {
+#pragma omp atomic write
+        err = OR_EMASKED;
+        continue;
+      }
+      double denom = 0.0;
+      for (int64_t j = 0; j < N; ++j) {
+        double p = (l[j] == -INFINITY) ? 0.0 : exp(l[j] - m);
+        denom += p;
+        for (int64_t c = 0; c < d; ++c) o[c] += p * v[j * d + c];
+      }
+      for (int64_t c = 0; c < d; ++c) o[c] /= denom;
+    }
+    free(l);
+  }
+  return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* C6b  Dense attention (CAR anchor step), one (batch, head) slice, in matrix
+ * form.  Written separately from C6a so that the two can check each other.
+ *
+ * [P1 방법론 3 / P4 Metodologia 3]: periodic anchor steps perform a dense
+ * update that refreshes the cached state of every token.
+ *
+ *   Lg = scale * Q K^T + 1 pad^T + Bias           ([Nq][N])
+ *   Pm = exp(Lg - rowmax(Lg));  O = (Pm V) ./ rowsum(Pm)
+ * computed one block of query rows at a time (to bound memory): first the
+ * whole logit block, then its row maxima, then the exponentials and row sums,
+ * then the block product with V.
+ */
+int oracle_attn_dense(int64_t Nq, int64_t N, int64_t d, const double *q,
+                      const double *k, const double *v, const double *pad,
+                      const double *bias, double scale, double *out) {
+  if (Nq < 0 || N <= 0 || d <= 0 || !q || !k || !v || !out) return OR_EINVAL;
+  const int64_t BR = 32; /* query rows per block */
+  int64_t nblk = (Nq + BR - 1) / BR;
+  int err = OR_OK;
+#pragma omp parallel
+  {
+    double *Lg = (double *)malloc(sizeof(double) * (size_t)(BR * N));
+    double *rmax = (double *)malloc(sizeof(double) * (size_t)BR);
+    double *rsum = (double *)malloc(sizeof(double) * (size_t)BR);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t blk = 0; blk < nblk; ++blk) {
+      int64_t i0 = blk * BR, nb = (Nq - i0 < BR) ? Nq - i0 : BR;
+      /* logit block */
+      for (int64_t a = 0; a < nb; ++a)
+        for (int64_t j = 0; j < N; ++j) {
+          double dot = 0.0;
+          for (int64_t c = 0; c < d; ++c)
+            dot += q[(i0 + a) * d + c] * k[j * d + c];
+          double x = scale * dot;
+          if (pad) x += pad[j];
+          if (bias) x += bias[(i0 + a) * N + j];
+          Lg[a * N + j] = x;
+        }
+      /* row maxima */
+      for (int64_t a = 0; a < nb; ++a) {
+        rmax[a] = -INFINITY;
+        for (int64_t j = 0; j < N; ++j)
+          if (Lg[a * N + j] > rmax[a]) rmax[a] = Lg[a * N + j];
+        if (rmax[a] == -INFINITY) {
+#pragma omp atomic write
+          err = OR_EMASKED;
+        }
+      }
+      /* exponentials and row sums */
+      for (int64_t a = 0; a < nb; ++a) {
+        rsum[a] = 0.0;
+        for (int64_t j = 0; j < N; ++j) {
+          double x = Lg[a * N + j];
+          double p = (x == -INFINITY || rmax[a] == -INFINITY) ? 0.0
+                                                              : exp(x - rmax[a]);
+          Lg[a * N + j] = p;
+          rsum[a] += p;
+        }
+      }
+      /* block product with V, then row normalisation */
+      for (int64_t a = 0; a < nb; ++a) {
+        double *o = out + (i0 + a) * d;
+        for (int64_t c = 0; c < d; ++c) {
+          double acc = 0.0;
+          for (int64_t j = 0; j < N; ++j) acc += Lg[a * N + j] * v[j * d + c];
+          o[c] = rsum[a] > 0.0 ? acc / rsum[a] : 0.0;
+        }
+      }
+    }
+    free(Lg);
+    free(rmax);
+    free(rsum);
+  }
+  return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* C7  State scatter and gather.
+ *
+ * [P1 방법론 3 / P4 Metodologia 3]: the context states are cached and reused
+ * between anchors; the sensitive rows computed on an SRSU step replace their
+ * entries in the cached state.
+ *   scatter: dst[idx[r]] = src[r]   (all other rows of dst untouched)
+ *   gather:  dst[r] = src[idx[r]]
+ * Rows are opaque byte strings of row_bytes each.  Every index is checked
+ * (range, and uniqueness for scatter) before anything is written.
+ */
+static int check_index(const int32_t *idx, int64_t n_idx, int64_t N,
+                       int unique) {
+  uint8_t *seen = unique ? (uint8_t *)calloc((size_t)(N > 0 ? N : 1), 1) : NULL;
+  if (unique && !seen) return OR_EINVAL;
+  int rc = OR_OK;
+  for (int64_t r = 0; r < n_idx && rc == OR_OK; ++r) {
+    if (idx[r] < 0 || idx[r] >= N)
+      rc = OR_EINDEX;
+    else if (unique) {
+      if (seen[idx[r]]) rc = OR_EINDEX;
+      seen[idx[r]] = 1;
+    }
+  }
+  free(seen);
+  return rc;
+}
+
+int oracle_scatter_rows(int64_t n_idx, int64_t N, int64_t row_bytes,
+                        const uint8_t *src, uint8_t *dst, const int32_t *idx) {
+  if (n_idx < 0 || N < 0 || row_bytes <= 0 || (n_idx && (!src || !idx)) || !dst)
+    return OR_EINVAL;
+  int rc = check_index(idx, n_idx, N, 1);
+  if (rc) return rc;
+  for (int64_t r = 0; r < n_idx; ++r)
+    memcpy(dst + (int64_t)idx[r] * row_bytes, src + r * row_bytes,
+           (size_t)row_bytes);
+  return OR_OK;
+}
+
+int oracle_gather_rows(int64_t n_idx, int64_t N, int64_t row_bytes,
+                       const uint8_t *src, uint8_t *dst, const int32_t *idx) {
+  if (n_idx < 0 || N < 0 || row_bytes <= 0 || (n_idx && (!dst || !idx)) || !src)
+    return OR_EINVAL;
+  int rc = check_index(idx, n_idx, N, 0);
+  if (rc) return rc;
+  for (int64_t r = 0; r < n_idx; ++r)
+    memcpy(dst + r * row_bytes, src + (int64_t)idx[r] * row_bytes,
+           (size_t)row_bytes);
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* C8  Sensitivity-weighted classifier-free guidance.
+ *
+ * [P1 방법론 4 / P4 Metodologia 4]: gamma_i = gamma_ctx + (gamma_sens -
+ * gamma_ctx) s_i, applied to the prediction after the forward pass.
+ * [P3 B.2]: spatial CFG, a high scale on focus tokens and a low one on the
+ * background (the binary-s special case).  Combine convention (reading):
+ *   out[i][f] = eps_u[i][f] + gamma_i * (eps_c[i][f] - eps_u[i][f]).
+ */
+void oracle_sw_cfg(int64_t N, int64_t F, const double *eps_c,
+                   const double *eps_u, const double *s, double gamma_ctx,
+                   double gamma_sens, double *out) {
+  for (int64_t i = 0; i < N; ++i) {
+    double g = gamma_ctx + (gamma_sens - gamma_ctx) * s[i];
+    for (int64_t f = 0; f < F; ++f) {
+      int64_t e = i * F + f;
+      out[e] = eps_u[e] + g * (eps_c[e] - eps_u[e]);
+    }
+  }
+}

@@ -1,0 +1,309 @@
+"""Pins of the fp64 CPU oracle against things other than itself: closed forms,
+hand-derived fixtures, brute force on tiny inputs, invariants the pages state,
+and library routines (torch float64 softmax / SDPA, numpy einsum) for the cases
+that reduce to them.  Each test names the passage it follows.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(20261202)
+
+
+def _lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+# ---------------------------------------------------------------------------
+# Attention (C6): SAFE-DiT summary, 방법론 3 (SRSU / CAR); AccelAes B.2.
+# ---------------------------------------------------------------------------
+def test_subset_rows_equal_dense_rows():
+    """An S row attends to the global K/V, so it equals the same row of the
+    dense (anchor) attention [SAFE-DiT summary, 방법론 3]."""
+    Nq, N, d = 67, 53, 12
+    q, k, v = rng.standard_normal((Nq, d)), rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    idx = np.sort(rng.choice(Nq, size=23, replace=False)).astype(np.int32)
+    dense = oracle.attn_dense(q, k, v)
+    sub = oracle.attn_subset(q, k, v, idx)
+    assert np.abs(sub - dense[idx]).max() <= 1e-13
+    ident = oracle.attn_subset(q, k, v, np.arange(Nq, dtype=np.int32))
+    assert np.abs(ident - dense).max() <= 1e-13
+
+
+def test_attention_matches_torch_sdpa_float64():
+    """Library routine: torch SDPA in float64 with an additive mask (key
+    padding + non-uniform bias), scale 1/sqrt(d) and a custom scale."""
+    Nq, N, d = 40, 70, 16
+    q, k, v = rng.standard_normal((Nq, d)), rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    pad = np.where(rng.random(N) < 0.2, -np.inf, 0.0)
+    pad[0] = 0.0
+    bias = rng.standard_normal((Nq, N))
+    for scale in (None, 0.37):
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.tensor(q)[None], torch.tensor(k)[None], torch.tensor(v)[None],
+            attn_mask=torch.tensor(pad[None, :] + bias)[None],
+            scale=scale).numpy()[0]
+        dense = oracle.attn_dense(q, k, v, pad=pad, bias=bias, scale=scale)
+        idx = np.arange(Nq, dtype=np.int32)[::3].copy()
+        sub = oracle.attn_subset(q, k, v, idx, pad=pad, bias_rows=bias[idx], scale=scale)
+        assert np.abs(dense - ref).max() <= 1e-12
+        assert np.abs(sub - ref[idx]).max() <= 1e-12
+    # transposed operand / wrong scale would fail this: check the scale is used
+    ref1 = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None], torch.tensor(k)[None], torch.tensor(v)[None]).numpy()[0]
+    assert np.abs(oracle.attn_dense(q, k, v, scale=0.9) - ref1).max() > 1e-3
+
+
+def test_row_constant_shift_is_invisible():
+    """An additive mask that shifts each row by a constant c_i does not change
+    softmax outputs [SAFE-DiT summary, 방법론 1; Italian page, Metodologia 1]."""
+    Nq, N, d = 33, 41, 8
+    q, k, v = rng.standard_normal((Nq, d)), rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    base = oracle.attn_dense(q, k, v)
+    c = rng.uniform(-4, 4, size=(Nq, 1)) * np.ones((1, N))
+    assert np.abs(oracle.attn_dense(q, k, v, bias=c) - base).max() <= 1e-13
+    idx = np.arange(0, Nq, 2, dtype=np.int32)
+    assert np.abs(oracle.attn_subset(q, k, v, idx, bias_rows=c[idx]) - base[idx]).max() <= 1e-13
+    zero = np.zeros((Nq, N))
+    assert np.array_equal(oracle.attn_dense(q, k, v, bias=zero), base)
+    # a non-uniform bias is not a shift: it must change the output
+    assert np.abs(oracle.attn_dense(q, k, v, bias=rng.standard_normal((Nq, N))) - base).max() > 1e-3
+
+
+def test_padding_keys_get_exactly_zero_weight_in_attention():
+    """Kept semantic masks [SAFE-DiT summary, 방법론 1 보존]: a -inf padded key
+    contributes exactly nothing; bit-identical to removing the key."""
+    Nq, N, d, n_pad = 20, 48, 8, 11
+    q, k, v = rng.standard_normal((Nq, d)), rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    pad = np.zeros(N)
+    pad[N - n_pad:] = -np.inf
+    with_pad = oracle.attn_subset(q, k, v, pad=pad)
+    removed = oracle.attn_subset(q, k[: N - n_pad], v[: N - n_pad])
+    assert np.array_equal(with_pad, removed)
+    v2 = v.copy()
+    v2[N - n_pad:] = 1e30  # garbage in padded values must not leak
+    assert np.array_equal(oracle.attn_subset(q, k, v2, pad=pad), removed)
+
+
+def test_attention_closed_forms():
+    d = 5
+    # one key: output is that value row
+    q, k, v = rng.standard_normal((3, d)), rng.standard_normal((1, d)), rng.standard_normal((1, d))
+    assert np.array_equal(oracle.attn_subset(q, k, v), np.repeat(v, 3, axis=0))
+    # all-equal logits (q = 0): output is the mean of V
+    N = 37
+    k, v = rng.standard_normal((N, d)), rng.standard_normal((N, d))
+    out = oracle.attn_dense(np.zeros((2, d)), k, v)
+    assert np.abs(out - v.mean(axis=0)).max() <= 1e-14
+    # d = 1, two keys: logistic weights
+    qs, k2, v2 = 0.7, np.array([[1.5], [-0.5]]), np.array([[2.0], [-3.0]])
+    w1 = 1.0 / (1.0 + math.exp(-(qs * (1.5 - (-0.5)) * 0.8)))
+    out = oracle.attn_subset(np.array([[qs]]), k2, v2, scale=0.8)
+    assert abs(out[0, 0] - (w1 * 2.0 + (1 - w1) * (-3.0))) <= 1e-15
+
+
+def test_fully_masked_row_is_an_error():
+    q, k, v = np.ones((2, 3)), np.ones((4, 3)), np.ones((4, 3))
+    with pytest.raises(oracle.OracleError):
+        oracle.attn_subset(q, k, v, pad=np.full(4, -np.inf))
+    with pytest.raises(oracle.OracleError):
+        oracle.attn_dense(q, k, v, pad=np.full(4, -np.inf))
+    with pytest.raises(oracle.OracleError):
+        oracle.attn_subset(q, k, v, idx=np.array([2], dtype=np.int32))
+
+
+# ---------------------------------------------------------------------------
+# Cross-attention probabilities (C1): SAFE-DiT summary 방법론 2; AccelAes B.1.
+# ---------------------------------------------------------------------------
+def test_cross_attn_probs_padding_and_softmax():
+    H, N, L, d, nv = 3, 17, 12, 8, 7
+    q, k = rng.standard_normal((H, N, d)), rng.standard_normal((H, L, d))
+    valid = np.zeros(L, dtype=np.uint8)
+    valid[:nv] = 1
+    P = oracle.cross_attn_probs(q, k, valid)
+    assert np.all(P[:, :, nv:] == 0.0)
+    assert np.abs(P.sum(-1) - 1.0).max() <= 1e-14
+    # library routine: float64 softmax over the valid keys
+    logits = torch.einsum("hnd,hld->hnl", torch.tensor(q), torch.tensor(k[:, :nv])) / math.sqrt(d)
+    ref = torch.softmax(logits, dim=-1).numpy()
+    assert np.abs(P[:, :, :nv] - ref).max() <= 1e-15
+    # the padded tail physically removed gives bit-identical probabilities
+    P2 = oracle.cross_attn_probs(q, k[:, :nv], valid[:nv])
+    assert np.array_equal(P[:, :, :nv], P2)
+    # non-prefix padding pattern
+    valid3 = (rng.random(L) < 0.5).astype(np.uint8)
+    valid3[3] = 1
+    P3 = oracle.cross_attn_probs(q, k, valid3)
+    assert np.all(P3[:, :, valid3 == 0] == 0.0)
+    with pytest.raises(oracle.OracleError):
+        oracle.cross_attn_probs(q, k, np.zeros(L, dtype=np.uint8))
+
+
+# ---------------------------------------------------------------------------
+# Partition (C2-C4): SAFE-DiT summary 방법론 2; AccelAes B.1 step 4.
+# ---------------------------------------------------------------------------
+def test_accumulate_matches_einsum_and_content_selection():
+    H, N, L = 4, 29, 10
+    P = rng.random((H, N, L))
+    content = (rng.random(L) < 0.6).astype(np.uint8)
+    start = rng.random(N)
+    got = oracle.partition_accumulate(P, content, start)
+    ref = start + np.einsum("hnl,l->n", P, content.astype(np.float64))
+    assert np.abs(got - ref).max() <= 1e-13
+    # only content positions count: changing a non-content column changes nothing
+    P2 = P.copy()
+    P2[:, :, content == 0] += 5.0
+    assert np.array_equal(oracle.partition_accumulate(P2, content, start), got)
+    # accumulation over calls adds up
+    twice = oracle.partition_accumulate(P, content, got)
+    assert np.abs(twice - (start + 2 * (ref - start))).max() <= 1e-12
+
+
+def _brute_topk(score, k):
+    """Exhaustive: the k-subset with the largest score multiset, ties broken
+    by the lexicographically smallest index set."""
+    best, best_key = None, None
+    n = len(score)
+    for comb in itertools.combinations(range(n), k):
+        key = (sorted((score[i] for i in comb), reverse=True), [-i for i in comb])
+        if best is None or key > best_key:
+            best, best_key = comb, key
+    return list(best)
+
+
+def test_partition_select_brute_force_tiny():
+    for trial in range(60):
+        n = int(rng.integers(1, 11))
+        k = int(rng.integers(0, n + 1))
+        # integer-valued scores to force ties at the threshold
+        score = rng.integers(0, 4, size=n).astype(np.float64)
+        idx_s, idx_c, _ = oracle.partition_select(score, k)
+        assert list(idx_s) == _brute_topk(list(score), k)
+        assert sorted(list(idx_s) + list(idx_c)) == list(range(n))
+        assert list(idx_c) == sorted(idx_c)
+
+
+def test_partition_select_against_python_sort():
+    for n in (37, 256):
+        for dup in (False, True):
+            score = rng.random(n)
+            if dup:
+                score = np.round(score * 8) / 8
+            for k in (0, 1, n // 4, n // 2, n - 1, n):
+                order = sorted(range(n), key=lambda i: (-score[i], i))
+                idx_s, idx_c, s = oracle.partition_select(score, k)
+                assert list(idx_s) == sorted(order[:k])
+                assert list(idx_c) == sorted(order[k:])
+                lo, hi = score.min(), score.max()
+                assert np.array_equal(s, ((score - lo) / (hi - lo)).astype(np.float32))
+
+
+def test_partition_hand_fixture():
+    for ln in _lines("partition_hand.txt"):
+        kk, sc, exp_s, exp_sv = [x.strip() for x in ln.split("|")]
+        score = np.array([float(x) for x in sc.split()])
+        exp_idx = [] if exp_s == "-" else [int(x) for x in exp_s.split()]
+        idx_s, idx_c, s = oracle.partition_select(score, int(kk))
+        assert list(idx_s) == exp_idx, ln
+        assert np.array_equal(s, np.array([float(x) for x in exp_sv.split()], dtype=np.float32)), ln
+
+
+def test_partition_s_is_minmax_and_affine_invariant():
+    score = rng.random(100) * 3 + 1
+    idx_s, _, s = oracle.partition_select(score, 30)
+    assert s[np.argmax(score)] == 1.0 and s[np.argmin(score)] == 0.0
+    assert np.all((s >= 0) & (s <= 1))
+    idx2, _, s2 = oracle.partition_select(score * 2.5 + 7.0, 30)
+    assert np.array_equal(idx_s, idx2)
+    assert np.abs(s - s2).max() <= 1e-6
+    with pytest.raises(oracle.OracleError):
+        oracle.partition_select(np.array([1.0, np.nan]), 1)
+
+
+# ---------------------------------------------------------------------------
+# Mask elision (C5): SAFE-DiT summary 방법론 1.
+# ---------------------------------------------------------------------------
+def test_mask_criterion_hand_fixture():
+    rows, expect = [], []
+    for ln in _lines("mask_rows_hand.txt"):
+        e, vals = ln.split("|")
+        expect.append(int(e))
+        rows.append([float(x) for x in vals.split()])
+    m = np.array(rows)
+    verdict, flags = oracle.mask_row_constant(m)
+    assert list(flags) == expect
+    assert verdict == 0
+    good = m[np.array(expect) == 1]
+    assert oracle.mask_row_constant(good)[0] == 1
+
+
+def test_mask_criterion_dtypes_and_bool():
+    # bf16 and fp16 row-constant masks widen exactly
+    c = torch.tensor(rng.uniform(-4, 4, size=(6, 1))).expand(6, 9)
+    for dt in (torch.bfloat16, torch.float16, torch.float32):
+        v, f = oracle.mask_row_constant(c.to(dt).contiguous())
+        assert v == 1 and f.all()
+    bm = torch.ones((3, 4, 10), dtype=torch.bool)
+    v, f = oracle.mask_row_constant(bm)
+    assert v == 1 and f.shape == (3, 4) and f.all()
+    bm[1, 2, 7] = False
+    v, f = oracle.mask_row_constant(bm)
+    assert v == 0 and f[1, 2] == 0 and f.sum() == 11
+    v, f = oracle.mask_row_constant(torch.zeros((1, 5), dtype=torch.bool))
+    assert v == 0  # all False: fully masked, not a shift
+
+
+# ---------------------------------------------------------------------------
+# Scatter / gather (C7): SAFE-DiT summary 방법론 3 (cached context state).
+# ---------------------------------------------------------------------------
+def test_scatter_gather_identities():
+    N, d = 50, 6
+    state = rng.standard_normal((N, d)).astype(np.float32)
+    fresh = rng.standard_normal((N, d)).astype(np.float32)
+    idx = np.sort(rng.choice(N, size=17, replace=False)).astype(np.int32)
+    # gather o scatter = id on S
+    merged = oracle.scatter_rows(fresh[idx], state, idx)
+    assert np.array_equal(oracle.gather_rows(merged, idx), fresh[idx])
+    # S rows from fresh, C rows from the cache
+    expect = state.copy()
+    expect[idx] = fresh[idx]
+    assert np.array_equal(merged, expect)
+    cidx = np.setdiff1d(np.arange(N), idx).astype(np.int32)
+    assert np.array_equal(oracle.gather_rows(merged, cidx), state[cidx])
+    with pytest.raises(oracle.OracleError):
+        oracle.scatter_rows(fresh[:2], state, np.array([3, 3], dtype=np.int32))
+    with pytest.raises(oracle.OracleError):
+        oracle.scatter_rows(fresh[:1], state, np.array([N], dtype=np.int32))
+    with pytest.raises(oracle.OracleError):
+        oracle.gather_rows(state, np.array([-1], dtype=np.int32))
+
+
+# ---------------------------------------------------------------------------
+# SW-CFG (C8): SAFE-DiT summary 방법론 4; AccelAes B.2 spatial CFG.
+# ---------------------------------------------------------------------------
+def test_sw_cfg_hand_fixture():
+    rows = np.array([[float(x) for x in ln.split()] for ln in _lines("sw_cfg_hand.txt")])
+    s, c, u, g, out = rows.T
+    got = oracle.sw_cfg(c[:, None], u[:, None], s, 3.0, 5.0)
+    assert np.array_equal(got[:, 0], out)
+
+
+def test_sw_cfg_special_cases():
+    N, F = 31, 16
+    c = rng.standard_normal((N, F)).astype(np.float32)
+    u = rng.standard_normal((N, F)).astype(np.float32)
+    s = rng.random(N).astype(np.float32)
+    assert np.abs(oracle.sw_cfg(c, u, s, 1.0, 1.0) - c).max() <= 1e-15
+    assert np.array_equal(oracle.sw_cfg(c, u, s, 0.0, 0.0), u.astype(np.float64))
+    sb = (rng.random(N) < 0.5).astype(np.float32)  # AccelAes binary focus map
+    got = oracle.sw_cfg(c, u, sb, 2.0, 7.5)
+    gam = np.where(sb > 0, 7.5, 2.0)[:, None]
+    assert np.abs(got - (u + gam * (c.astype(np.float64) - u))).max() <= 1e-14
