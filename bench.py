@@ -1,0 +1,443 @@
+"""Benchmark of the mask-free spatially adaptive DiT attention path on B200.
+
+One step = one denoising trajectory of the 2560^2-equivalent workload
+(B=2 cond/uncond, H=24, N=25600 image tokens, d=96, L=256 text tokens with 128
+valid, |S| = 0.3 N = 7680): 10 denoising steps with dense anchors at t = 0, 5;
+t = 0 is also the PCSP warm-up (cross-attention probabilities -> score), the
+S/C split follows it, the image mask is checked once, every SRSU step
+scatters the fresh S-row K/V into the cached state and runs subset attention
+with the output scattered into O_state, and every step ends with the
+guidance combine.  Every row of the hot path runs in libsafedit.so kernels.
+
+value = SRSU subset-attention TFLOP/s (4 k N d B H flop per call) over all SRSU
+launches of the timed steps, timed with CUDA events on the launching stream;
+whole-job aggregate over ranks (sum of flop / max of per-rank time).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+(for N > 1 launch under torchrun; each rank runs its own independent replica).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from spatially_adaptive_dit_b200 import workloads as wl  # noqa: E402
+
+METRIC = "SRSU subset-attention TFLOP/s & ms at N=25600,|S|=0.3N; partition/CFG HBM GB/s"
+W = wl.W2560
+WORKLOAD = ("2560^2-equivalent: B=2 (cond/uncond), H=24, N=25600 (160x160), d=96, L=256 (128 valid), "
+            "|S|=0.3N=7680, 10-step trajectory with anchors at t=0,5 (t=0 = PCSP warm-up)")
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        try:
+            self.dev = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.dev = str(device_index)
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_dev{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in open(self.path):
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        busy = [x for x in sm if x > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+class Trajectory:
+    """Device-resident buffers and the launch sequence of one trajectory."""
+
+    def __init__(self, w, dev, seed_step=0):
+        from spatially_adaptive_dit_b200 import safedit as sd
+        self.sd, self.w, self.dev = sd, w, dev
+        B, H, N, d, L, k = w.B, w.H, w.N, w.d, w.L, w.k
+        self.k = k
+        self.q, self.k_full, self.v_full = wl.qkv(w, step=seed_step, device=dev)
+        self.k_s, self.v_s = wl.fresh_sensitive_kv(w, k, step=seed_step, device=dev)
+        self.k_state = torch.empty_like(self.k_full)
+        self.v_state = torch.empty_like(self.v_full)
+        self.k_state.copy_(self.k_full)
+        self.v_state.copy_(self.v_full)
+        self.o_state = torch.zeros_like(self.q)
+        self.q_img, self.k_txt, self.valid, self.content = wl.text(w, step=seed_step, device=dev)
+        self.P = torch.empty(H, N, L, device=dev)
+        self.score = torch.zeros(N, dtype=torch.float64, device=dev)
+        self.idx_s = torch.empty(k, dtype=torch.int32, device=dev)
+        self.idx_c = torch.empty(N - k, dtype=torch.int32, device=dev)
+        self.s = torch.zeros(N, device=dev)
+        # Image self-attention mask as the backbone passes it: an all-valid key
+        # mask broadcast over queries ([B,1,1,N] -> [B,1,N,N]).
+        self.mask = torch.zeros(B, 1, 1, N, dtype=torch.bfloat16, device=dev).expand(B, 1, N, N)
+        self.verdict = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.eps_c, self.eps_u = wl.cfg_preds(w, step=seed_step, device=dev)
+        self.cfg_out = torch.empty_like(self.eps_c)
+        self.flop_srsu = 4.0 * k * N * d * B * H
+        self.flop_dense = 4.0 * N * N * d * B * H
+        self.bytes = {
+            "cross_attn_probs": H * N * L * 4 + H * N * d * 2 + H * L * d * 2,
+            "partition_accumulate": H * N * L * 4 + N * 16 + L,
+            "scatter_state": 2 * (2 * B * H * k * d * 2) + 4 * k,
+            "sw_cfg": 3 * N * w.F * 4 + 4 * N,
+        }
+
+    def run(self, stream, ev=None):
+        """Enqueue one trajectory on `stream`.  ev: dict name -> list to which
+        (start, end) CUDA events of each launch are appended."""
+        sd, w = self.sd, self.w
+
+        def timed(name, fn):
+            if ev is None:
+                fn()
+                return
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ev.setdefault(name, []).append((a, b))
+
+        self.score.zero_()
+        for t in range(w.steps):
+            anchor = (t % w.period == 0)
+            if t < w.warmup:  # PCSP warm-up on the cond branch
+                timed("cross_attn_probs", lambda: sd.safedit_cross_attn_probs(
+                    self.q_img, self.k_txt, self.valid, 0, 0.0, self.P, stream))
+                timed("partition_accumulate", lambda: sd.safedit_partition_accumulate(
+                    self.P, self.content, self.score, stream))
+            if t == w.warmup - 1:
+                timed("partition_finalize", lambda: sd.safedit_partition_finalize(
+                    self.score, w.N, self.k, self.idx_s, self.idx_c, self.s, stream))
+            if t == 0:
+                timed("mask_is_row_constant", lambda: sd.safedit_mask_is_row_constant(
+                    self.mask, self.verdict, None, stream))
+            if anchor:
+                # CAR: fresh K/V become the cached state (buffer swap), dense refresh of all rows
+                self.k_state, self.k_full = self.k_full, self.k_state
+                self.v_state, self.v_full = self.v_full, self.v_state
+                timed("attn_dense_anchor", lambda: sd.safedit_attn_subset(
+                    self.q, self.k_state, self.v_state, None, 0, None, None, 0.0, self.o_state, 0,
+                    stream))
+            else:
+                timed("scatter_state", lambda: sd.safedit_scatter_state(
+                    [self.k_s, self.v_s], [self.k_state, self.v_state], self.idx_s, self.k, stream))
+                timed("attn_subset_srsu", lambda: sd.safedit_attn_subset(
+                    self.q, self.k_state, self.v_state, self.idx_s, self.k, None, None, 0.0,
+                    self.o_state, 1, stream))
+            g_ctx = w.gamma_ctx
+            g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx  # global CFG before the split
+            timed("sw_cfg", lambda: sd.safedit_sw_cfg(self.eps_c, self.eps_u, self.s, g_ctx, g_sens,
+                                                       self.cfg_out, stream))
+
+
+def run_ours(args):
+    ws, rank, local = _dist()
+    if ws > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from spatially_adaptive_dit_b200 import safedit as sd
+    tr = Trajectory(W, dev, seed_step=1000 * rank)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            tr.run(stream)
+    stream.synchronize()
+    assert sd.safedit_get_device_status(stream) == 0
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev = {}
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    n0 = sd.safedit_kernel_launch_count()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            tr.run(stream, ev)
+    t1.record(stream)
+    t1.synchronize()
+    torch.cuda.synchronize()
+    launches = sd.safedit_kernel_launch_count() - n0
+    if ws > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    status = sd.safedit_get_device_status(stream)
+    total_ms = t0.elapsed_time(t1)
+    per = {n: [a.elapsed_time(b) for a, b in lst] for n, lst in ev.items()}
+    srsu_ms = sum(per["attn_subset_srsu"])
+    n_srsu = len(per["attn_subset_srsu"])
+    stats = torch.tensor([total_ms, srsu_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
+    total_ms, srsu_ms = float(stats[0]), float(stats[1])
+
+    # ---- end to end through the public API with host buffers (pinned)
+    e2e = run_e2e(tr, stream, args)
+    if ws > 1:
+        e2e_t = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
+        e2e["ms"] = float(e2e_t[0])
+
+    if rank == 0:
+        hbm, bf16_burst, bf16_sust, src = _peaks()
+        flop_total = tr.flop_srsu * n_srsu * ws
+        value = flop_total / (srsu_ms * 1e-3) / 1e12
+        srsu_call_ms = srsu_ms / n_srsu
+        achieved = tr.flop_srsu / (srsu_call_ms * 1e-3) / 1e12
+        kern = {}
+        for n, v in per.items():
+            m = statistics.mean(v)
+            entry = {"ms_mean": round(m, 4), "calls_per_step": len(v) // args.steps}
+            if n in tr.bytes:
+                gbs = tr.bytes[n] / (m * 1e-3) / 1e9
+                entry.update({"gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)})
+            if n == "attn_dense_anchor":
+                entry["tflops"] = round(tr.flop_dense / (m * 1e-3) / 1e12, 1)
+            if n == "attn_subset_srsu":
+                entry["tflops"] = round(tr.flop_srsu / (m * 1e-3) / 1e12, 1)
+            kern[n] = entry
+        traffic = _ncu_traffic()
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": W.B * ws, "seq_len": W.N,
+                       "parallelism": f"replicas x{ws} (independent trajectories, no collective)",
+                       "l2": "inputs larger than L2 (Q/K/V/state 236 MB each), no flush needed",
+                       "srsu_calls_per_step": n_srsu // args.steps,
+                       "srsu_ms_per_call": round(srsu_call_ms, 4)},
+            "kernels": kern,
+            "roofline": {"kernel": "attn_subset (SRSU)", "bound": "tensor", "achieved": round(achieved, 1),
+                         "peak": bf16_sust, "peak_kind": f"bf16_tflops_sustained ({src})",
+                         "unit": "TFLOP/s", "frac": round(achieved / bf16_sust, 4), "traffic": traffic},
+            "gpu_launches": launches,
+            "device_status": status,
+            "e2e": {"value": round(tr.flop_srsu * n_srsu / args.steps * ws / (e2e["ms"] * 1e-3) / 1e12, 3),
+                    "unit": "TFLOP/s", "ms_per_step": round(e2e["ms"], 3),
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+            "clocks": clk,
+        }
+        if ws == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def _ncu_traffic():
+    """dram bytes per SRSU launch from the committed ncu summary, if present and current."""
+    p = os.path.join(ROOT, "profiles", "attn_subset_srsu_2560.traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("bytes_per_launch")
+    except Exception:
+        return None
+
+
+def run_e2e(tr, stream, args):
+    """Same trajectory, with every denoising step's inputs copied from pinned
+    host memory and each step's guided prediction copied back, inside the
+    timed region."""
+    w = tr.w
+    host = {}
+    for name in ("q", "k_s", "v_s", "k_full", "v_full", "q_img", "k_txt", "eps_c", "eps_u"):
+        t = getattr(tr, name)
+        host[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        host[name].copy_(t)
+    out_h = torch.empty(tr.cfg_out.shape, dtype=tr.cfg_out.dtype, pin_memory=True)
+    h2d = d2h = 0
+
+    def step(count):
+        nonlocal h2d, d2h
+        sd = tr.sd
+        tr.score.zero_()
+        for t in range(w.steps):
+            anchor = (t % w.period == 0)
+            names = ["q", "eps_c", "eps_u"] + (["q_img", "k_txt"] if t < w.warmup else []) + \
+                (["k_full", "v_full"] if anchor else ["k_s", "v_s"])
+            for n in names:
+                dst = getattr(tr, n)
+                dst.copy_(host[n], non_blocking=True)
+                if count:
+                    h2d += host[n].numel() * host[n].element_size()
+            if t < w.warmup:
+                sd.safedit_cross_attn_probs(tr.q_img, tr.k_txt, tr.valid, 0, 0.0, tr.P, stream)
+                sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream)
+            if t == w.warmup - 1:
+                sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s, stream)
+            if t == 0:
+                sd.safedit_mask_is_row_constant(tr.mask, tr.verdict, None, stream)
+            if anchor:
+                tr.k_state, tr.k_full = tr.k_full, tr.k_state
+                tr.v_state, tr.v_full = tr.v_full, tr.v_state
+                sd.safedit_attn_subset(tr.q, tr.k_state, tr.v_state, None, 0, None, None, 0.0,
+                                       tr.o_state, 0, stream)
+            else:
+                sd.safedit_scatter_state([tr.k_s, tr.v_s], [tr.k_state, tr.v_state], tr.idx_s, tr.k,
+                                         stream)
+                sd.safedit_attn_subset(tr.q, tr.k_state, tr.v_state, tr.idx_s, tr.k, None, None, 0.0,
+                                       tr.o_state, 1, stream)
+            g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx
+            sd.safedit_sw_cfg(tr.eps_c, tr.eps_u, tr.s, w.gamma_ctx, g_sens, tr.cfg_out, stream)
+            out_h.copy_(tr.cfg_out, non_blocking=True)
+            if count:
+                d2h += out_h.numel() * out_h.element_size()
+
+    with torch.cuda.stream(stream):
+        step(False)
+        stream.synchronize()
+        n = max(1, min(args.steps, 5))
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(n):
+            step(True)
+        stream.synchronize()
+        ms = (time.perf_counter() - t0) * 1e3 / n
+    return {"ms": ms, "h2d": h2d // n, "d2h": d2h // n}
+
+
+def cpu_baseline(seconds=12.0, rows=None):
+    """The fp64 oracle, as it stands, on the host cores: SRSU attention rows of
+    one (b,h) slice of the workload over all N keys.  Reported in the same
+    unit (TFLOP/s of the SRSU attention)."""
+    import numpy as np
+    import oracle
+    w = W
+    g = torch.Generator().manual_seed(4321)
+    q = torch.randn(1024, w.d, generator=g).to(torch.bfloat16).double().numpy()
+    k = torch.randn(w.N, w.d, generator=g).to(torch.bfloat16).double().numpy()
+    v = torch.randn(w.N, w.d, generator=g).to(torch.bfloat16).double().numpy()
+    n = rows or 16
+    dt = 0.0
+    while True:
+        idx = np.arange(n, dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.attn_subset(q, k, v, idx)
+        dt = time.perf_counter() - t0
+        if rows or dt >= seconds * 0.5 or n >= 1024:
+            break
+        n = min(1024, max(n * 2, int(n * seconds / max(dt, 1e-3) * 0.9)))
+    flop = 4.0 * n * w.N * w.d
+    return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} SRSU query rows of one (b,h) slice over all N={w.N} keys, d={w.d}, fp64 "
+                      f"({dt:.1f} s)"}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    import oracle  # noqa: F401
+    vals = []
+    # calibrate the sample once, then time K steps of that fixed sample
+    cal = cpu_baseline(seconds=4.0)
+    n_rows = int(cal["sample"].split()[0])
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(rows=n_rows)
+        if i >= args.warmup:
+            vals.append(r["value"])
+    value = statistics.mean(vals)
+    ms_per_step = 4.0 * n_rows * W.N * W.d / (value * 1e12) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": W.B, "seq_len": W.N,
+                       "parallelism": "host cores (OpenMP)"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": r["cores"], "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

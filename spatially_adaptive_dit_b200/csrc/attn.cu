@@ -1,0 +1,571 @@
+// attn.cu -- SRSU subset attention and CAR dense anchor on sm_100a.
+//
+// SAFE-DiT summary (gist.science 2606.29360), 방법론 3 / Italian page
+// Metodologia 3: on a non-anchor step only the sensitive query rows are
+// updated, and they attend over the global key/value set (fresh sensitive
+// states plus cached context states); an anchor step refreshes every row.
+// AccelAes summary (gist.science 2603.12575), B.2 SkipSparse: queries only on
+// focus tokens, keys and values from the whole image.
+//
+//   o_r = sum_j softmax_j(scale q_{idx[r]} . k_j + pad_j + bias_{idx[r],j}) v_j
+//
+// Design (one CTA per SM, 320 threads = 10 warps):
+//   * 2 query tiles of 128 rows (256 rows per CTA).  The softmax warpgroup of
+//     tile t (warps 4t..4t+3) gathers its rows q[idx[r]] with 16-byte loads
+//     straight into the swizzled K-major shared-memory layout the tensor core
+//     reads (the indexed gather replaces a copy of Q_S).
+//   * warp 8 streams K and V tiles (128 keys) through an NS-stage TMA ring.
+//   * warp 9 issues tcgen05.mma: S_t = Q_t K_j^T into TMEM (fp32, 128 cols per
+//     tile) and O_t += P_t V_j with P_t read back from TMEM (the bf16 softmax
+//     probabilities overwrite S_t in place), so P never touches shared memory.
+//   * softmax: thread = query row = TMEM lane.  Online softmax in base 2 with
+//     a lazy rescale (the running max only moves when it grows by more than
+//     2^8, which is exact after the final division by the row sum).
+// Every mbarrier wait is bounded; an expired wait raises the CTA's abort
+// flag, drains in-flight TMA loads and MMAs, frees TMEM and returns.
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace sd {
+
+template <int D>
+struct AttnCfg {
+  static constexpr int BM = 128;                       // query rows per tile
+  static constexpr int BN = 128;                       // keys per tile
+  static constexpr int CH = (D % 64 == 0) ? 64 : 32;   // elements per swizzle chunk row
+  static constexpr int NCH = D / CH;                   // chunks per row
+  static constexpr int ROWB = CH * 2;                  // bytes per chunk row
+  static constexpr uint32_t LAYOUT = (CH == 64) ? 2u : 4u;  // 128B / 64B swizzle
+  static constexpr int CHUNK_BYTES = 128 * ROWB;       // one chunk of a 128-row tile
+  static constexpr int TILE_BYTES = NCH * CHUNK_BYTES; // 128 rows x D bf16
+  static constexpr int NS = (D == 64) ? 4 : (D == 96 ? 3 : 2);  // K/V ring depth
+  static constexpr int UNITS = D * 2 / 16;             // 16-byte units per row
+  static constexpr int SMEM_TILES = 2 + 2 * NS;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES * TILE_BYTES + BAR_BYTES;
+  static_assert(D == 64 || D == 96 || D == 128, "head dim");
+  static_assert(256 + 2 * D <= 512, "TMEM columns");
+};
+
+struct AttnParams {
+  const __nv_bfloat16* q;
+  int64_t q_sb, q_sh, q_sr;  // element strides
+  const int* idx;            // nullable
+  int n_rows, Nq, Nk, H;
+  float scale_log2;          // scale * log2(e)
+  const float* pad;          // nullable, [B, Nk]
+  int64_t pad_sb;
+  const void* bias;          // nullable
+  int bias_f32;
+  int64_t bias_sb, bias_sh, bias_sq;
+  __nv_bfloat16* out;
+  int64_t o_sb, o_sh, o_sr;
+  int out_scattered;
+  int* status;
+  uint64_t wait_limit;
+};
+
+constexpr int kAttnThreads = 320;
+constexpr uint64_t kDrainNs = 1000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+__device__ __forceinline__ uint32_t swizzle_off(uint32_t off, uint32_t layout) {
+  return layout == 2u ? (off ^ (((off >> 7) & 7u) << 4)) : (off ^ (((off >> 7) & 3u) << 4));
+}
+
+template <int D, bool PAD, bool BIAS>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_subset_kernel(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase;                               // 2 tiles
+  const uint32_t sK = sbase + 2 * C::TILE_BYTES;           // NS tiles
+  const uint32_t sV = sK + C::NS * C::TILE_BYTES;          // NS tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_TILES * C::TILE_BYTES);
+  // barrier slots
+  const uint32_t b0 = smem_u32(bars);
+  auto BAR = [&](int i) { return b0 + 8u * uint32_t(i); };
+  const int Q_FULL = 0, K_FULL = 2, K_EMPTY = K_FULL + C::NS, V_FULL = K_EMPTY + C::NS,
+            V_EMPTY = V_FULL + C::NS, S_FULL = V_EMPTY + C::NS, P_FULL = S_FULL + 2,
+            O_FULL = P_FULL + 2, DRAIN = O_FULL + 1, NBARS = DRAIN + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int row0 = blockIdx.x * 256;
+  const int nk = (p.Nk + C::BN - 1) / C::BN;
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(BAR(Q_FULL + t), 128);
+      mbar_init(BAR(S_FULL + t), 1);
+      mbar_init(BAR(P_FULL + t), 128);
+    }
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(BAR(K_FULL + s), 1);
+      mbar_init(BAR(K_EMPTY + s), 1);
+      mbar_init(BAR(V_FULL + s), 1);
+      mbar_init(BAR(V_EMPTY + s), 1);
+    }
+    mbar_init(BAR(O_FULL), 1);
+    mbar_init(BAR(DRAIN), 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit};
+
+  if (warp < 8) {
+    // ================================================== softmax warpgroups
+    const int t = warp >> 2;            // query tile
+    const int wr = warp & 3;            // TMEM lane quarter
+    const int tid = threadIdx.x & 127;  // thread within the warpgroup
+    const int tile_row0 = row0 + t * 128;
+    // ---- indexed gather of the tile's query rows into swizzled smem
+    {
+      const uint32_t qs = sQ + t * C::TILE_BYTES;
+      const __nv_bfloat16* qbh = p.q + b * p.q_sb + h * p.q_sh;
+      for (int u = tid; u < 128 * C::UNITS; u += 128) {
+        const int rr = u / C::UNITS, cu = u - rr * C::UNITS;
+        const int gr = tile_row0 + rr;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (gr < p.n_rows) {
+          const int qi = p.idx ? __ldg(p.idx + gr) : gr;
+          if (qi >= 0 && qi < p.Nq)
+            val = __ldg(reinterpret_cast<const uint4*>(qbh + int64_t(qi) * p.q_sr) + cu);
+          else if (cu == 0)
+            set_status(p.status, SAFEDIT_ERR_INDEX);
+        }
+        constexpr int UPC = C::ROWB / 16;  // units per chunk row
+        const int chunk = cu / UPC, cin = cu - chunk * UPC;
+        const uint32_t off = uint32_t(chunk * C::CHUNK_BYTES) +
+                             swizzle_off(uint32_t(rr * C::ROWB + cin * 16), C::LAYOUT);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(qs + off), "r"(val.x),
+                     "r"(val.y), "r"(val.z), "r"(val.w)
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(Q_FULL + t));
+    }
+
+    const uint32_t lane_base = uint32_t(wr * 32) << 16;
+    const uint32_t tS = tmem + uint32_t(t * 128) + lane_base;
+    const uint32_t tO = tmem + 256u + uint32_t(t * D) + lane_base;
+    const int my_row = tile_row0 + wr * 32 + lane;
+    int my_q = -1;  // query index of this thread's row, -1 if none
+    if (my_row < p.n_rows) {
+      my_q = p.idx ? __ldg(p.idx + my_row) : my_row;
+      if (my_q < 0 || my_q >= p.Nq) my_q = -1;
+    }
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nk; ++j) {
+      if (!wait_warp(BAR(S_FULL + t), uint32_t(j & 1), ctl)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float x[128];
+      {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(tS + uint32_t(c * 32), r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]) * sl2;
+        }
+      }
+      const int key0 = j * C::BN;
+      if (PAD) {
+        const float* pr = p.pad + b * p.pad_sb + key0;
+        const int lim = p.Nk - key0;
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          if (c + 4 <= lim) {
+            const float4 pv = __ldg(reinterpret_cast<const float4*>(pr + c));
+            x[c] = fmaf(pv.x, kLog2e, x[c]);
+            x[c + 1] = fmaf(pv.y, kLog2e, x[c + 1]);
+            x[c + 2] = fmaf(pv.z, kLog2e, x[c + 2]);
+            x[c + 3] = fmaf(pv.w, kLog2e, x[c + 3]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (c + e < lim) x[c + e] = fmaf(__ldg(pr + c + e), kLog2e, x[c + e]);
+          }
+        }
+      }
+      if (BIAS && my_q >= 0) {
+        const int lim = p.Nk - key0;
+        if (p.bias_f32) {
+          const float* br = static_cast<const float*>(p.bias) + b * p.bias_sb + h * p.bias_sh +
+                            int64_t(my_q) * p.bias_sq + key0;
+#pragma unroll
+          for (int c = 0; c < 128; c += 4) {
+            if (c + 4 <= lim) {
+              const float4 bv = __ldg(reinterpret_cast<const float4*>(br + c));
+              x[c] = fmaf(bv.x, kLog2e, x[c]);
+              x[c + 1] = fmaf(bv.y, kLog2e, x[c + 1]);
+              x[c + 2] = fmaf(bv.z, kLog2e, x[c + 2]);
+              x[c + 3] = fmaf(bv.w, kLog2e, x[c + 3]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (c + e < lim) x[c + e] = fmaf(__ldg(br + c + e), kLog2e, x[c + e]);
+            }
+          }
+        } else {
+          const __nv_bfloat16* br = static_cast<const __nv_bfloat16*>(p.bias) + b * p.bias_sb +
+                                    h * p.bias_sh + int64_t(my_q) * p.bias_sq + key0;
+#pragma unroll
+          for (int c = 0; c < 128; c += 8) {
+            if (c + 8 <= lim) {
+              const uint4 w = __ldg(reinterpret_cast<const uint4*>(br + c));
+              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                x[c + 2 * e] = fmaf(__uint_as_float(ws[e] << 16), kLog2e, x[c + 2 * e]);
+                x[c + 2 * e + 1] =
+                    fmaf(__uint_as_float(ws[e] & 0xFFFF0000u), kLog2e, x[c + 2 * e + 1]);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                if (c + e < lim) x[c + e] = fmaf(__bfloat162float(br[c + e]), kLog2e, x[c + e]);
+            }
+          }
+        }
+      }
+      if (key0 + C::BN > p.Nk) {  // ragged last key tile
+        const int lim = p.Nk - key0;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) x[c] = -INFINITY;
+      }
+      float mt = x[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mt = fmaxf(mt, x[c]);
+      // lazy rescale
+      bool need_o = false;
+      float alpha = 1.f;
+      if (mt > m_run + kRescaleThreshold) {
+        alpha = ex2_approx(m_run - mt);  // 0 when m_run = -inf
+        l_run *= alpha;
+        m_run = mt;
+        need_o = (j > 0);
+      }
+      if (__any_sync(0xffffffffu, need_o)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + uint32_t(c * 32), r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(tO + uint32_t(c * 32), r);
+        }
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2_approx(x[c * 32 + 2 * e] - m_use);
+          const float p1 = ex2_approx(x[c * 32 + 2 * e + 1] - m_use);
+          rs += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + uint32_t(c * 16), pk);
+      }
+      l_run += rs;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(P_FULL + t));
+    }
+    // ---- epilogue: O / l -> bf16 rows
+    if (ok && wait_warp(BAR(O_FULL), 0u, ctl)) {
+      tc_fence_after();
+      const bool live = my_q >= 0;
+      if (live && !(l_run > 0.f)) set_status(p.status, SAFEDIT_ERR_MASKED_ROW);
+      const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      __nv_bfloat16* orow = nullptr;
+      if (live) {
+        const int64_t orow_idx = p.out_scattered ? int64_t(my_q) : int64_t(my_row);
+        orow = p.out + b * p.o_sb + h * p.o_sh + orow_idx * p.o_sr;
+      }
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + uint32_t(c * 32), r);
+        tmem_wait_ld();
+        if (live) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+    }
+  } else if (warp == 8) {
+    // ================================================== TMA producer (K, V)
+    if (lane == 0) {
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < nk; ++j) {
+        const int s = j % C::NS;
+        const uint32_t ph = uint32_t((j / C::NS) & 1);
+        if (!wait_bounded(BAR(K_EMPTY + s), ph ^ 1u, ctl)) break;
+        mbar_arrive_expect_tx(BAR(K_FULL + s), C::TILE_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c)
+          tma_load_4d(sK + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmK, BAR(K_FULL + s), c * C::CH,
+                      j * C::BN, h, b);
+        issued_k = j + 1;
+        if (!wait_bounded(BAR(V_EMPTY + s), ph ^ 1u, ctl)) break;
+        mbar_arrive_expect_tx(BAR(V_FULL + s), C::TILE_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c)
+          tma_load_4d(sV + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmV, BAR(V_FULL + s), c * C::CH,
+                      j * C::BN, h, b);
+        issued_v = j + 1;
+      }
+      if (*abort_flag) {  // drain the loads still in flight before leaving
+        for (int j = (issued_k > C::NS ? issued_k - C::NS : 0); j < issued_k; ++j)
+          wait_drain(BAR(K_FULL + j % C::NS), uint32_t((j / C::NS) & 1), kDrainNs);
+        for (int j = (issued_v > C::NS ? issued_v - C::NS : 0); j < issued_v; ++j)
+          wait_drain(BAR(V_FULL + j % C::NS), uint32_t((j / C::NS) & 1), kDrainNs);
+      }
+    }
+  } else {
+    // ================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t tS0 = tmem, tS1 = tmem + 128u;
+      const uint32_t tO0 = tmem + 256u, tO1 = tmem + 256u + uint32_t(D);
+      constexpr uint32_t SBO = 8u * C::ROWB;
+      auto issue_qk = [&](uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int chunk = (kk * 16) / C::CH;
+          const uint32_t within = uint32_t(((kk * 16) % C::CH) * 2);
+          const uint32_t off = uint32_t(chunk * C::CHUNK_BYTES) + within;
+          mma_ss(d_tmem, smem_desc(q_smem + off, 16u, SBO, C::LAYOUT),
+                 smem_desc(k_smem + off, 16u, SBO, C::LAYOUT), idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          const uint64_t bdesc =
+              smem_desc(v_smem + uint32_t(kk * 16 * C::ROWB), uint32_t(C::CHUNK_BYTES), SBO, C::LAYOUT);
+          mma_ts(d_tmem, p_tmem + uint32_t(kk * 8), bdesc, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = wait_bounded(BAR(Q_FULL + 0), 0u, ctl) && wait_bounded(BAR(Q_FULL + 1), 0u, ctl) &&
+                wait_bounded(BAR(K_FULL + 0), 0u, ctl);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(tS0, sQ, sK);
+        tc_commit(BAR(S_FULL + 0));
+        issue_qk(tS1, sQ + C::TILE_BYTES, sK);
+        tc_commit(BAR(S_FULL + 1));
+        tc_commit(BAR(K_EMPTY + 0));
+      }
+      for (int j = 0; ok && j < nk; ++j) {
+        const int s = j % C::NS;
+        const uint32_t ph = uint32_t((j / C::NS) & 1);
+        const bool more = (j + 1 < nk);
+        const int s1 = (j + 1) % C::NS;
+        const uint32_t ph1 = uint32_t(((j + 1) / C::NS) & 1);
+        if (!(ok = wait_bounded(BAR(V_FULL + s), ph, ctl))) break;
+        if (!(ok = wait_bounded(BAR(P_FULL + 0), uint32_t(j & 1), ctl))) break;
+        tc_fence_after();
+        issue_pv(tO0, tS0, sV + s * C::TILE_BYTES, j > 0);
+        if (more) {
+          if (!(ok = wait_bounded(BAR(K_FULL + s1), ph1, ctl))) break;
+          tc_fence_after();
+          issue_qk(tS0, sQ, sK + s1 * C::TILE_BYTES);
+          tc_commit(BAR(S_FULL + 0));
+        }
+        if (!(ok = wait_bounded(BAR(P_FULL + 1), uint32_t(j & 1), ctl))) break;
+        tc_fence_after();
+        issue_pv(tO1, tS1, sV + s * C::TILE_BYTES, j > 0);
+        tc_commit(BAR(V_EMPTY + s));
+        if (more) {
+          issue_qk(tS1, sQ + C::TILE_BYTES, sK + s1 * C::TILE_BYTES);
+          tc_commit(BAR(S_FULL + 1));
+          tc_commit(BAR(K_EMPTY + s1));
+        }
+      }
+      if (ok) {
+        tc_commit(BAR(O_FULL));
+      } else {  // wait for every MMA already issued before TMEM is freed
+        tc_commit(BAR(DRAIN));
+        wait_drain(BAR(DRAIN), 0u, kDrainNs);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool PAD, bool BIAS>
+static safedit_status launch_attn(const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                  const AttnParams& p, int B, cudaStream_t stream) {
+  using C = AttnCfg<D>;
+  auto kern = attn_subset_kernel<D, PAD, BIAS>;
+  safedit_status st = set_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES);
+  if (st != SAFEDIT_OK) return st;
+  dim3 grid((p.n_rows + 255) / 256, B * p.H);
+  kern<<<grid, kAttnThreads, C::SMEM_BYTES, stream>>>(tmK, tmV, p);
+  return after_launch(1);
+}
+
+template <int D>
+static safedit_status dispatch_attn(const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                    const AttnParams& p, int B, cudaStream_t s) {
+  const bool pad = p.pad != nullptr, bias = p.bias != nullptr;
+  if (pad && bias) return launch_attn<D, true, true>(tmK, tmV, p, B, s);
+  if (pad) return launch_attn<D, true, false>(tmK, tmV, p, B, s);
+  if (bias) return launch_attn<D, false, true>(tmK, tmV, p, B, s);
+  return launch_attn<D, false, false>(tmK, tmV, p, B, s);
+}
+
+static safedit_status check_bhnd(const safedit_tensor* t) {
+  safedit_status st = check_tensor(t, 4);
+  if (st != SAFEDIT_OK) return st;
+  if (t->dtype != SAFEDIT_BF16) return SAFEDIT_ERR_DTYPE;
+  if (t->strides[3] != 1) return SAFEDIT_ERR_ALIGNMENT;
+  for (int i = 0; i < 3; ++i)
+    if (t->strides[i] % 8 != 0 || t->strides[i] < 0) return SAFEDIT_ERR_ALIGNMENT;
+  if (!aligned16(t->data)) return SAFEDIT_ERR_ALIGNMENT;
+  return SAFEDIT_OK;
+}
+
+static safedit_status make_kv_map(CUtensorMap* m, const safedit_tensor* t, int D) {
+  const int ch = (D % 64 == 0) ? 64 : 32;
+  const uint64_t dims[4] = {uint64_t(t->dims[3]), uint64_t(t->dims[2]), uint64_t(t->dims[1]),
+                            uint64_t(t->dims[0])};
+  const uint64_t strides[3] = {uint64_t(t->strides[2]) * 2, uint64_t(t->strides[1]) * 2,
+                               uint64_t(t->strides[0]) * 2};
+  const uint32_t box[4] = {uint32_t(ch), 128u, 1u, 1u};
+  return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t->data, dims, strides, box,
+                     ch == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+}  // namespace sd
+
+using namespace sd;
+
+extern "C" safedit_status safedit_attn_subset(const safedit_tensor* q, const safedit_tensor* k,
+                                              const safedit_tensor* v, const int32_t* d_idx,
+                                              int32_t n_idx, const safedit_tensor* key_pad,
+                                              const safedit_tensor* bias, float scale,
+                                              const safedit_tensor* out, int32_t out_scattered,
+                                              void* stream) {
+  safedit_status st;
+  if ((st = check_bhnd(q)) != SAFEDIT_OK) return st;
+  if ((st = check_bhnd(k)) != SAFEDIT_OK) return st;
+  if ((st = check_bhnd(v)) != SAFEDIT_OK) return st;
+  if ((st = check_bhnd(out)) != SAFEDIT_OK) return st;
+  const int64_t B = q->dims[0], H = q->dims[1], Nq = q->dims[2], D = q->dims[3];
+  const int64_t Nk = k->dims[2];
+  for (const safedit_tensor* t : {k, v})
+    if (t->dims[0] != B || t->dims[1] != H || t->dims[3] != D || t->dims[2] != Nk)
+      return SAFEDIT_ERR_SHAPE;
+  if (D != 64 && D != 96 && D != 128) return SAFEDIT_ERR_UNSUPPORTED;
+  if (Nk < 1 || Nq > INT32_MAX || Nk > INT32_MAX || B * H > 65535) return SAFEDIT_ERR_SHAPE;
+  if (out_scattered != 0 && out_scattered != 1) return SAFEDIT_ERR_INVALID_ARG;
+  if (d_idx && n_idx < 0) return SAFEDIT_ERR_INVALID_ARG;
+  const int64_t n_rows = d_idx ? n_idx : Nq;
+  if (out->dims[0] != B || out->dims[1] != H || out->dims[3] != D) return SAFEDIT_ERR_SHAPE;
+  if (out_scattered ? (out->dims[2] != Nq) : (out->dims[2] != n_rows)) return SAFEDIT_ERR_SHAPE;
+  AttnParams p{};
+  if (key_pad) {
+    if ((st = check_tensor(key_pad, 2)) != SAFEDIT_OK) return st;
+    if (key_pad->dtype != SAFEDIT_F32) return SAFEDIT_ERR_DTYPE;
+    if (key_pad->dims[0] != B || key_pad->dims[1] != Nk) return SAFEDIT_ERR_SHAPE;
+    if (key_pad->strides[1] != 1 || key_pad->strides[0] % 4 != 0 || !aligned16(key_pad->data))
+      return SAFEDIT_ERR_ALIGNMENT;
+    p.pad = static_cast<const float*>(key_pad->data);
+    p.pad_sb = key_pad->strides[0];
+  }
+  if (bias) {
+    if ((st = check_tensor(bias, 4)) != SAFEDIT_OK) return st;
+    if (bias->dtype != SAFEDIT_F32 && bias->dtype != SAFEDIT_BF16) return SAFEDIT_ERR_DTYPE;
+    if (bias->dims[0] != B || (bias->dims[1] != 1 && bias->dims[1] != H) || bias->dims[2] != Nq ||
+        bias->dims[3] != Nk)
+      return SAFEDIT_ERR_SHAPE;
+    const int vecw = bias->dtype == SAFEDIT_F32 ? 4 : 8;
+    if (bias->strides[3] != 1 || bias->strides[2] % vecw != 0 || bias->strides[1] % vecw != 0 ||
+        bias->strides[0] % vecw != 0 || !aligned16(bias->data))
+      return SAFEDIT_ERR_ALIGNMENT;
+    p.bias = bias->data;
+    p.bias_f32 = bias->dtype == SAFEDIT_F32;
+    p.bias_sb = bias->strides[0];
+    p.bias_sh = bias->dims[1] == 1 ? 0 : bias->strides[1];
+    p.bias_sq = bias->strides[2];
+  }
+  if (n_rows == 0 || B * H == 0) return SAFEDIT_OK;
+  p.q = static_cast<const __nv_bfloat16*>(q->data);
+  p.q_sb = q->strides[0];
+  p.q_sh = q->strides[1];
+  p.q_sr = q->strides[2];
+  p.idx = d_idx;
+  p.n_rows = static_cast<int>(n_rows);
+  p.Nq = static_cast<int>(Nq);
+  p.Nk = static_cast<int>(Nk);
+  p.H = static_cast<int>(H);
+  const float sc = (scale > 0.f) ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale_log2 = sc * kLog2e;
+  p.out = static_cast<__nv_bfloat16*>(out->data);
+  p.o_sb = out->strides[0];
+  p.o_sh = out->strides[1];
+  p.o_sr = out->strides[2];
+  p.out_scattered = out_scattered;
+  p.wait_limit = wait_limit_ns();
+  CUtensorMap tmK, tmV;
+  if ((st = make_kv_map(&tmK, k, static_cast<int>(D))) != SAFEDIT_OK) return st;
+  if ((st = make_kv_map(&tmV, v, static_cast<int>(D))) != SAFEDIT_OK) return st;
+  p.status = status_ptr();
+  if (!p.status) return SAFEDIT_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (D) {
+    case 64: return dispatch_attn<64>(tmK, tmV, p, static_cast<int>(B), s);
+    case 96: return dispatch_attn<96>(tmK, tmV, p, static_cast<int>(B), s);
+    default: return dispatch_attn<128>(tmK, tmV, p, static_cast<int>(B), s);
+  }
+}

@@ -1,0 +1,254 @@
+// rows_cfg.cu -- the bandwidth kernels of the state update and the guidance
+// combine:
+//   * scatter_state / gather_rows: indexed row copies of up to four
+//     [B,H,rows,d] tensors in one launch (SAFE-DiT summary, 방법론 3: cached
+//     context states, refreshed sensitive rows), 16-byte vector accesses,
+//     every row a contiguous run so that a warp touches whole lines;
+//   * sw_cfg: gamma_i = gamma_ctx + (gamma_sens - gamma_ctx) s_i and
+//     out = u + gamma_i (c - u) (SAFE-DiT summary, 방법론 4), one fp32 FMA
+//     chain per element on 128-bit loads.
+#include "common.cuh"
+#include "internal.h"
+
+namespace sd {
+
+constexpr int kMaxRowTensors = 4;
+
+struct RowCopyParams {
+  const char* src[kMaxRowTensors];
+  char* dst[kMaxRowTensors];
+  // byte strides of the compact side (b, h, row) and of the indexed side
+  int64_t c_sb[kMaxRowTensors], c_sh[kMaxRowTensors], c_sr[kMaxRowTensors];
+  int64_t x_sb[kMaxRowTensors], x_sh[kMaxRowTensors], x_sr[kMaxRowTensors];
+  int H[kMaxRowTensors], BH[kMaxRowTensors], units[kMaxRowTensors];
+  int rows_per_pass[kMaxRowTensors];
+  int n_idx;       // compact rows
+  int n_rows_x;    // rows of the indexed side
+  const int* idx;
+  int scatter;     // 1: compact -> indexed; 0: indexed -> compact
+  int* status;
+};
+
+constexpr int kRowThreads = 256;
+constexpr int kRowIters = 4;  // independent 16-byte copies in flight per thread
+
+// grid: x = row blocks, y = b*H + h, z = tensor.
+__global__ void __launch_bounds__(kRowThreads) row_copy_kernel(RowCopyParams p) {
+  const int t = blockIdx.z;
+  const int bh = blockIdx.y;
+  if (bh >= p.BH[t]) return;
+  const int U = p.units[t];
+  const int rpp = p.rows_per_pass[t];
+  const int sub = threadIdx.x / U;
+  const int unit = threadIdx.x - sub * U;
+  if (sub >= rpp) return;
+  const int b = bh / p.H[t], h = bh - b * p.H[t];
+  const char* cb_src;
+  char* cb_dst;
+  const int64_t c_off = b * p.c_sb[t] + h * p.c_sh[t] + int64_t(unit) * 16;
+  const int64_t x_off = b * p.x_sb[t] + h * p.x_sh[t] + int64_t(unit) * 16;
+  const int r_base = blockIdx.x * (rpp * kRowIters) + sub;
+
+  uint4 v[kRowIters];
+  int64_t dst_off[kRowIters];
+  bool ok[kRowIters];
+#pragma unroll
+  for (int it = 0; it < kRowIters; ++it) {
+    const int r = r_base + it * rpp;
+    ok[it] = r < p.n_idx;
+    if (!ok[it]) continue;
+    const int i = __ldg(p.idx + r);
+    if (i < 0 || i >= p.n_rows_x) {
+      set_status(p.status, SAFEDIT_ERR_INDEX);
+      ok[it] = false;
+      continue;
+    }
+    int64_t s_off, d_off;
+    if (p.scatter) {
+      s_off = c_off + int64_t(r) * p.c_sr[t];
+      d_off = x_off + int64_t(i) * p.x_sr[t];
+    } else {
+      s_off = x_off + int64_t(i) * p.x_sr[t];
+      d_off = c_off + int64_t(r) * p.c_sr[t];
+    }
+    cb_src = p.src[t] + s_off;
+    v[it] = __ldcs(reinterpret_cast<const uint4*>(cb_src));
+    dst_off[it] = d_off;
+  }
+#pragma unroll
+  for (int it = 0; it < kRowIters; ++it) {
+    if (!ok[it]) continue;
+    cb_dst = p.dst[t] + dst_off[it];
+    *reinterpret_cast<uint4*>(cb_dst) = v[it];
+  }
+}
+
+static safedit_status row_copy(const safedit_tensor* src, const safedit_tensor* dst, int n_tensors,
+                               const int32_t* d_idx, int32_t n_idx, void* stream, int scatter) {
+  if (!src || !dst || n_tensors < 1 || n_tensors > kMaxRowTensors || n_idx < 0)
+    return SAFEDIT_ERR_INVALID_ARG;
+  if (n_idx > 0 && !d_idx) return SAFEDIT_ERR_INVALID_ARG;
+  RowCopyParams p{};
+  int max_bh = 0, max_blocks = 0;
+  int n_rows_x = -1;
+  for (int t = 0; t < n_tensors; ++t) {
+    const safedit_tensor& s = src[t];
+    const safedit_tensor& d = dst[t];
+    safedit_status st;
+    if ((st = check_tensor(&s, 4)) != SAFEDIT_OK) return st;
+    if ((st = check_tensor(&d, 4)) != SAFEDIT_OK) return st;
+    if (s.dtype != d.dtype) return SAFEDIT_ERR_DTYPE;
+    const int es = elt_size(s.dtype);
+    if (es != 2 && es != 4) return SAFEDIT_ERR_DTYPE;
+    const safedit_tensor& compact = scatter ? s : d;
+    const safedit_tensor& indexed = scatter ? d : s;
+    if (compact.dims[0] != indexed.dims[0] || compact.dims[1] != indexed.dims[1] ||
+        compact.dims[3] != indexed.dims[3])
+      return SAFEDIT_ERR_SHAPE;
+    if (compact.dims[2] != n_idx) return SAFEDIT_ERR_SHAPE;
+    if (n_rows_x < 0) n_rows_x = static_cast<int>(indexed.dims[2]);
+    if (indexed.dims[2] != n_rows_x) return SAFEDIT_ERR_SHAPE;
+    if (s.strides[3] != 1 || d.strides[3] != 1) return SAFEDIT_ERR_ALIGNMENT;
+    const int64_t row_bytes = s.dims[3] * es;
+    if (row_bytes % 16 != 0 || row_bytes == 0) return SAFEDIT_ERR_ALIGNMENT;
+    for (int k = 0; k < 3; ++k)
+      if ((s.strides[k] * es) % 16 != 0 || (d.strides[k] * es) % 16 != 0)
+        return SAFEDIT_ERR_ALIGNMENT;
+    if (!aligned16(s.data) || !aligned16(d.data)) return SAFEDIT_ERR_ALIGNMENT;
+    if (row_bytes / 16 > kRowThreads) return SAFEDIT_ERR_UNSUPPORTED;
+    if (s.dims[0] * s.dims[1] > 65535) return SAFEDIT_ERR_UNSUPPORTED;
+    p.src[t] = static_cast<const char*>(s.data);
+    p.dst[t] = static_cast<char*>(d.data);
+    p.c_sb[t] = compact.strides[0] * es;
+    p.c_sh[t] = compact.strides[1] * es;
+    p.c_sr[t] = compact.strides[2] * es;
+    p.x_sb[t] = indexed.strides[0] * es;
+    p.x_sh[t] = indexed.strides[1] * es;
+    p.x_sr[t] = indexed.strides[2] * es;
+    p.H[t] = static_cast<int>(s.dims[1]);
+    p.BH[t] = static_cast<int>(s.dims[0] * s.dims[1]);
+    p.units[t] = static_cast<int>(row_bytes / 16);
+    p.rows_per_pass[t] = kRowThreads / p.units[t];
+    const int rows_per_block = p.rows_per_pass[t] * kRowIters;
+    const int blocks = (n_idx + rows_per_block - 1) / rows_per_block;
+    if (p.BH[t] > max_bh) max_bh = p.BH[t];
+    if (blocks > max_blocks) max_blocks = blocks;
+  }
+  if (n_idx == 0 || max_bh == 0) return SAFEDIT_OK;
+  p.n_idx = n_idx;
+  p.n_rows_x = n_rows_x;
+  p.idx = d_idx;
+  p.scatter = scatter;
+  p.status = status_ptr();
+  if (!p.status) return SAFEDIT_ERR_CUDA;
+  dim3 grid(max_blocks, max_bh, n_tensors);
+  row_copy_kernel<<<grid, kRowThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return after_launch(1);
+}
+
+// --------------------------------------------------------------- sw_cfg ---
+struct CfgParams {
+  const float* c;
+  const float* u;
+  const float* s;
+  float* out;
+  int64_t N, F;
+  int64_t sc, su, so;  // row strides (elements)
+  float g_ctx, g_diff;
+};
+
+__global__ void __launch_bounds__(256) sw_cfg_vec4_kernel(CfgParams p) {
+  const int64_t F4 = p.F >> 2;
+  const int64_t total = p.N * F4;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t i = e / F4;
+    const int64_t f = (e - i * F4) << 2;
+    const float g = fmaf(p.g_diff, __ldg(p.s + i), p.g_ctx);
+    const float4 c = __ldcs(reinterpret_cast<const float4*>(p.c + i * p.sc + f));
+    const float4 u = __ldcs(reinterpret_cast<const float4*>(p.u + i * p.su + f));
+    float4 o;
+    o.x = fmaf(g, c.x - u.x, u.x);
+    o.y = fmaf(g, c.y - u.y, u.y);
+    o.z = fmaf(g, c.z - u.z, u.z);
+    o.w = fmaf(g, c.w - u.w, u.w);
+    __stcs(reinterpret_cast<float4*>(p.out + i * p.so + f), o);
+  }
+}
+
+__global__ void __launch_bounds__(256) sw_cfg_scalar_kernel(CfgParams p) {
+  const int64_t total = p.N * p.F;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t i = e / p.F;
+    const int64_t f = e - i * p.F;
+    const float g = fmaf(p.g_diff, p.s[i], p.g_ctx);
+    const float c = p.c[i * p.sc + f], u = p.u[i * p.su + f];
+    p.out[i * p.so + f] = fmaf(g, c - u, u);
+  }
+}
+
+}  // namespace sd
+
+using namespace sd;
+
+extern "C" {
+
+safedit_status safedit_scatter_state(const safedit_tensor* src, const safedit_tensor* dst,
+                                     int32_t n_tensors, const int32_t* d_idx, int32_t n_idx,
+                                     void* stream) {
+  return row_copy(src, dst, n_tensors, d_idx, n_idx, stream, 1);
+}
+
+safedit_status safedit_gather_rows(const safedit_tensor* src, const safedit_tensor* dst,
+                                   int32_t n_tensors, const int32_t* d_idx, int32_t n_idx,
+                                   void* stream) {
+  return row_copy(src, dst, n_tensors, d_idx, n_idx, stream, 0);
+}
+
+safedit_status safedit_sw_cfg(const safedit_tensor* eps_c, const safedit_tensor* eps_u,
+                              const float* d_s, float gamma_ctx, float gamma_sens,
+                              const safedit_tensor* out, void* stream) {
+  safedit_status st;
+  if ((st = check_tensor(eps_c, 2)) != SAFEDIT_OK) return st;
+  if ((st = check_tensor(eps_u, 2)) != SAFEDIT_OK) return st;
+  if ((st = check_tensor(out, 2)) != SAFEDIT_OK) return st;
+  if (!d_s) return SAFEDIT_ERR_INVALID_ARG;
+  if (eps_c->dtype != SAFEDIT_F32 || eps_u->dtype != SAFEDIT_F32 || out->dtype != SAFEDIT_F32)
+    return SAFEDIT_ERR_DTYPE;
+  const int64_t N = eps_c->dims[0], F = eps_c->dims[1];
+  if (eps_u->dims[0] != N || eps_u->dims[1] != F || out->dims[0] != N || out->dims[1] != F)
+    return SAFEDIT_ERR_SHAPE;
+  if (eps_c->strides[1] != 1 || eps_u->strides[1] != 1 || out->strides[1] != 1)
+    return SAFEDIT_ERR_ALIGNMENT;
+  if (N == 0 || F == 0) return SAFEDIT_OK;
+  CfgParams p;
+  p.c = static_cast<const float*>(eps_c->data);
+  p.u = static_cast<const float*>(eps_u->data);
+  p.s = d_s;
+  p.out = static_cast<float*>(out->data);
+  p.N = N;
+  p.F = F;
+  p.sc = eps_c->strides[0];
+  p.su = eps_u->strides[0];
+  p.so = out->strides[0];
+  p.g_ctx = gamma_ctx;
+  p.g_diff = gamma_sens - gamma_ctx;
+  const bool vec = (F % 4 == 0) && (p.sc % 4 == 0) && (p.su % 4 == 0) && (p.so % 4 == 0) &&
+                   aligned16(p.c) && aligned16(p.u) && aligned16(p.out);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t work = vec ? N * (F / 4) : N * F;
+  int64_t blocks = (work + 255) / 256;
+  const int64_t cap = int64_t(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (vec)
+    sw_cfg_vec4_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+  else
+    sw_cfg_scalar_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+  return after_launch(1);
+}
+
+}  // extern "C"

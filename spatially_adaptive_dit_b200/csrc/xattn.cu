@@ -1,0 +1,315 @@
+// xattn.cu -- PCSP score producer: image->text cross-attention probabilities
+// for one batch entry (SAFE-DiT summary, 방법론 2: attention weights from
+// image tokens to text tokens gathered during warm-up; AccelAes summary B.1
+// step 3).  Text padding is a kept semantic mask (방법론 1 보존): padding keys
+// receive exactly 0.
+//
+// One CTA = 128 image rows of one head, 128 threads (thread = row = TMEM
+// lane).  TMA brings the Q tile and the whole text-key block (L <= 256) into
+// swizzled shared memory; one elected thread issues tcgen05.mma for
+// S = Q K^T (M=128, N=L rounded up to 16) into TMEM; the softmax runs in
+// three TMEM passes (max; exp + sum with the exponentials written back to
+// TMEM; scale) and the probabilities leave through a double-buffered,
+// 128B-swizzled shared-memory stage and TMA tensor stores, so the 4-byte
+// P writes reach HBM as full lines.
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace sd {
+
+template <int D>
+struct XCfg {
+  static constexpr int CH = (D % 64 == 0) ? 64 : 32;
+  static constexpr int NCH = D / CH;
+  static constexpr int ROWB = CH * 2;
+  static constexpr uint32_t LAYOUT = (CH == 64) ? 2u : 4u;
+  static constexpr int Q_CHUNK = 128 * ROWB;
+  static constexpr int Q_BYTES = NCH * Q_CHUNK;
+  static constexpr int K_CHUNK = 256 * ROWB;  // room for L <= 256 rows
+  static constexpr int K_BYTES = NCH * K_CHUNK;
+  static constexpr int STAGE_BYTES = 128 * 128;  // 128 rows x 32 f32
+  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + K_BYTES + 2 * STAGE_BYTES + 256 + 1024;
+};
+
+struct XParams {
+  const uint8_t* key_valid;  // [L] of the selected batch entry
+  int L, Lpad, N, b, tmem_cols;
+  float scale_log2;
+  int* status;
+  uint64_t wait_limit;
+};
+
+constexpr float kXLog2e = 1.4426950408889634f;
+
+template <int D>
+__global__ void __launch_bounds__(128)
+    xattn_probs_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmKt,
+                       const __grid_constant__ CUtensorMap tmP, const XParams p) {
+  using C = XCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sK = sQ + C::Q_BYTES;
+  const uint32_t sStage = sK + C::K_BYTES;
+  uint8_t* tail = smem + C::Q_BYTES + C::K_BYTES + 2 * C::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + 32);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tail + 40);
+  float* vadd = reinterpret_cast<float*>(tail + 256);  // [256] additive validity
+  const uint32_t bar_load = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[1]);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.y;
+  const int row0 = blockIdx.x * 128;
+
+  if (tid == 0) {
+    mbar_init(bar_load, 1);
+    mbar_init(bar_mma, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  for (int j = tid; j < 256; j += 128)
+    vadd[j] = (j < p.L && p.key_valid[j] != 0) ? 0.f : -INFINITY;
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), uint32_t(p.tmem_cols));
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit};
+
+  bool ok = true;
+  if (tid == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmKt);
+    mbar_arrive_expect_tx(bar_load, uint32_t(C::Q_BYTES + C::NCH * p.Lpad * C::ROWB));
+#pragma unroll
+    for (int c = 0; c < C::NCH; ++c) {
+      tma_load_4d(sQ + c * C::Q_CHUNK, &tmQ, bar_load, c * C::CH, row0, h, p.b);
+      tma_load_4d(sK + c * C::K_CHUNK, &tmKt, bar_load, c * C::CH, 0, h, p.b);
+    }
+    if (wait_bounded(bar_load, 0u, ctl)) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(128, p.Lpad, 0, 0);
+      constexpr uint32_t SBO = 8u * C::ROWB;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int chunk = (kk * 16) / C::CH;
+        const uint32_t within = uint32_t(((kk * 16) % C::CH) * 2);
+        mma_ss(tmem, smem_desc(sQ + chunk * C::Q_CHUNK + within, 16u, SBO, C::LAYOUT),
+               smem_desc(sK + chunk * C::K_CHUNK + within, 16u, SBO, C::LAYOUT), idesc,
+               kk > 0 ? 1u : 0u);
+      }
+      tc_commit(bar_mma);
+    } else {
+      wait_drain(bar_load, 0u, 1000000000ull);
+    }
+  }
+  ok = wait_warp(bar_mma, 0u, ctl);
+
+  if (ok) {
+    tc_fence_after();
+    const uint32_t tl = tmem + (uint32_t(warp * 32) << 16);
+    const int nc = p.Lpad / 32 + ((p.Lpad % 32) ? 1 : 0);  // 32-column chunks (Lpad % 16 == 0)
+    const float sl2 = p.scale_log2;
+    // pass 1: row max over valid keys
+    float m = -INFINITY;
+    for (int c = 0; c < nc; ++c) {
+      const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
+      uint32_t r[32];
+      if (ncol == 32) {
+        tmem_ld32(tl + uint32_t(c * 32), r);
+      } else {
+        uint32_t r16[16];
+        tmem_ld16(tl + uint32_t(c * 32), r16);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) r[e] = r16[e];
+      }
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (e < ncol) m = fmaxf(m, fmaf(__uint_as_float(r[e]), sl2, vadd[c * 32 + e]));
+    }
+    const float m_use = (m == -INFINITY) ? 0.f : m;
+    // pass 2: exponentials (written back to TMEM) and their sum
+    float sum = 0.f;
+    for (int c = 0; c < nc; ++c) {
+      const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
+      uint32_t r[32];
+      if (ncol == 32) {
+        tmem_ld32(tl + uint32_t(c * 32), r);
+      } else {
+        uint32_t r16[16];
+        tmem_ld16(tl + uint32_t(c * 32), r16);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) r[e] = r16[e];
+      }
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float ev =
+            (e < ncol) ? ex2_approx(fmaf(__uint_as_float(r[e]), sl2, vadd[c * 32 + e]) - m_use)
+                       : 0.f;
+        sum += ev;
+        r[e] = __float_as_uint(ev);
+      }
+      if (ncol == 32) {
+        tmem_st32(tl + uint32_t(c * 32), r);
+      } else {
+        uint32_t r16[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) r16[e] = r[e];
+        tmem_st16(tl + uint32_t(c * 32), r16);
+      }
+    }
+    tmem_wait_st();
+    if (!(sum > 0.f) && row0 + tid < p.N) set_status(p.status, SAFEDIT_ERR_MASKED_ROW);
+    const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
+    // pass 3: normalise, stage (128B swizzle) and store 128 x 32 boxes
+    for (int c = 0; c < nc; ++c) {
+      const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
+      uint32_t r[32];
+      if (ncol == 32) {
+        tmem_ld32(tl + uint32_t(c * 32), r);
+      } else {
+        uint32_t r16[16];
+        tmem_ld16(tl + uint32_t(c * 32), r16);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) r[e] = r16[e];
+#pragma unroll
+        for (int e = 16; e < 32; ++e) r[e] = 0u;
+      }
+      tmem_wait_ld();
+      const uint32_t buf = sStage + uint32_t((c & 1) * C::STAGE_BYTES);
+      if (c >= 2) {
+        if (tid == 0) bulk_wait_read<1>();
+        named_bar_sync(1, 128);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t off = uint32_t(tid * 128 + ((u ^ (tid & 7)) * 16));
+        const float a0 = __uint_as_float(r[4 * u]) * inv, a1 = __uint_as_float(r[4 * u + 1]) * inv,
+                    a2 = __uint_as_float(r[4 * u + 2]) * inv,
+                    a3 = __uint_as_float(r[4 * u + 3]) * inv;
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(buf + off), "f"(a0),
+                     "f"(a1), "f"(a2), "f"(a3)
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (tid == 0) {
+        tma_store_3d(&tmP, buf, c * 32, row0, h);
+        bulk_commit();
+      }
+    }
+    if (tid == 0) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, uint32_t(p.tmem_cols));
+  }
+}
+
+template <int D>
+static safedit_status launch_x(const CUtensorMap& a, const CUtensorMap& k, const CUtensorMap& pm,
+                               const XParams& p, int H, cudaStream_t s) {
+  auto kern = xattn_probs_kernel<D>;
+  safedit_status st = set_smem(reinterpret_cast<const void*>(kern), XCfg<D>::SMEM_BYTES);
+  if (st != SAFEDIT_OK) return st;
+  dim3 grid((p.N + 127) / 128, H);
+  kern<<<grid, 128, XCfg<D>::SMEM_BYTES, s>>>(a, k, pm, p);
+  return after_launch(1);
+}
+
+}  // namespace sd
+
+using namespace sd;
+
+extern "C" safedit_status safedit_cross_attn_probs(const safedit_tensor* q_img,
+                                                   const safedit_tensor* k_txt,
+                                                   const uint8_t* d_key_valid,
+                                                   int32_t batch_index, float scale,
+                                                   const safedit_tensor* p_out, void* stream) {
+  safedit_status st;
+  for (const safedit_tensor* t : {q_img, k_txt}) {
+    if ((st = check_tensor(t, 4)) != SAFEDIT_OK) return st;
+    if (t->dtype != SAFEDIT_BF16) return SAFEDIT_ERR_DTYPE;
+    if (t->strides[3] != 1 || !aligned16(t->data)) return SAFEDIT_ERR_ALIGNMENT;
+    for (int i = 0; i < 3; ++i)
+      if (t->strides[i] % 8 != 0 || t->strides[i] < 0) return SAFEDIT_ERR_ALIGNMENT;
+  }
+  if ((st = check_tensor(p_out, 3)) != SAFEDIT_OK) return st;
+  if (!d_key_valid) return SAFEDIT_ERR_INVALID_ARG;
+  const int64_t B = q_img->dims[0], H = q_img->dims[1], N = q_img->dims[2], D = q_img->dims[3];
+  const int64_t L = k_txt->dims[2];
+  if (k_txt->dims[0] != B || k_txt->dims[1] != H || k_txt->dims[3] != D) return SAFEDIT_ERR_SHAPE;
+  if (batch_index < 0 || batch_index >= B) return SAFEDIT_ERR_INVALID_ARG;
+  if (D != 64 && D != 96 && D != 128) return SAFEDIT_ERR_UNSUPPORTED;
+  if (L < 1 || L > 256) return SAFEDIT_ERR_UNSUPPORTED;
+  if (p_out->dtype != SAFEDIT_F32) return SAFEDIT_ERR_DTYPE;
+  if (p_out->dims[0] != H || p_out->dims[1] != N || p_out->dims[2] != L) return SAFEDIT_ERR_SHAPE;
+  if (p_out->strides[2] != 1 || p_out->strides[1] % 4 != 0 || p_out->strides[0] % 4 != 0 ||
+      !aligned16(p_out->data))
+    return SAFEDIT_ERR_ALIGNMENT;
+  if (N == 0 || H == 0) return SAFEDIT_OK;
+  if (H > 65535) return SAFEDIT_ERR_SHAPE;
+  XParams p{};
+  p.key_valid = d_key_valid + int64_t(batch_index) * L;
+  p.L = static_cast<int>(L);
+  p.Lpad = static_cast<int>((L + 15) / 16 * 16);
+  p.N = static_cast<int>(N);
+  p.b = batch_index;
+  int cols = 32;
+  while (cols < p.Lpad) cols <<= 1;
+  p.tmem_cols = cols;
+  const float sc = (scale > 0.f) ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale_log2 = sc * kXLog2e;
+  p.wait_limit = wait_limit_ns();
+  const int ch = (D % 64 == 0) ? 64 : 32;
+  const CUtensorMapSwizzle swz = ch == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap tq, tk, tp;
+  {
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(N), uint64_t(H), uint64_t(B)};
+    const uint64_t str[3] = {uint64_t(q_img->strides[2]) * 2, uint64_t(q_img->strides[1]) * 2,
+                             uint64_t(q_img->strides[0]) * 2};
+    const uint32_t box[4] = {uint32_t(ch), 128u, 1u, 1u};
+    if ((st = encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, q_img->data, dims, str, box,
+                          swz)) != SAFEDIT_OK)
+      return st;
+  }
+  {
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(L), uint64_t(H), uint64_t(B)};
+    const uint64_t str[3] = {uint64_t(k_txt->strides[2]) * 2, uint64_t(k_txt->strides[1]) * 2,
+                             uint64_t(k_txt->strides[0]) * 2};
+    const uint32_t box[4] = {uint32_t(ch), uint32_t(p.Lpad), 1u, 1u};
+    if ((st = encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, k_txt->data, dims, str, box,
+                          swz)) != SAFEDIT_OK)
+      return st;
+  }
+  {
+    const uint64_t dims[3] = {uint64_t(L), uint64_t(N), uint64_t(H)};
+    const uint64_t str[2] = {uint64_t(p_out->strides[1]) * 4, uint64_t(p_out->strides[0]) * 4};
+    const uint32_t box[3] = {32u, 128u, 1u};
+    if ((st = encode_tmap(&tp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p_out->data, dims, str, box,
+                          CU_TENSOR_MAP_SWIZZLE_128B)) != SAFEDIT_OK)
+      return st;
+  }
+  p.status = status_ptr();
+  if (!p.status) return SAFEDIT_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (D) {
+    case 64: return launch_x<64>(tq, tk, tp, p, static_cast<int>(H), s);
+    case 96: return launch_x<96>(tq, tk, tp, p, static_cast<int>(H), s);
+    default: return launch_x<128>(tq, tk, tp, p, static_cast<int>(H), s);
+  }
+}

@@ -1,0 +1,151 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every entry point
+include/safedit.h declares, and rejects bad arguments on the host before any
+CUDA call (no GPU needed, nothing is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def sd():
+    from spatially_adaptive_dit_b200 import build
+    build.build()
+    from spatially_adaptive_dit_b200 import safedit
+    return safedit
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "safedit.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(safedit_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(sd):
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(sd.lib(), n), n
+        assert hasattr(sd, n), f"python binding lacks {n}"
+    assert set(names) == set(sd.EXPORTED)
+
+
+def test_status_strings_and_counters(sd):
+    assert sd.status_string(0) == "ok"
+    for c in range(1, 10):
+        assert sd.status_string(c) not in ("ok", "unknown status")
+    assert sd.status_string(77) == "unknown status"
+    assert sd.safedit_kernel_launch_count() >= 0
+    old = sd.safedit_debug_set_wait_limit_ns(12345)
+    assert sd.safedit_debug_set_wait_limit_ns(old) == 12345
+
+
+def _desc(sd, dims, strides, dtype, ptr=0x10000):
+    d = sd.SafeditTensor()
+    d.data = ptr
+    d.dtype = dtype
+    d.ndim = len(dims)
+    for i, (a, b) in enumerate(zip(dims, strides)):
+        d.dims[i] = a
+        d.strides[i] = b
+    return d
+
+
+def _bhnd(sd, B, H, N, D, dtype=None, ptr=0x10000, strides=None):
+    dtype = sd.BF16 if dtype is None else dtype
+    st = strides or (H * N * D, N * D, D, 1)
+    return _desc(sd, (B, H, N, D), st, dtype, ptr)
+
+
+def test_attn_host_validation(sd):
+    call = lambda *a: sd.raw_call("safedit_attn_subset", *a)  # noqa: E731
+    q, k, v, o = (_bhnd(sd, 1, 2, 256, 64) for _ in range(4))
+    R = ctypes.byref
+    # null tensor
+    assert call(None, R(k), R(v), None, 0, None, None, 0.0, R(o), 0, None) == sd.ERR_INVALID_ARG
+    # wrong dtype
+    qf = _bhnd(sd, 1, 2, 256, 64, dtype=sd.F32)
+    assert call(R(qf), R(k), R(v), None, 0, None, None, 0.0, R(o), 0, None) == sd.ERR_DTYPE
+    # unsupported head dim
+    q80, k80, v80, o80 = (_bhnd(sd, 1, 2, 256, 80) for _ in range(4))
+    assert call(R(q80), R(k80), R(v80), None, 0, None, None, 0.0, R(o80), 0, None) == sd.ERR_UNSUPPORTED
+    # misaligned pointer / stride
+    qm = _bhnd(sd, 1, 2, 256, 64, ptr=0x10008)
+    assert call(R(qm), R(k), R(v), None, 0, None, None, 0.0, R(o), 0, None) == sd.ERR_ALIGNMENT
+    qs = _bhnd(sd, 1, 2, 256, 64, strides=(2 * 256 * 68, 256 * 68, 68, 1))
+    assert call(R(qs), R(k), R(v), None, 0, None, None, 0.0, R(o), 0, None) == sd.ERR_ALIGNMENT
+    # shape mismatch between k and v
+    v2 = _bhnd(sd, 1, 2, 128, 64)
+    assert call(R(q), R(k), R(v2), None, 0, None, None, 0.0, R(o), 0, None) == sd.ERR_SHAPE
+    # compact output must have n_idx rows
+    o_bad = _bhnd(sd, 1, 2, 10, 64)
+    assert call(R(q), R(k), R(v), ctypes.c_void_p(0x20000), 11, None, None, 0.0, R(o_bad), 0,
+                None) == sd.ERR_SHAPE
+    assert call(R(q), R(k), R(v), None, 0, None, None, 0.0, R(o), 2, None) == sd.ERR_INVALID_ARG
+    # key pad of the wrong length, bias of the wrong dtype
+    pad = _desc(sd, (1, 255), (256, 1), sd.F32)
+    assert call(R(q), R(k), R(v), None, 0, R(pad), None, 0.0, R(o), 0, None) == sd.ERR_SHAPE
+    bias = _desc(sd, (1, 1, 256, 256), (65536, 65536, 256, 1), sd.F16)
+    assert call(R(q), R(k), R(v), None, 0, None, R(bias), 0.0, R(o), 0, None) == sd.ERR_DTYPE
+
+
+def test_bandwidth_kernels_host_validation(sd):
+    R = ctypes.byref
+    src = (sd.SafeditTensor * 1)(_bhnd(sd, 1, 2, 10, 96))
+    dst = (sd.SafeditTensor * 1)(_bhnd(sd, 1, 2, 100, 96))
+    f = lambda *a: sd.raw_call("safedit_scatter_state", *a)  # noqa: E731
+    assert f(src, dst, 0, ctypes.c_void_p(0x20000), 10, None) == sd.ERR_INVALID_ARG
+    assert f(src, dst, 5, ctypes.c_void_p(0x20000), 10, None) == sd.ERR_INVALID_ARG
+    assert f(src, dst, 1, None, 10, None) == sd.ERR_INVALID_ARG
+    assert f(src, dst, 1, ctypes.c_void_p(0x20000), 11, None) == sd.ERR_SHAPE
+    dst_f = (sd.SafeditTensor * 1)(_bhnd(sd, 1, 2, 100, 96, dtype=sd.F32))
+    assert f(src, dst_f, 1, ctypes.c_void_p(0x20000), 10, None) == sd.ERR_DTYPE
+    # rows of 6 bf16 are not 16-byte multiples
+    src6 = (sd.SafeditTensor * 1)(_bhnd(sd, 1, 2, 10, 6))
+    dst6 = (sd.SafeditTensor * 1)(_bhnd(sd, 1, 2, 100, 6))
+    assert f(src6, dst6, 1, ctypes.c_void_p(0x20000), 10, None) == sd.ERR_ALIGNMENT
+
+    c = _desc(sd, (100, 16), (16, 1), sd.F32)
+    u = _desc(sd, (100, 16), (16, 1), sd.F32)
+    o_bad = _desc(sd, (100, 8), (8, 1), sd.F32)
+    g = lambda *a: sd.raw_call("safedit_sw_cfg", *a)  # noqa: E731
+    assert g(R(c), R(u), None, 3.0, 5.0, R(u), None) == sd.ERR_INVALID_ARG
+    assert g(R(c), R(u), ctypes.c_void_p(0x30000), 3.0, 5.0, R(o_bad), None) == sd.ERR_SHAPE
+    cb = _desc(sd, (100, 16), (16, 1), sd.BF16)
+    assert g(R(cb), R(u), ctypes.c_void_p(0x30000), 3.0, 5.0, R(u), None) == sd.ERR_DTYPE
+
+    fin = lambda *a: sd.raw_call("safedit_partition_finalize", *a)  # noqa: E731
+    assert fin(None, 10, 3, None, None, None, None) == sd.ERR_INVALID_ARG
+    assert fin(ctypes.c_void_p(0x40000), 10, 11, None, None, None, None) == sd.ERR_INVALID_ARG
+    assert fin(ctypes.c_void_p(0x40000), 10, -1, None, None, None, None) == sd.ERR_INVALID_ARG
+
+    P = _desc(sd, (2, 16, 32), (512, 32, 1), sd.BF16)
+    acc = lambda *a: sd.raw_call("safedit_partition_accumulate", *a)  # noqa: E731
+    assert acc(R(P), ctypes.c_void_p(0x50000), ctypes.c_void_p(0x60000), None) == sd.ERR_DTYPE
+    Pf = _desc(sd, (2, 16, 32), (512, 32, 2), sd.F32)
+    assert acc(R(Pf), ctypes.c_void_p(0x50000), ctypes.c_void_p(0x60000), None) == sd.ERR_ALIGNMENT
+
+    m = _desc(sd, (4, 4, 8, 8), (256, 64, 8, 1), sd.I32)
+    mk = lambda *a: sd.raw_call("safedit_mask_is_row_constant", *a)  # noqa: E731
+    assert mk(R(m), ctypes.c_void_p(0x70000), None, None) == sd.ERR_DTYPE
+    m1 = _desc(sd, (8,), (1,), sd.F32)
+    assert mk(R(m1), ctypes.c_void_p(0x70000), None, None) == sd.ERR_SHAPE
+    m2 = _desc(sd, (8, 8), (8, 2), sd.F32)
+    assert mk(R(m2), ctypes.c_void_p(0x70000), None, None) == sd.ERR_ALIGNMENT
+
+    xq = _bhnd(sd, 2, 2, 256, 64)
+    xk = _bhnd(sd, 2, 2, 300, 64)
+    xp = _desc(sd, (2, 256, 300), (256 * 300, 300, 1), sd.F32)
+    x = lambda *a: sd.raw_call("safedit_cross_attn_probs", *a)  # noqa: E731
+    assert x(R(xq), R(xk), ctypes.c_void_p(0x80000), 0, 0.0, R(xp), None) == sd.ERR_UNSUPPORTED
+    xk2 = _bhnd(sd, 2, 2, 32, 64)
+    xp2 = _desc(sd, (2, 256, 32), (256 * 32, 32, 1), sd.F32)
+    assert x(R(xq), R(xk2), ctypes.c_void_p(0x80000), 2, 0.0, R(xp2), None) == sd.ERR_INVALID_ARG
+    assert x(R(xq), R(xk2), None, 0, 0.0, R(xp2), None) == sd.ERR_INVALID_ARG
+    xp3 = _desc(sd, (2, 256, 30), (256 * 30, 30, 1), sd.F32)
+    xk3 = _bhnd(sd, 2, 2, 30, 64)
+    assert x(R(xq), R(xk3), ctypes.c_void_p(0x80000), 0, 0.0, R(xp3), None) == sd.ERR_ALIGNMENT

@@ -1,0 +1,219 @@
+"""GPU vs oracle parity of the SRSU subset attention / CAR dense anchor kernel
+(tcgen05/TMEM), from tiny ragged cases to the full-size launch configuration
+the benchmark times (sampled rows), plus the kernel's edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from spatially_adaptive_dit_b200 import workloads as wl
+from tests.gpu_util import check_attn, expect_status, f64, sd
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+BF = torch.bfloat16
+
+
+def _gen(seed):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return g
+
+
+def _rand_idx(n_total, k, seed):
+    return torch.sort(torch.randperm(n_total, generator=_gen(seed))[:k]).values.to(torch.int32)
+
+
+def _qkv(B, H, Nq, Nk, D, seed):
+    g = _gen(seed)
+    q = torch.randn(B, H, Nq, D, generator=g).to(BF)
+    k = torch.randn(B, H, Nk, D, generator=g).to(BF)
+    v = torch.randn(B, H, Nk, D, generator=g).to(BF)
+    return q, k, v
+
+
+def run(q, k, v, idx=None, pad=None, bias=None, scale=0.0, out=None, scattered=False, status=0):
+    B, H, Nq, D = q.shape
+    n = Nq if idx is None else idx.numel()
+    if out is None:
+        out = torch.zeros(B, H, Nq if scattered else n, D, dtype=BF, device=DEV)
+    sd().safedit_attn_subset(q, k, v, idx, n, pad, bias, scale, out, int(scattered))
+    expect_status(status)
+    return out
+
+
+def oracle_rows(q, k, v, idx, b, h, rows=None, pad=None, bias=None, scale=None):
+    """Oracle output rows r (positions in idx) of slice (b,h)."""
+    qi = q[b, h]
+    sel = np.arange(len(idx)) if rows is None else np.asarray(rows)
+    ix = np.asarray(idx)[sel].astype(np.int32)
+    brow = None
+    if bias is not None:
+        bb = bias[b, 0 if bias.shape[1] == 1 else h]
+        brow = f64(bb[torch.as_tensor(ix, dtype=torch.long, device=bb.device)])
+    return oracle.attn_subset(f64(qi), f64(k[b, h]), f64(v[b, h]), ix,
+                              pad=None if pad is None else f64(pad[b]), bias_rows=brow, scale=scale)
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,D,k_rows", [(1, 2, 256, 256, 64, 64),     # tiny config shape
+                                                 (2, 3, 300, 300, 96, 77),     # ragged rows and keys
+                                                 (1, 2, 517, 200, 128, 130),   # ragged, d=128
+                                                 (1, 1, 64, 1, 96, 3),         # one key
+                                                 (1, 2, 2000, 700, 96, 600)])  # several tiles, 3 CTAs
+def test_subset_matches_oracle(B, H, Nq, Nk, D, k_rows):
+    q, k, v = _qkv(B, H, Nq, Nk, D, seed=B * 1000 + Nq + D)
+    idx = _rand_idx(Nq, k_rows, seed=Nk + k_rows)
+    qd, kd, vd, idd = q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV)
+    out = run(qd, kd, vd, idd)
+    for b in range(B):
+        for h in range(H):
+            ref = oracle_rows(q, k, v, idx.numpy(), b, h)
+            check_attn(f64(out[b, h]), ref, f"b{b}h{h}")
+
+
+@pytest.mark.parametrize("N,D", [(256, 64), (129, 96), (384, 128)])
+def test_dense_anchor_and_subset_rows_agree(N, D):
+    """idx = NULL is the CAR anchor: all rows.  An SRSU row must equal the
+    same row of the anchor (the S queries attend to the global K/V)."""
+    q, k, v = _qkv(1, 2, N, N, D, seed=N + D)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    dense = run(qd, kd, vd)
+    for h in range(2):
+        ref = oracle.attn_dense(f64(q[0, h]), f64(k[0, h]), f64(v[0, h]))
+        check_attn(f64(dense[0, h]), ref, f"dense h{h}")
+    idx = _rand_idx(N, N // 3, seed=5)
+    sub = run(qd, kd, vd, idx.to(DEV))
+    assert torch.equal(sub, dense[:, :, idx.long()])
+
+
+def test_scattered_output_leaves_context_rows_untouched():
+    B, H, N, D, kr = 2, 2, 700, 96, 211
+    q, k, v = _qkv(B, H, N, N, D, seed=77)
+    idx = _rand_idx(N, kr, seed=78)
+    state = torch.randn(B, H, N, D, generator=_gen(79)).to(BF)
+    st_d = state.to(DEV)
+    run(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), out=st_d, scattered=True)
+    mask = torch.ones(N, dtype=torch.bool)
+    mask[idx.long()] = False
+    assert torch.equal(st_d.cpu()[:, :, mask], state[:, :, mask])
+    for b in range(B):
+        for h in range(H):
+            ref = oracle_rows(q, k, v, idx.numpy(), b, h)
+            check_attn(f64(st_d[b, h, idx.long()]), ref)
+
+
+def test_kept_masks_key_padding_and_bias():
+    """Kept semantic masks: key padding (exact zero weight) and a non-uniform
+    bias, in f32 and bf16, with a per-head and a broadcast head dim."""
+    B, H, N, D, kr = 2, 2, 640, 128, 150
+    q, k, v = _qkv(B, H, N, N, D, seed=11)
+    idx = _rand_idx(N, kr, seed=12)
+    pad = torch.zeros(B, N)
+    pad[0, N - N // 8:] = float("-inf")
+    pad[1, ::3] = float("-inf")
+    g = _gen(13)
+    for bias in (torch.randn(B, H, N, N, generator=g), torch.randn(B, 1, N, N, generator=g).to(BF)):
+        bd = bias.to(DEV)
+        out = run(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), pad=pad.to(DEV), bias=bd)
+        for b in range(B):
+            for h in range(H):
+                ref = oracle_rows(q, k, v, idx.numpy(), b, h, pad=pad, bias=bias)
+                check_attn(f64(out[b, h]), ref, f"b{b}h{h}")
+    # padded keys carry no weight: garbage in their values must not leak
+    vg = v.clone()
+    vg[0, :, N - N // 8:] = 1e4
+    o1 = run(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), pad=pad.to(DEV))
+    o2 = run(q.to(DEV), k.to(DEV), vg.to(DEV), idx.to(DEV), pad=pad.to(DEV))
+    assert torch.equal(o1[0], o2[0])
+
+
+def test_row_constant_mask_elision_is_invisible():
+    """A row-constant additive bias (removable by the criterion) changes the
+    GPU result only by rounding."""
+    B, H, N, D = 1, 2, 512, 96
+    q, k, v = _qkv(B, H, N, N, D, seed=21)
+    c = (torch.rand(N, 1, generator=_gen(22)) * 8 - 4).expand(N, N)
+    bias = c.reshape(1, 1, N, N).contiguous()
+    idx = _rand_idx(N, 100, seed=23).to(DEV)
+    with_mask = run(q.to(DEV), k.to(DEV), v.to(DEV), idx, bias=bias.to(DEV))
+    without = run(q.to(DEV), k.to(DEV), v.to(DEV), idx)
+    check_attn(f64(with_mask), f64(without), "elided vs kept row-constant mask")
+
+
+def test_explicit_scale_and_fully_masked_row_and_bad_index():
+    B, H, N, D = 1, 1, 256, 64
+    q, k, v = _qkv(B, H, N, N, D, seed=31)
+    idx = torch.arange(0, 256, 4, dtype=torch.int32)
+    out = run(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), scale=0.3)
+    check_attn(f64(out[0, 0]), oracle.attn_subset(f64(q[0, 0]), f64(k[0, 0]), f64(v[0, 0]), idx.numpy(),
+                                                  scale=0.3))
+    pad = torch.full((1, N), float("-inf"), device=DEV)
+    out = run(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), pad=pad, status=sd().ERR_MASKED_ROW)
+    assert torch.count_nonzero(out) == 0
+    bad = idx.clone()
+    bad[5] = N
+    out = torch.full((1, 1, idx.numel(), D), 7.0, dtype=BF, device=DEV)
+    run(q.to(DEV), k.to(DEV), v.to(DEV), bad.to(DEV), out=out, status=sd().ERR_INDEX)
+    assert torch.all(out[0, 0, 5] == 7.0)  # the bad row is skipped
+
+
+def test_config_1024_full_size():
+    w = wl.W1024
+    q, k, v = wl.qkv(w, device=DEV)
+    idx = _rand_idx(w.N, w.k, seed=41).to(DEV)
+    out = run(q, k, v, idx)
+    rows = np.arange(0, w.k, 7)
+    for (b, h) in [(0, 0), (1, 23), (0, 11)]:
+        ref = oracle_rows(q, k, v, idx.cpu().numpy(), b, h, rows=rows)
+        check_attn(f64(out[b, h, torch.as_tensor(rows, device=DEV)]), ref, f"b{b}h{h}")
+
+
+def test_config_2560_srsu_launch_as_benchmarked():
+    """The headline workload, in the launch configuration the benchmark
+    times: gathered S rows from the partition, scattered into O_state."""
+    w = wl.W2560
+    q, k, v = wl.qkv(w, device=DEV)
+    score = wl.blob_scores(wl.Workload("2560b", 2, B=1, H=1, N=w.N, d=w.d, L=1, n_valid=1,
+                                       rho=w.rho, grid=w.grid)).to(DEV)
+    idx = torch.empty(w.k, dtype=torch.int32, device=DEV)
+    sd().safedit_partition_finalize(score, w.N, w.k, idx, None, None)
+    state = torch.zeros(w.B, w.H, w.N, w.d, dtype=BF, device=DEV)
+    run(q, k, v, idx, out=state, scattered=True)
+    rows = np.linspace(0, w.k - 1, 48).astype(np.int64)
+    ic = idx.cpu().numpy()
+    for (b, h) in [(0, 0), (1, 17)]:
+        ref = oracle_rows(q, k, v, ic, b, h, rows=rows)
+        got = state[b, h, torch.as_tensor(ic[rows].astype(np.int64), device=DEV)]
+        check_attn(f64(got), ref, f"b{b}h{h}")
+
+
+def test_config_stress_kept_masks_sampled():
+    w = wl.STRESS
+    q, k, v = wl.qkv(w, device=DEV)
+    score = wl.blob_scores(w).to(DEV)
+    idx = torch.empty(w.k, dtype=torch.int32, device=DEV)
+    sd().safedit_partition_finalize(score, w.N, w.k, idx, None, None)
+    pad = torch.zeros(1, w.N, device=DEV)
+    pad[:, w.N - w.N // 8:] = float("-inf")   # text-padding style key mask (kept)
+    bias = wl.mask(w, "bias", device=DEV)     # non-uniform bias (kept), [1,1,N,N] bf16
+    out = run(q, k, v, idx, pad=pad, bias=bias)
+    rows = np.linspace(0, w.k - 1, 24).astype(np.int64)
+    ic = idx.cpu().numpy()
+    for h in (0, 31):
+        ref = oracle_rows(q, k, v, ic, 0, h, rows=rows, pad=pad, bias=bias)
+        check_attn(f64(out[0, h, torch.as_tensor(rows, device=DEV)]), ref, f"h{h}")
+
+
+def test_3072_sweep_sampled():
+    w = wl.W3072
+    q, k, v = wl.qkv(w, device=DEV)
+    score = wl.blob_scores(w).to(DEV)
+    for rho in w.rho_sweep:
+        kk = wl.k_of(rho, w.N)
+        idx = torch.empty(kk, dtype=torch.int32, device=DEV)
+        sd().safedit_partition_finalize(score, w.N, kk, idx, None, None)
+        out = run(q, k, v, idx)
+        rows = np.linspace(0, kk - 1, 12).astype(np.int64)
+        ref = oracle_rows(q, k, v, idx.cpu().numpy(), 1, 5, rows=rows)
+        check_attn(f64(out[1, 5, torch.as_tensor(rows, device=DEV)]), ref, f"rho={rho}")
+        del out
