@@ -296,12 +296,18 @@ def run_ours(args):
 
 
 def _ncu_traffic():
-    """dram bytes per SRSU launch from the committed ncu summary, if present and current."""
+    """DRAM bytes per SRSU launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from the committed ncu summary, or None when the kernel source changed
+    since those counters were taken."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "attn_subset_srsu_2560.traffic.json")
+    src = os.path.join(ROOT, "spatially_adaptive_dit_b200", "csrc", "attn.cu")
     try:
         with open(p) as f:
             d = json.load(f)
-        return d.get("bytes_per_launch")
+        with open(src, "rb") as f:
+            cur = hashlib.sha256(f.read()).hexdigest()[:16]
+        return d.get("bytes_per_launch") if d.get("attn_cu_sha256_16") == cur else None
     except Exception:
         return None
 
@@ -422,6 +428,66 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_only(args):
+    """One kernel of the path in isolation, `--reps` times on the bench
+    workload's buffers (the target of ncu captures and quick timing).  Prints
+    per-launch CUDA-event times; not a bench line."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    from spatially_adaptive_dit_b200 import safedit as sd
+    tr = Trajectory(W, dev)
+    stream = torch.cuda.Stream(device=dev)
+    w = W
+    with torch.cuda.stream(stream):
+        sd.safedit_cross_attn_probs(tr.q_img, tr.k_txt, tr.valid, 0, 0.0, tr.P, stream)
+        sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream)
+        sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s, stream)
+    stream.synchronize()
+    extra = {}
+    if args.only == "mask":
+        extra["mask"] = torch.zeros(1, 1, wl.STRESS.N, wl.STRESS.N, dtype=torch.bfloat16, device=dev)
+    fns = {
+        "srsu": (lambda: sd.safedit_attn_subset(tr.q, tr.k_state, tr.v_state, tr.idx_s, tr.k, None, None,
+                                                0.0, tr.o_state, 1, stream), tr.flop_srsu, None),
+        "anchor": (lambda: sd.safedit_attn_subset(tr.q, tr.k_state, tr.v_state, None, 0, None, None, 0.0,
+                                                  tr.o_state, 0, stream), tr.flop_dense, None),
+        "xattn": (lambda: sd.safedit_cross_attn_probs(tr.q_img, tr.k_txt, tr.valid, 0, 0.0, tr.P, stream),
+                  None, tr.bytes["cross_attn_probs"]),
+        "accumulate": (lambda: sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream), None,
+                       tr.bytes["partition_accumulate"]),
+        "finalize": (lambda: sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s,
+                                                           stream), None, None),
+        "scatter": (lambda: sd.safedit_scatter_state([tr.k_s, tr.v_s], [tr.k_state, tr.v_state], tr.idx_s,
+                                                     tr.k, stream), None, tr.bytes["scatter_state"]),
+        "cfg": (lambda: sd.safedit_sw_cfg(tr.eps_c, tr.eps_u, tr.s, w.gamma_ctx, w.gamma_sens, tr.cfg_out,
+                                          stream), None, tr.bytes["sw_cfg"]),
+        "mask": (lambda: sd.safedit_mask_is_row_constant(extra["mask"], tr.verdict, None, stream), None,
+                 wl.STRESS.N * wl.STRESS.N * 2),
+    }
+    fn, flop, nbytes = fns[args.only]
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(args.reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            times.append((a, b))
+    stream.synchronize()
+    ms = [a.elapsed_time(b) for a, b in times]
+    status = sd.safedit_get_device_status(stream)
+    out = {"only": args.only, "reps": args.reps, "ms": [round(x, 4) for x in ms], "status": status}
+    best = min(ms[1:] if len(ms) > 1 else ms)
+    if flop:
+        out["tflops_best"] = round(flop / (best * 1e-3) / 1e12, 1)
+    if nbytes:
+        out["gbs_best"] = round(nbytes / (best * 1e-3) / 1e9, 1)
+    print(json.dumps(out), flush=True)
+    if status != 0:
+        sys.exit(3)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -430,7 +496,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default=None,
+                    choices=["srsu", "anchor", "xattn", "accumulate", "finalize", "scatter", "cfg", "mask"],
+                    help="run one kernel of the path in isolation (profiling target)")
+    ap.add_argument("--reps", type=int, default=5)
     args = ap.parse_args()
+    if args.only:
+        run_only(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":

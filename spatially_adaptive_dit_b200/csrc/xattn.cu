@@ -35,7 +35,9 @@ struct XCfg {
 
 struct XParams {
   const uint8_t* key_valid;  // [L] of the selected batch entry
-  int L, Lpad, N, b, tmem_cols;
+  float* P;                  // [H,N,L] output (for the L % 4 tail columns)
+  int64_t p_sh, p_sn;        // element strides of P
+  int L, L4, Lpad, N, b, tmem_cols;  // L4 = L rounded down to 4: the TMA-stored columns
   float scale_log2;
   int* status;
   uint64_t wait_limit;
@@ -62,7 +64,7 @@ __global__ void __launch_bounds__(128)
   float* vadd = reinterpret_cast<float*>(tail + 256);  // [256] additive validity
   const uint32_t bar_load = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[1]);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int h = blockIdx.y;
   const int row0 = blockIdx.x * 128;
 
@@ -203,9 +205,18 @@ __global__ void __launch_bounds__(128)
       }
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
-      if (tid == 0) {
+      if (tid == 0 && c * 32 < p.L4) {
+        // the tensor map spans the first L4 columns: TMA stores move whole
+        // 16-byte units, so the last L % 4 columns are written below instead
         tma_store_3d(&tmP, buf, c * 32, row0, h);
         bulk_commit();
+      }
+      if (p.L4 < p.L && row0 + tid < p.N) {
+        for (int e = 0; e < 32; ++e) {
+          const int j = c * 32 + e;
+          if (j >= p.L4 && j < p.L)
+            p.P[h * p.p_sh + int64_t(row0 + tid) * p.p_sn + j] = __uint_as_float(r[e]) * inv;
+        }
       }
     }
     if (tid == 0) bulk_wait<0>();
@@ -266,6 +277,10 @@ extern "C" safedit_status safedit_cross_attn_probs(const safedit_tensor* q_img,
   XParams p{};
   p.key_valid = d_key_valid + int64_t(batch_index) * L;
   p.L = static_cast<int>(L);
+  p.L4 = static_cast<int>(L & ~int64_t(3));
+  p.P = static_cast<float*>(p_out->data);
+  p.p_sh = p_out->strides[0];
+  p.p_sn = p_out->strides[1];
   p.Lpad = static_cast<int>((L + 15) / 16 * 16);
   p.N = static_cast<int>(N);
   p.b = batch_index;
@@ -277,7 +292,7 @@ extern "C" safedit_status safedit_cross_attn_probs(const safedit_tensor* q_img,
   p.wait_limit = wait_limit_ns();
   const int ch = (D % 64 == 0) ? 64 : 32;
   const CUtensorMapSwizzle swz = ch == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  CUtensorMap tq, tk, tp;
+  CUtensorMap tq, tk, tp{};
   {
     const uint64_t dims[4] = {uint64_t(D), uint64_t(N), uint64_t(H), uint64_t(B)};
     const uint64_t str[3] = {uint64_t(q_img->strides[2]) * 2, uint64_t(q_img->strides[1]) * 2,
@@ -296,8 +311,8 @@ extern "C" safedit_status safedit_cross_attn_probs(const safedit_tensor* q_img,
                           swz)) != SAFEDIT_OK)
       return st;
   }
-  {
-    const uint64_t dims[3] = {uint64_t(L), uint64_t(N), uint64_t(H)};
+  if (p.L4 > 0) {
+    const uint64_t dims[3] = {uint64_t(p.L4), uint64_t(N), uint64_t(H)};
     const uint64_t str[2] = {uint64_t(p_out->strides[1]) * 4, uint64_t(p_out->strides[0]) * 4};
     const uint32_t box[3] = {32u, 128u, 1u};
     if ((st = encode_tmap(&tp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p_out->data, dims, str, box,

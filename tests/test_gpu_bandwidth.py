@@ -208,7 +208,7 @@ def test_mask_edge_cases():
             expect_status(0)
             rv, rf = oracle.mask_row_constant(full)
             assert np.array_equal(fl.cpu().numpy(), rf) and int(v.item()) == rv
-            if cols == 5:
+            if cols == 5 and dt == torch.float32:  # the hand verdicts are for fp32 values
                 assert np.array_equal(rf, expect)
     # bool masks, 4-D, with a broadcast head dim (stride 0) and a broadcast query dim
     bm = torch.ones(2, 1, 64, 96, dtype=torch.bool)
