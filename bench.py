@@ -376,29 +376,32 @@ def run_e2e(tr, stream, args):
 
 def cpu_baseline(seconds=12.0, rows=None):
     """The fp64 oracle, as it stands, on the host cores: SRSU attention rows of
-    one (b,h) slice of the workload over all N keys.  Reported in the same
-    unit (TFLOP/s of the SRSU attention)."""
+    the workload (all k = 7680 sensitive rows of one (b,h) slice per call, over
+    all N keys), as many calls as fit in about `seconds` (or exactly `rows`
+    rows).  Reported in the metric's unit (TFLOP/s of SRSU attention)."""
     import numpy as np
     import oracle
     w = W
     g = torch.Generator().manual_seed(4321)
-    q = torch.randn(1024, w.d, generator=g).to(torch.bfloat16).double().numpy()
+    q = torch.randn(w.k, w.d, generator=g).to(torch.bfloat16).double().numpy()
     k = torch.randn(w.N, w.d, generator=g).to(torch.bfloat16).double().numpy()
     v = torch.randn(w.N, w.d, generator=g).to(torch.bfloat16).double().numpy()
-    n = rows or 16
-    dt = 0.0
+    done, dt = 0, 0.0
+    chunk = w.k if rows is None else min(rows, w.k)
+    t_start = time.perf_counter()
     while True:
-        idx = np.arange(n, dtype=np.int32)
-        t0 = time.perf_counter()
-        oracle.attn_subset(q, k, v, idx)
-        dt = time.perf_counter() - t0
-        if rows or dt >= seconds * 0.5 or n >= 1024:
+        n = chunk if rows is None else min(chunk, rows - done)
+        oracle.attn_subset(q, k, v, np.arange(n, dtype=np.int32))
+        done += n
+        dt = time.perf_counter() - t_start
+        if (rows is None and dt >= seconds) or (rows is not None and done >= rows):
             break
-        n = min(1024, max(n * 2, int(n * seconds / max(dt, 1e-3) * 0.9)))
-    flop = 4.0 * n * w.N * w.d
+        if rows is None and done == chunk and dt < seconds / 64:
+            chunk = w.k  # already full slices
+    flop = 4.0 * done * w.N * w.d
     return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{n} SRSU query rows of one (b,h) slice over all N={w.N} keys, d={w.d}, fp64 "
-                      f"({dt:.1f} s)"}
+            "sample": f"{done} SRSU query rows ({done / w.k:.2f} slices of k={w.k}) over all N={w.N} keys, "
+                      f"d={w.d}, fp64, {dt:.1f} s"}
 
 
 def run_reference(args):
@@ -407,8 +410,8 @@ def run_reference(args):
         return
     import oracle  # noqa: F401
     vals = []
-    # calibrate the sample once, then time K steps of that fixed sample
-    cal = cpu_baseline(seconds=4.0)
+    # calibrate the sample once (about 6 s), then time K steps of that fixed sample
+    cal = cpu_baseline(seconds=6.0)
     n_rows = int(cal["sample"].split()[0])
     for i in range(args.warmup + args.steps):
         r = cpu_baseline(rows=n_rows)

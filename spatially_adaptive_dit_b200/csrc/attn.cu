@@ -67,7 +67,22 @@ struct AttnParams {
   uint64_t wait_limit;
 };
 
-constexpr int kAttnThreads = 320;
+// 12 warps: two softmax warpgroups (warps 0-7), then TMA producer (8), MMA
+// issuer (9) and two spare warps (10, 11) completing the third warpgroup, so
+// that setmaxnreg can move registers from the control warpgroup (72 each) to
+// the softmax warpgroups (216 each): 256*216 + 128*72 = 384*168.
+constexpr int kAttnThreads = 384;
+constexpr uint32_t kSoftmaxRegs = 216;
+constexpr uint32_t kControlRegs = 72;
+// Column pairs (bit e of the mask = pair e of each 16-pair group) whose
+// exponentials go to the FMA-pipe polynomial instead of the MUFU unit, on the
+// mask-free path.  Balances the two pipes (measured on B200 at the 2560^2
+// SRSU launch: 1/4 of the pairs is best, 1/2 is slower than none); exact
+// zero weights of kept masks stay on the MUFU path.
+#ifndef SAFEDIT_EXP2_FMA_MASK
+#define SAFEDIT_EXP2_FMA_MASK 0x8888u
+#endif
+constexpr uint32_t kExp2FmaMask = SAFEDIT_EXP2_FMA_MASK;
 constexpr uint64_t kDrainNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -81,6 +96,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_subset_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = AttnCfg<D>;
+  constexpr bool MASKED = PAD || BIAS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -89,7 +105,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t sK = sbase + 2 * C::TILE_BYTES;           // NS tiles
   const uint32_t sV = sK + C::NS * C::TILE_BYTES;          // NS tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_TILES * C::TILE_BYTES);
-  // barrier slots
   const uint32_t b0 = smem_u32(bars);
   auto BAR = [&](int i) { return b0 + 8u * uint32_t(i); };
   const int Q_FULL = 0, K_FULL = 2, K_EMPTY = K_FULL + C::NS, V_FULL = K_EMPTY + C::NS,
@@ -137,6 +152,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp < 8) {
     // ================================================== softmax warpgroups
+    setmaxnreg_inc<kSoftmaxRegs>();
     const int t = warp >> 2;            // query tile
     const int wr = warp & 3;            // TMEM lane quarter
     const int tid = threadIdx.x & 127;  // thread within the warpgroup
@@ -186,18 +202,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         break;
       }
       tc_fence_after();
+      // x = raw scores (mask-free path) or log2-domain logits (kept masks)
       float x[128];
       {
-        uint32_t r[32];
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(tS + 0u, r0);
+        tmem_ld32(tS + 32u, r1);
+        tmem_ld32(tS + 64u, r2);
+        tmem_ld32(tS + 96u, r3);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tS + uint32_t(c * 32), r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]) * sl2;
+        for (int e = 0; e < 32; ++e) {
+          x[e] = __uint_as_float(r0[e]);
+          x[32 + e] = __uint_as_float(r1[e]);
+          x[64 + e] = __uint_as_float(r2[e]);
+          x[96 + e] = __uint_as_float(r3[e]);
         }
       }
       const int key0 = j * C::BN;
+      if (MASKED) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) x[c] *= sl2;
+      }
       if (PAD) {
         const float* pr = p.pad + b * p.pad_sb + key0;
         const int lim = p.Nk - key0;
@@ -263,10 +289,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (c >= lim) x[c] = -INFINITY;
       }
-      float mt = x[0];
+      // row max of the tile (in log2 units)
+      float mt;
+      {
+        float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mt = fmaxf(mt, x[c]);
-      // lazy rescale
+        for (int c = 6; c < 126; c += 4) {
+          m0 = max3(m0, x[c], x[c + 1]);
+          m1 = max3(m1, x[c + 2], x[c + 3]);
+        }
+        mt = max3(m0, m1, fmaxf(x[126], x[127]));
+        if (!MASKED) mt *= sl2;  // sl2 > 0: the max commutes with the scale
+      }
+      // lazy rescale: the running max moves only when it grows by > 2^8
       bool need_o = false;
       float alpha = 1.f;
       if (mt > m_run + kRescaleThreshold) {
@@ -286,21 +321,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_st32(tO + uint32_t(c * 32), r);
         }
       }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float rs = 0.f;
+      const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+      const float mul = MASKED ? 1.f : sl2;
+      const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(neg_m, neg_m);
+      uint64_t sum2 = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2_approx(x[c * 32 + 2 * e] - m_use);
-          const float p1 = ex2_approx(x[c * 32 + 2 * e + 1] - m_use);
-          rs += p0 + p1;
+          const uint64_t a2 = f2_fma(f2_pack(x[c * 32 + 2 * e], x[c * 32 + 2 * e + 1]), mul2, negm2);
+          float a0, a1, p0, p1;
+          f2_unpack(a2, a0, a1);
+          if (!MASKED && ((kExp2FmaMask >> e) & 1u)) {
+            exp2_pair_fma(a0, a1, p0, p1);
+          } else {
+            p0 = ex2_approx(a0);
+            p1 = ex2_approx(a1);
+          }
+          sum2 = f2_add(sum2, f2_pack(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + uint32_t(c * 16), pk);
       }
-      l_run += rs;
+      {
+        float s0, s1;
+        f2_unpack(sum2, s0, s1);
+        l_run += s0 + s1;
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(P_FULL + t));
@@ -333,102 +381,105 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     }
-  } else if (warp == 8) {
-    // ================================================== TMA producer (K, V)
-    if (lane == 0) {
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < nk; ++j) {
-        const int s = j % C::NS;
-        const uint32_t ph = uint32_t((j / C::NS) & 1);
-        if (!wait_bounded(BAR(K_EMPTY + s), ph ^ 1u, ctl)) break;
-        mbar_arrive_expect_tx(BAR(K_FULL + s), C::TILE_BYTES);
-#pragma unroll
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_4d(sK + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmK, BAR(K_FULL + s), c * C::CH,
-                      j * C::BN, h, b);
-        issued_k = j + 1;
-        if (!wait_bounded(BAR(V_EMPTY + s), ph ^ 1u, ctl)) break;
-        mbar_arrive_expect_tx(BAR(V_FULL + s), C::TILE_BYTES);
-#pragma unroll
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_4d(sV + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmV, BAR(V_FULL + s), c * C::CH,
-                      j * C::BN, h, b);
-        issued_v = j + 1;
-      }
-      if (*abort_flag) {  // drain the loads still in flight before leaving
-        for (int j = (issued_k > C::NS ? issued_k - C::NS : 0); j < issued_k; ++j)
-          wait_drain(BAR(K_FULL + j % C::NS), uint32_t((j / C::NS) & 1), kDrainNs);
-        for (int j = (issued_v > C::NS ? issued_v - C::NS : 0); j < issued_v; ++j)
-          wait_drain(BAR(V_FULL + j % C::NS), uint32_t((j / C::NS) & 1), kDrainNs);
-      }
-    }
   } else {
-    // ================================================== MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t tS0 = tmem, tS1 = tmem + 128u;
-      const uint32_t tO0 = tmem + 256u, tO1 = tmem + 256u + uint32_t(D);
-      constexpr uint32_t SBO = 8u * C::ROWB;
-      auto issue_qk = [&](uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+    setmaxnreg_dec<kControlRegs>();
+    if (warp == 8) {
+      // ================================================ TMA producer (K, V)
+      if (lane == 0) {
+        int issued_k = 0, issued_v = 0;
+        for (int j = 0; j < nk; ++j) {
+          const int s = j % C::NS;
+          const uint32_t ph = uint32_t((j / C::NS) & 1);
+          if (!wait_bounded(BAR(K_EMPTY + s), ph ^ 1u, ctl)) break;
+          mbar_arrive_expect_tx(BAR(K_FULL + s), C::TILE_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int chunk = (kk * 16) / C::CH;
-          const uint32_t within = uint32_t(((kk * 16) % C::CH) * 2);
-          const uint32_t off = uint32_t(chunk * C::CHUNK_BYTES) + within;
-          mma_ss(d_tmem, smem_desc(q_smem + off, 16u, SBO, C::LAYOUT),
-                 smem_desc(k_smem + off, 16u, SBO, C::LAYOUT), idesc_qk, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, bool acc) {
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_4d(sK + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmK, BAR(K_FULL + s),
+                        c * C::CH, j * C::BN, h, b);
+          issued_k = j + 1;
+          if (!wait_bounded(BAR(V_EMPTY + s), ph ^ 1u, ctl)) break;
+          mbar_arrive_expect_tx(BAR(V_FULL + s), C::TILE_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          const uint64_t bdesc =
-              smem_desc(v_smem + uint32_t(kk * 16 * C::ROWB), uint32_t(C::CHUNK_BYTES), SBO, C::LAYOUT);
-          mma_ts(d_tmem, p_tmem + uint32_t(kk * 8), bdesc, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_4d(sV + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmV, BAR(V_FULL + s),
+                        c * C::CH, j * C::BN, h, b);
+          issued_v = j + 1;
         }
-      };
-      bool ok = wait_bounded(BAR(Q_FULL + 0), 0u, ctl) && wait_bounded(BAR(Q_FULL + 1), 0u, ctl) &&
-                wait_bounded(BAR(K_FULL + 0), 0u, ctl);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(tS0, sQ, sK);
-        tc_commit(BAR(S_FULL + 0));
-        issue_qk(tS1, sQ + C::TILE_BYTES, sK);
-        tc_commit(BAR(S_FULL + 1));
-        tc_commit(BAR(K_EMPTY + 0));
+        if (*abort_flag) {  // drain the loads still in flight before leaving
+          for (int j = (issued_k > C::NS ? issued_k - C::NS : 0); j < issued_k; ++j)
+            wait_drain(BAR(K_FULL + j % C::NS), uint32_t((j / C::NS) & 1), kDrainNs);
+          for (int j = (issued_v > C::NS ? issued_v - C::NS : 0); j < issued_v; ++j)
+            wait_drain(BAR(V_FULL + j % C::NS), uint32_t((j / C::NS) & 1), kDrainNs);
+        }
       }
-      for (int j = 0; ok && j < nk; ++j) {
-        const int s = j % C::NS;
-        const uint32_t ph = uint32_t((j / C::NS) & 1);
-        const bool more = (j + 1 < nk);
-        const int s1 = (j + 1) % C::NS;
-        const uint32_t ph1 = uint32_t(((j + 1) / C::NS) & 1);
-        if (!(ok = wait_bounded(BAR(V_FULL + s), ph, ctl))) break;
-        if (!(ok = wait_bounded(BAR(P_FULL + 0), uint32_t(j & 1), ctl))) break;
-        tc_fence_after();
-        issue_pv(tO0, tS0, sV + s * C::TILE_BYTES, j > 0);
-        if (more) {
-          if (!(ok = wait_bounded(BAR(K_FULL + s1), ph1, ctl))) break;
+    } else if (warp == 9) {
+      // ================================================ MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+        const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+        const uint32_t tS0 = tmem, tS1 = tmem + 128u;
+        const uint32_t tO0 = tmem + 256u, tO1 = tmem + 256u + uint32_t(D);
+        constexpr uint32_t SBO = 8u * C::ROWB;
+        auto issue_qk = [&](uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int chunk = (kk * 16) / C::CH;
+            const uint32_t within = uint32_t(((kk * 16) % C::CH) * 2);
+            const uint32_t off = uint32_t(chunk * C::CHUNK_BYTES) + within;
+            mma_ss(d_tmem, smem_desc(q_smem + off, 16u, SBO, C::LAYOUT),
+                   smem_desc(k_smem + off, 16u, SBO, C::LAYOUT), idesc_qk, kk > 0 ? 1u : 0u);
+          }
+        };
+        auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, bool acc) {
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk) {
+            const uint64_t bdesc = smem_desc(v_smem + uint32_t(kk * 16 * C::ROWB),
+                                             uint32_t(C::CHUNK_BYTES), SBO, C::LAYOUT);
+            mma_ts(d_tmem, p_tmem + uint32_t(kk * 8), bdesc, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          }
+        };
+        bool ok = wait_bounded(BAR(Q_FULL + 0), 0u, ctl) &&
+                  wait_bounded(BAR(Q_FULL + 1), 0u, ctl) && wait_bounded(BAR(K_FULL + 0), 0u, ctl);
+        if (ok) {
           tc_fence_after();
-          issue_qk(tS0, sQ, sK + s1 * C::TILE_BYTES);
+          issue_qk(tS0, sQ, sK);
           tc_commit(BAR(S_FULL + 0));
-        }
-        if (!(ok = wait_bounded(BAR(P_FULL + 1), uint32_t(j & 1), ctl))) break;
-        tc_fence_after();
-        issue_pv(tO1, tS1, sV + s * C::TILE_BYTES, j > 0);
-        tc_commit(BAR(V_EMPTY + s));
-        if (more) {
-          issue_qk(tS1, sQ + C::TILE_BYTES, sK + s1 * C::TILE_BYTES);
+          issue_qk(tS1, sQ + C::TILE_BYTES, sK);
           tc_commit(BAR(S_FULL + 1));
-          tc_commit(BAR(K_EMPTY + s1));
+          tc_commit(BAR(K_EMPTY + 0));
         }
-      }
-      if (ok) {
-        tc_commit(BAR(O_FULL));
-      } else {  // wait for every MMA already issued before TMEM is freed
-        tc_commit(BAR(DRAIN));
-        wait_drain(BAR(DRAIN), 0u, kDrainNs);
+        for (int j = 0; ok && j < nk; ++j) {
+          const int s = j % C::NS;
+          const uint32_t ph = uint32_t((j / C::NS) & 1);
+          const bool more = (j + 1 < nk);
+          const int s1 = (j + 1) % C::NS;
+          const uint32_t ph1 = uint32_t(((j + 1) / C::NS) & 1);
+          if (!(ok = wait_bounded(BAR(V_FULL + s), ph, ctl))) break;
+          if (!(ok = wait_bounded(BAR(P_FULL + 0), uint32_t(j & 1), ctl))) break;
+          tc_fence_after();
+          issue_pv(tO0, tS0, sV + s * C::TILE_BYTES, j > 0);
+          if (more) {
+            if (!(ok = wait_bounded(BAR(K_FULL + s1), ph1, ctl))) break;
+            tc_fence_after();
+            issue_qk(tS0, sQ, sK + s1 * C::TILE_BYTES);
+            tc_commit(BAR(S_FULL + 0));
+          }
+          if (!(ok = wait_bounded(BAR(P_FULL + 1), uint32_t(j & 1), ctl))) break;
+          tc_fence_after();
+          issue_pv(tO1, tS1, sV + s * C::TILE_BYTES, j > 0);
+          tc_commit(BAR(V_EMPTY + s));
+          if (more) {
+            issue_qk(tS1, sQ + C::TILE_BYTES, sK + s1 * C::TILE_BYTES);
+            tc_commit(BAR(S_FULL + 1));
+            tc_commit(BAR(K_EMPTY + s1));
+          }
+        }
+        if (ok) {
+          tc_commit(BAR(O_FULL));
+        } else {  // wait for every MMA already issued before TMEM is freed
+          tc_commit(BAR(DRAIN));
+          wait_drain(BAR(DRAIN), 0u, kDrainNs);
+        }
       }
     }
   }

@@ -280,4 +280,70 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ------------------------------------------------- packed fp32 pairs ---
+// Blackwell executes one instruction on a pair of fp32 values held in a
+// 64-bit register (halving issue slots of the softmax arithmetic).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// exp2 of a pair on the FMA pipe: 2^x = 2^j 2^f, j = round(x) by the
+// 1.5*2^23 magic add, f = x - j in [-1/2, 1/2], 2^f by a degree-3 polynomial
+// whose coefficients minimise the maximum relative error on [-1/2, 1/2]
+// (Remez exchange, csrc/exp2_poly_fit.py; scheme error <= 7.5e-5 relative,
+// below the 2^-9 rounding of the bf16 probabilities it feeds), and 2^j added
+// into the exponent bits.  Inputs are clamped at -126 (results below 2^-126
+// are not needed: they are far under the rounding of the row sum).
+constexpr float kExp2C0 = 0.999928057f;
+constexpr float kExp2C1 = 0.693260968f;
+constexpr float kExp2C2 = 0.242611125f;
+constexpr float kExp2C3 = 0.0551716685f;
+constexpr float kExp2Magic = 12582912.0f;
+
+__device__ __forceinline__ void exp2_pair_fma(float a, float b, float& ea, float& eb) {
+  a = fmaxf(a, -126.f);
+  b = fmaxf(b, -126.f);
+  const uint64_t x = f2_pack(a, b);
+  const uint64_t t = f2_add(x, f2_pack(kExp2Magic, kExp2Magic));
+  const uint64_t j = f2_add(t, f2_pack(-kExp2Magic, -kExp2Magic));
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  float pa, pb, ta, tb;
+  f2_unpack(p, pa, pb);
+  f2_unpack(t, ta, tb);
+  ea = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
+  eb = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 }  // namespace sd
