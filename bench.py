@@ -235,22 +235,15 @@ def run_ours(args):
     per = {n: [a.elapsed_time(b) for a, b in lst] for n, lst in ev.items()}
     srsu_ms = sum(per["attn_subset_srsu"])
     n_srsu = len(per["attn_subset_srsu"])
-    stats = torch.tensor([total_ms, srsu_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
-    total_ms, srsu_ms = float(stats[0]), float(stats[1])
+    total_ms, srsu_ms = max_over_ranks([total_ms, srsu_ms], dev)
 
     # ---- end to end through the public API with host buffers (pinned)
     e2e = run_e2e(tr, stream, args)
-    if ws > 1:
-        e2e_t = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
-        e2e["ms"] = float(e2e_t[0])
+    e2e["ms"] = max_over_ranks([e2e["ms"]], dev)[0]
 
     if rank == 0:
         hbm, bf16_burst, bf16_sust, src = _peaks()
-        flop_total = tr.flop_srsu * n_srsu * ws
-        value = flop_total / (srsu_ms * 1e-3) / 1e12
+        value = whole_job_tflops(tr.flop_srsu * n_srsu, ws, srsu_ms)
         srsu_call_ms = srsu_ms / n_srsu
         achieved = tr.flop_srsu / (srsu_call_ms * 1e-3) / 1e12
         kern = {}
@@ -282,7 +275,7 @@ def run_ours(args):
                          "unit": "TFLOP/s", "frac": round(achieved / bf16_sust, 4), "traffic": traffic},
             "gpu_launches": launches,
             "device_status": status,
-            "e2e": {"value": round(tr.flop_srsu * n_srsu / args.steps * ws / (e2e["ms"] * 1e-3) / 1e12, 3),
+            "e2e": {"value": round(whole_job_tflops(tr.flop_srsu * n_srsu / args.steps, ws, e2e["ms"]), 3),
                     "unit": "TFLOP/s", "ms_per_step": round(e2e["ms"], 3),
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
             "clocks": clk,
@@ -293,6 +286,22 @@ def run_ours(args):
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def max_over_ranks(values, device):
+    """Element-wise max of a list of floats over all ranks (identity when not
+    distributed).  Works with NCCL (CUDA device) and gloo (CPU)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized() \
+            and torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tflops(flop_per_rank, n_ranks, max_ms):
+    """Weak scaling: every rank runs its own replica, so the job processed
+    n_ranks times the per-rank work in the slowest rank's time."""
+    return flop_per_rank * n_ranks / (max_ms * 1e-3) / 1e12
 
 
 def _ncu_traffic():
@@ -313,65 +322,86 @@ def _ncu_traffic():
 
 
 def run_e2e(tr, stream, args):
-    """Same trajectory, with every denoising step's inputs copied from pinned
-    host memory and each step's guided prediction copied back, inside the
-    timed region."""
+    """Same trajectory through the C ABI with host buffers: every denoising
+    step's inputs are copied from pinned host memory (Q, eps_c, eps_u; the
+    text tensors on the warm-up step; fresh S-row K/V on SRSU steps, full K/V
+    on anchor steps) and each step's guided prediction is copied back, all
+    inside the timed region.  A copy stream fills a second buffer set for
+    step t+1 while step t computes; events order every reuse."""
     w = tr.w
+    names = ("q", "k_s", "v_s", "q_img", "k_txt", "eps_c", "eps_u")
     host = {}
-    for name in ("q", "k_s", "v_s", "k_full", "v_full", "q_img", "k_txt", "eps_c", "eps_u"):
-        t = getattr(tr, name)
-        host[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-        host[name].copy_(t)
-    out_h = torch.empty(tr.cfg_out.shape, dtype=tr.cfg_out.dtype, pin_memory=True)
-    h2d = d2h = 0
+    for n in names + ("k_full", "v_full"):
+        t = getattr(tr, n)
+        host[n] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        host[n].copy_(t)
+    sets = [{n: getattr(tr, n) for n in names}, {n: torch.empty_like(getattr(tr, n)) for n in names}]
+    out_h = [torch.empty(tr.cfg_out.shape, dtype=tr.cfg_out.dtype, pin_memory=True) for _ in range(2)]
+    copy_stream = torch.cuda.Stream(device=tr.dev)
+    sd = tr.sd
+    counts = {"h2d": 0, "d2h": 0}
 
-    def step(count):
-        nonlocal h2d, d2h
-        sd = tr.sd
-        tr.score.zero_()
+    freed = [None, None]  # per buffer set: event after the last step that used it
+
+    def trajectory(count):
+        with torch.cuda.stream(stream):
+            tr.score.zero_()
         for t in range(w.steps):
             anchor = (t % w.period == 0)
-            names = ["q", "eps_c", "eps_u"] + (["q_img", "k_txt"] if t < w.warmup else []) + \
-                (["k_full", "v_full"] if anchor else ["k_s", "v_s"])
-            for n in names:
-                dst = getattr(tr, n)
-                dst.copy_(host[n], non_blocking=True)
+            cur = sets[t % 2]
+            need = ["q", "eps_c", "eps_u"] + (["q_img", "k_txt"] if t < w.warmup else []) + \
+                ([] if anchor else ["k_s", "v_s"])
+            ready = torch.cuda.Event()
+            with torch.cuda.stream(copy_stream):
+                if freed[t % 2] is not None:
+                    copy_stream.wait_event(freed[t % 2])  # step t-2 is done with this set
+                for n in need:
+                    cur[n].copy_(host[n], non_blocking=True)
+                    if count:
+                        counts["h2d"] += host[n].numel() * host[n].element_size()
+                if anchor:
+                    if freed[(t + 1) % 2] is not None:
+                        copy_stream.wait_event(freed[(t + 1) % 2])  # step t-1 still reads the state
+                    for n, dst in (("k_full", tr.k_state), ("v_full", tr.v_state)):
+                        dst.copy_(host[n], non_blocking=True)
+                        if count:
+                            counts["h2d"] += host[n].numel() * host[n].element_size()
+                ready.record(copy_stream)
+            stream.wait_event(ready)
+            with torch.cuda.stream(stream):
+                if t < w.warmup:
+                    sd.safedit_cross_attn_probs(cur["q_img"], cur["k_txt"], tr.valid, 0, 0.0, tr.P, stream)
+                    sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream)
+                if t == w.warmup - 1:
+                    sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s, stream)
+                if t == 0:
+                    sd.safedit_mask_is_row_constant(tr.mask, tr.verdict, None, stream)
+                if anchor:
+                    sd.safedit_attn_subset(cur["q"], tr.k_state, tr.v_state, None, 0, None, None, 0.0,
+                                           tr.o_state, 0, stream)
+                else:
+                    sd.safedit_scatter_state([cur["k_s"], cur["v_s"]], [tr.k_state, tr.v_state], tr.idx_s,
+                                             tr.k, stream)
+                    sd.safedit_attn_subset(cur["q"], tr.k_state, tr.v_state, tr.idx_s, tr.k, None, None,
+                                           0.0, tr.o_state, 1, stream)
+                g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx
+                sd.safedit_sw_cfg(cur["eps_c"], cur["eps_u"], tr.s, w.gamma_ctx, g_sens, tr.cfg_out, stream)
+                out_h[t % 2].copy_(tr.cfg_out, non_blocking=True)
                 if count:
-                    h2d += host[n].numel() * host[n].element_size()
-            if t < w.warmup:
-                sd.safedit_cross_attn_probs(tr.q_img, tr.k_txt, tr.valid, 0, 0.0, tr.P, stream)
-                sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream)
-            if t == w.warmup - 1:
-                sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s, stream)
-            if t == 0:
-                sd.safedit_mask_is_row_constant(tr.mask, tr.verdict, None, stream)
-            if anchor:
-                tr.k_state, tr.k_full = tr.k_full, tr.k_state
-                tr.v_state, tr.v_full = tr.v_full, tr.v_state
-                sd.safedit_attn_subset(tr.q, tr.k_state, tr.v_state, None, 0, None, None, 0.0,
-                                       tr.o_state, 0, stream)
-            else:
-                sd.safedit_scatter_state([tr.k_s, tr.v_s], [tr.k_state, tr.v_state], tr.idx_s, tr.k,
-                                         stream)
-                sd.safedit_attn_subset(tr.q, tr.k_state, tr.v_state, tr.idx_s, tr.k, None, None, 0.0,
-                                       tr.o_state, 1, stream)
-            g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx
-            sd.safedit_sw_cfg(tr.eps_c, tr.eps_u, tr.s, w.gamma_ctx, g_sens, tr.cfg_out, stream)
-            out_h.copy_(tr.cfg_out, non_blocking=True)
-            if count:
-                d2h += out_h.numel() * out_h.element_size()
+                    counts["d2h"] += out_h[t % 2].numel() * out_h[t % 2].element_size()
+                ev = torch.cuda.Event()
+                ev.record(stream)
+                freed[t % 2] = ev
 
-    with torch.cuda.stream(stream):
-        step(False)
-        stream.synchronize()
-        n = max(1, min(args.steps, 5))
-        torch.cuda.synchronize()
-        t0 = time.perf_counter()
-        for _ in range(n):
-            step(True)
-        stream.synchronize()
-        ms = (time.perf_counter() - t0) * 1e3 / n
-    return {"ms": ms, "h2d": h2d // n, "d2h": d2h // n}
+    trajectory(False)
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 5))
+    t0 = time.perf_counter()
+    for _ in range(n):
+        trajectory(True)
+    torch.cuda.synchronize()
+    ms = (time.perf_counter() - t0) * 1e3 / n
+    return {"ms": ms, "h2d": counts["h2d"] // n, "d2h": counts["d2h"] // n}
 
 
 def cpu_baseline(seconds=12.0, rows=None):
@@ -447,6 +477,11 @@ def run_only(args):
         sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s, stream)
     stream.synchronize()
     extra = {}
+    if args.only == "cfg" and args.cfg_f != w.F:
+        # bandwidth sweep of the guidance combine at a wider prediction (synthetic)
+        tr.eps_c, tr.eps_u = wl.cfg_preds(w, device=dev, F=args.cfg_f)
+        tr.cfg_out = torch.empty_like(tr.eps_c)
+        tr.bytes["sw_cfg"] = 3 * w.N * args.cfg_f * 4 + 4 * w.N
     if args.only == "mask":
         extra["mask"] = torch.zeros(1, 1, wl.STRESS.N, wl.STRESS.N, dtype=torch.bfloat16, device=dev)
     fns = {
@@ -481,6 +516,8 @@ def run_only(args):
     ms = [a.elapsed_time(b) for a, b in times]
     status = sd.safedit_get_device_status(stream)
     out = {"only": args.only, "reps": args.reps, "ms": [round(x, 4) for x in ms], "status": status}
+    if args.only == "cfg":
+        out["F"] = args.cfg_f
     best = min(ms[1:] if len(ms) > 1 else ms)
     if flop:
         out["tflops_best"] = round(flop / (best * 1e-3) / 1e12, 1)
@@ -503,6 +540,7 @@ def main():
                     choices=["srsu", "anchor", "xattn", "accumulate", "finalize", "scatter", "cfg", "mask"],
                     help="run one kernel of the path in isolation (profiling target)")
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--cfg-f", type=int, default=W.F, help="prediction width for --only cfg")
     args = ap.parse_args()
     if args.only:
         run_only(args)

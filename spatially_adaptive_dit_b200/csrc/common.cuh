@@ -57,6 +57,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared control block of a pipelined CTA: an abort flag that every role
 // polls while it waits, the wait limit, and the global status word.
 struct WaitCtl {
@@ -67,9 +79,15 @@ struct WaitCtl {
 
 // Bounded wait on one mbarrier phase by the calling thread.  Returns false if
 // the CTA aborted or the limit passed (then the abort flag is raised and the
-// status word records the timeout).
+// status word records the timeout).  The first probe does not block, so a
+// limit of 0 gives up on exactly the waits that are not already satisfied.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitCtl& c) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
+  if (c.limit_ns == 0) {
+    *c.abort_flag = 1;
+    set_status(c.status, SAFEDIT_ERR_TIMEOUT);
+    return false;
+  }
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;

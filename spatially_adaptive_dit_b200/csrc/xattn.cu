@@ -29,24 +29,33 @@ struct XCfg {
   static constexpr int Q_BYTES = NCH * Q_CHUNK;
   static constexpr int K_CHUNK = 256 * ROWB;  // room for L <= 256 rows
   static constexpr int K_BYTES = NCH * K_CHUNK;
-  static constexpr int STAGE_BYTES = 128 * 128;  // 128 rows x 32 f32
-  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + K_BYTES + 2 * STAGE_BYTES + 256 + 1024;
+  static constexpr int STAGE_BYTES = Q_BYTES + K_BYTES;  // one Q tile + one text block
+  static constexpr int NSTAGE = (D == 128) ? 1 : 2;
+  static constexpr int OUT_BYTES = 128 * 128;          // 128 rows x 32 f32
+  static constexpr int SMEM_BYTES =
+      1024 + NSTAGE * STAGE_BYTES + 4 * OUT_BYTES + 256 + 1024;
 };
 
 struct XParams {
   const uint8_t* key_valid;  // [L] of the selected batch entry
   float* P;                  // [H,N,L] output (for the L % 4 tail columns)
   int64_t p_sh, p_sn;        // element strides of P
-  int L, L4, Lpad, N, b, tmem_cols;  // L4 = L rounded down to 4: the TMA-stored columns
+  int L, L4, Lpad, N, H, b;  // L4 = L rounded down to 4: the TMA-stored columns
+  int tiles;                 // 128-row tiles per head
+  int units;                 // H * tiles
   float scale_log2;
   int* status;
   uint64_t wait_limit;
 };
 
 constexpr float kXLog2e = 1.4426950408889634f;
+constexpr uint64_t kXDrainNs = 1000000000ull;
 
+// Persistent: CTA c owns a contiguous range of (head, 128-row tile) units.
+// Warps 0-3 and 4-7: two softmax warpgroups taking alternate units, each on
+// its own 256-column TMEM accumulator; warp 8: TMA producer; warp 9: MMA.
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(320, 1)
     xattn_probs_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmKt,
                        const __grid_constant__ CUtensorMap tmP, const XParams p) {
@@ -54,30 +63,36 @@ __global__ void __launch_bounds__(128)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const uint32_t sQ = smem_u32(smem);
-  const uint32_t sK = sQ + C::Q_BYTES;
-  const uint32_t sStage = sK + C::K_BYTES;
-  uint8_t* tail = smem + C::Q_BYTES + C::K_BYTES + 2 * C::STAGE_BYTES;
+  const uint32_t sStage = smem_u32(smem);
+  const uint32_t sOut = sStage + C::NSTAGE * C::STAGE_BYTES;  // 4 staging buffers
+  uint8_t* tail = smem + C::NSTAGE * C::STAGE_BYTES + 4 * C::OUT_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + 32);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tail + 40);
+  // bars: [0,2) stage_full, [2,4) stage_empty, [4,6) s_full, [6,8) s_empty, 8 drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + 96);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tail + 104);
   float* vadd = reinterpret_cast<float*>(tail + 256);  // [256] additive validity
-  const uint32_t bar_load = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[1]);
+  auto BAR = [&](int i) { return smem_u32(&bars[i]); };
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int h = blockIdx.y;
-  const int row0 = blockIdx.x * 128;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int per = p.units / int(gridDim.x), extra = p.units % int(gridDim.x);
+  const int u0 = int(blockIdx.x) * per + min(int(blockIdx.x), extra);
+  const int n_local = per + (int(blockIdx.x) < extra ? 1 : 0);
 
   if (tid == 0) {
-    mbar_init(bar_load, 1);
-    mbar_init(bar_mma, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(0 + i), 1);
+      mbar_init(BAR(2 + i), 1);
+      mbar_init(BAR(4 + i), 1);
+      mbar_init(BAR(6 + i), 128);
+    }
+    mbar_init(BAR(8), 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  for (int j = tid; j < 256; j += 128)
+  for (int j = tid; j < 256; j += blockDim.x)
     vadd[j] = (j < p.L && p.key_valid[j] != 0) ? 0.f : -INFINITY;
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), uint32_t(p.tmem_cols));
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_slot), 512u);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -86,159 +101,205 @@ __global__ void __launch_bounds__(128)
   const uint32_t tmem = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.status, p.wait_limit};
 
-  bool ok = true;
-  if (tid == 0) {
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmKt);
-    mbar_arrive_expect_tx(bar_load, uint32_t(C::Q_BYTES + C::NCH * p.Lpad * C::ROWB));
-#pragma unroll
-    for (int c = 0; c < C::NCH; ++c) {
-      tma_load_4d(sQ + c * C::Q_CHUNK, &tmQ, bar_load, c * C::CH, row0, h, p.b);
-      tma_load_4d(sK + c * C::K_CHUNK, &tmKt, bar_load, c * C::CH, 0, h, p.b);
-    }
-    if (wait_bounded(bar_load, 0u, ctl)) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(128, p.Lpad, 0, 0);
-      constexpr uint32_t SBO = 8u * C::ROWB;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const int chunk = (kk * 16) / C::CH;
-        const uint32_t within = uint32_t(((kk * 16) % C::CH) * 2);
-        mma_ss(tmem, smem_desc(sQ + chunk * C::Q_CHUNK + within, 16u, SBO, C::LAYOUT),
-               smem_desc(sK + chunk * C::K_CHUNK + within, 16u, SBO, C::LAYOUT), idesc,
-               kk > 0 ? 1u : 0u);
-      }
-      tc_commit(bar_mma);
-    } else {
-      wait_drain(bar_load, 0u, 1000000000ull);
-    }
-  }
-  ok = wait_warp(bar_mma, 0u, ctl);
-
-  if (ok) {
-    tc_fence_after();
-    const uint32_t tl = tmem + (uint32_t(warp * 32) << 16);
-    const int nc = p.Lpad / 32 + ((p.Lpad % 32) ? 1 : 0);  // 32-column chunks (Lpad % 16 == 0)
+  if (warp < 8) {
+    // ============================================= softmax warpgroups
+    const int w = warp >> 2, wq = warp & 3, r = tid & 127;
+    const uint32_t tl = tmem + uint32_t(w * 256) + (uint32_t(wq * 32) << 16);
+    const int nc = p.Lpad / 32 + ((p.Lpad % 32) ? 1 : 0);
     const float sl2 = p.scale_log2;
-    // pass 1: row max over valid keys
-    float m = -INFINITY;
-    for (int c = 0; c < nc; ++c) {
-      const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
-      uint32_t r[32];
-      if (ncol == 32) {
-        tmem_ld32(tl + uint32_t(c * 32), r);
-      } else {
-        uint32_t r16[16];
-        tmem_ld16(tl + uint32_t(c * 32), r16);
+    int nstore = 0;  // TMA stores issued by this warpgroup (staging buffer = nstore & 1)
+    for (int i = w; i < n_local; i += 2) {
+      const int u = u0 + i, h = u / p.tiles, tile = u - h * p.tiles;
+      const int row0 = tile * 128;
+      if (!wait_warp(BAR(4 + w), uint32_t((i >> 1) & 1), ctl)) break;
+      tc_fence_after();
+      // pass 1: row max over valid keys
+      float m = -INFINITY;
+      for (int c = 0; c < nc; ++c) {
+        const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
+        uint32_t v[32];
+        if (ncol == 32) {
+          tmem_ld32(tl + uint32_t(c * 32), v);
+        } else {
+          uint32_t v16[16];
+          tmem_ld16(tl + uint32_t(c * 32), v16);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = r16[e];
-      }
-      tmem_wait_ld();
+          for (int e = 0; e < 16; ++e) v[e] = v16[e];
+        }
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (e < ncol) m = fmaxf(m, fmaf(__uint_as_float(r[e]), sl2, vadd[c * 32 + e]));
-    }
-    const float m_use = (m == -INFINITY) ? 0.f : m;
-    // pass 2: exponentials (written back to TMEM) and their sum
-    float sum = 0.f;
-    for (int c = 0; c < nc; ++c) {
-      const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
-      uint32_t r[32];
-      if (ncol == 32) {
-        tmem_ld32(tl + uint32_t(c * 32), r);
-      } else {
-        uint32_t r16[16];
-        tmem_ld16(tl + uint32_t(c * 32), r16);
+        for (int e = 0; e < 32; ++e)
+          if (e < ncol) m = fmaxf(m, fmaf(__uint_as_float(v[e]), sl2, vadd[c * 32 + e]));
+      }
+      const float m_use = (m == -INFINITY) ? 0.f : m;
+      // pass 2: exponentials (written back to TMEM) and their sum
+      float sum = 0.f;
+      for (int c = 0; c < nc; ++c) {
+        const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
+        uint32_t v[32];
+        if (ncol == 32) {
+          tmem_ld32(tl + uint32_t(c * 32), v);
+        } else {
+          uint32_t v16[16];
+          tmem_ld16(tl + uint32_t(c * 32), v16);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = r16[e];
-      }
-      tmem_wait_ld();
+          for (int e = 0; e < 16; ++e) v[e] = v16[e];
+        }
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float ev =
-            (e < ncol) ? ex2_approx(fmaf(__uint_as_float(r[e]), sl2, vadd[c * 32 + e]) - m_use)
-                       : 0.f;
-        sum += ev;
-        r[e] = __float_as_uint(ev);
-      }
-      if (ncol == 32) {
-        tmem_st32(tl + uint32_t(c * 32), r);
-      } else {
-        uint32_t r16[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r16[e] = r[e];
-        tmem_st16(tl + uint32_t(c * 32), r16);
-      }
-    }
-    tmem_wait_st();
-    if (!(sum > 0.f) && row0 + tid < p.N) set_status(p.status, SAFEDIT_ERR_MASKED_ROW);
-    const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
-    // pass 3: normalise, stage (128B swizzle) and store 128 x 32 boxes
-    for (int c = 0; c < nc; ++c) {
-      const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
-      uint32_t r[32];
-      if (ncol == 32) {
-        tmem_ld32(tl + uint32_t(c * 32), r);
-      } else {
-        uint32_t r16[16];
-        tmem_ld16(tl + uint32_t(c * 32), r16);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = r16[e];
-#pragma unroll
-        for (int e = 16; e < 32; ++e) r[e] = 0u;
-      }
-      tmem_wait_ld();
-      const uint32_t buf = sStage + uint32_t((c & 1) * C::STAGE_BYTES);
-      if (c >= 2) {
-        if (tid == 0) bulk_wait_read<1>();
-        named_bar_sync(1, 128);
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t off = uint32_t(tid * 128 + ((u ^ (tid & 7)) * 16));
-        const float a0 = __uint_as_float(r[4 * u]) * inv, a1 = __uint_as_float(r[4 * u + 1]) * inv,
-                    a2 = __uint_as_float(r[4 * u + 2]) * inv,
-                    a3 = __uint_as_float(r[4 * u + 3]) * inv;
-        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(buf + off), "f"(a0),
-                     "f"(a1), "f"(a2), "f"(a3)
-                     : "memory");
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (tid == 0 && c * 32 < p.L4) {
-        // the tensor map spans the first L4 columns: TMA stores move whole
-        // 16-byte units, so the last L % 4 columns are written below instead
-        tma_store_3d(&tmP, buf, c * 32, row0, h);
-        bulk_commit();
-      }
-      if (p.L4 < p.L && row0 + tid < p.N) {
         for (int e = 0; e < 32; ++e) {
-          const int j = c * 32 + e;
-          if (j >= p.L4 && j < p.L)
-            p.P[h * p.p_sh + int64_t(row0 + tid) * p.p_sn + j] = __uint_as_float(r[e]) * inv;
+          const float ev =
+              (e < ncol) ? ex2_approx(fmaf(__uint_as_float(v[e]), sl2, vadd[c * 32 + e]) - m_use)
+                         : 0.f;
+          sum += ev;
+          v[e] = __float_as_uint(ev);
+        }
+        if (ncol == 32) {
+          tmem_st32(tl + uint32_t(c * 32), v);
+        } else {
+          uint32_t v16[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v16[e] = v[e];
+          tmem_st16(tl + uint32_t(c * 32), v16);
+        }
+      }
+      tmem_wait_st();
+      if (!(sum > 0.f) && row0 + r < p.N) set_status(p.status, SAFEDIT_ERR_MASKED_ROW);
+      const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
+      // pass 3: normalise, stage (128B swizzle) and store 128 x 32 boxes
+      for (int c = 0; c < nc; ++c) {
+        const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
+        uint32_t v[32];
+        if (ncol == 32) {
+          tmem_ld32(tl + uint32_t(c * 32), v);
+        } else {
+          uint32_t v16[16];
+          tmem_ld16(tl + uint32_t(c * 32), v16);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = v16[e];
+#pragma unroll
+          for (int e = 16; e < 32; ++e) v[e] = 0u;
+        }
+        tmem_wait_ld();
+        if (c == nc - 1) {  // the accumulator is free for the next unit
+          tc_fence_before();
+          mbar_arrive(BAR(6 + w));
+        }
+        const uint32_t buf = sOut + uint32_t((w * 2 + (nstore & 1)) * C::OUT_BYTES);
+        if (nstore >= 2) {
+          if (r == 0) bulk_wait_read<1>();
+          named_bar_sync(1 + w, 128);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t off = uint32_t(r * 128 + ((q ^ (r & 7)) * 16));
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(buf + off),
+                       "f"(__uint_as_float(v[4 * q]) * inv), "f"(__uint_as_float(v[4 * q + 1]) * inv),
+                       "f"(__uint_as_float(v[4 * q + 2]) * inv),
+                       "f"(__uint_as_float(v[4 * q + 3]) * inv)
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1 + w, 128);
+        if (c * 32 < p.L4) {
+          // the tensor map spans the first L4 columns: TMA stores move whole
+          // 16-byte units, so the last L % 4 columns are written below instead
+          if (r == 0) {
+            tma_store_3d(&tmP, buf, c * 32, row0, h);
+            bulk_commit();
+          }
+          ++nstore;
+        }
+        if (p.L4 < p.L && row0 + r < p.N) {
+          for (int e = 0; e < 32; ++e) {
+            const int j = c * 32 + e;
+            if (j >= p.L4 && j < p.L)
+              p.P[h * p.p_sh + int64_t(row0 + r) * p.p_sn + j] = __uint_as_float(v[e]) * inv;
+          }
         }
       }
     }
-    if (tid == 0) bulk_wait<0>();
+    if (r == 0) bulk_wait<0>();
+  } else if (warp == 8) {
+    // ============================================= TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmKt);
+      int khead[2] = {-1, -1};
+      int issued = 0;
+      for (int i = 0; i < n_local; ++i) {
+        const int st = i % C::NSTAGE;
+        const uint32_t ph = uint32_t((i / C::NSTAGE) & 1);
+        if (!wait_bounded(BAR(2 + st), ph ^ 1u, ctl)) break;
+        const int u = u0 + i, h = u / p.tiles, tile = u - h * p.tiles;
+        const bool newk = khead[st] != h;
+        const uint32_t sQ = sStage + uint32_t(st * C::STAGE_BYTES), sK = sQ + C::Q_BYTES;
+        mbar_arrive_expect_tx(BAR(0 + st),
+                              uint32_t(C::Q_BYTES + (newk ? C::NCH * p.Lpad * C::ROWB : 0)));
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          tma_load_4d(sQ + c * C::Q_CHUNK, &tmQ, BAR(0 + st), c * C::CH, tile * 128, h, p.b);
+          if (newk) tma_load_4d(sK + c * C::K_CHUNK, &tmKt, BAR(0 + st), c * C::CH, 0, h, p.b);
+        }
+        khead[st] = h;
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        for (int i = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); i < issued; ++i)
+          wait_drain(BAR(0 + i % C::NSTAGE), uint32_t((i / C::NSTAGE) & 1), kXDrainNs);
+      }
+    }
+  } else {
+    // ============================================= MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, p.Lpad, 0, 0);
+      constexpr uint32_t SBO = 8u * C::ROWB;
+      bool ok = true;
+      for (int i = 0; i < n_local && ok; ++i) {
+        const int st = i % C::NSTAGE, buf = i & 1;
+        if (!(ok = wait_bounded(BAR(0 + st), uint32_t((i / C::NSTAGE) & 1), ctl))) break;
+        if (!(ok = wait_bounded(BAR(6 + buf), uint32_t(((i >> 1) & 1) ^ 1), ctl))) break;
+        tc_fence_after();
+        const uint32_t sQ = sStage + uint32_t(st * C::STAGE_BYTES), sK = sQ + C::Q_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int chunk = (kk * 16) / C::CH;
+          const uint32_t within = uint32_t(((kk * 16) % C::CH) * 2);
+          mma_ss(tmem + uint32_t(buf * 256),
+                 smem_desc(sQ + chunk * C::Q_CHUNK + within, 16u, SBO, C::LAYOUT),
+                 smem_desc(sK + chunk * C::K_CHUNK + within, 16u, SBO, C::LAYOUT), idesc,
+                 kk > 0 ? 1u : 0u);
+        }
+        tc_commit(BAR(4 + buf));
+        tc_commit(BAR(2 + st));
+      }
+      if (!ok) {
+        tc_commit(BAR(8));
+        wait_drain(BAR(8), 0u, kXDrainNs);
+      }
+    }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 8) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, uint32_t(p.tmem_cols));
+    tmem_dealloc(tmem, 512u);
   }
 }
 
 template <int D>
 static safedit_status launch_x(const CUtensorMap& a, const CUtensorMap& k, const CUtensorMap& pm,
-                               const XParams& p, int H, cudaStream_t s) {
+                               const XParams& p, cudaStream_t s) {
   auto kern = xattn_probs_kernel<D>;
   safedit_status st = set_smem(reinterpret_cast<const void*>(kern), XCfg<D>::SMEM_BYTES);
   if (st != SAFEDIT_OK) return st;
-  dim3 grid((p.N + 127) / 128, H);
-  kern<<<grid, 128, XCfg<D>::SMEM_BYTES, s>>>(a, k, pm, p);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = p.units < sms ? p.units : sms;
+  kern<<<grid, 320, XCfg<D>::SMEM_BYTES, s>>>(a, k, pm, p);
   return after_launch(1);
 }
 
@@ -283,10 +344,11 @@ extern "C" safedit_status safedit_cross_attn_probs(const safedit_tensor* q_img,
   p.p_sn = p_out->strides[1];
   p.Lpad = static_cast<int>((L + 15) / 16 * 16);
   p.N = static_cast<int>(N);
+  p.H = static_cast<int>(H);
   p.b = batch_index;
-  int cols = 32;
-  while (cols < p.Lpad) cols <<= 1;
-  p.tmem_cols = cols;
+  p.tiles = static_cast<int>((N + 127) / 128);
+  if (int64_t(p.tiles) * H > INT32_MAX) return SAFEDIT_ERR_SHAPE;
+  p.units = p.tiles * p.H;
   const float sc = (scale > 0.f) ? scale : 1.0f / std::sqrt(static_cast<float>(D));
   p.scale_log2 = sc * kXLog2e;
   p.wait_limit = wait_limit_ns();
@@ -323,8 +385,8 @@ extern "C" safedit_status safedit_cross_attn_probs(const safedit_tensor* q_img,
   if (!p.status) return SAFEDIT_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {
-    case 64: return launch_x<64>(tq, tk, tp, p, static_cast<int>(H), s);
-    case 96: return launch_x<96>(tq, tk, tp, p, static_cast<int>(H), s);
-    default: return launch_x<128>(tq, tk, tp, p, static_cast<int>(H), s);
+    case 64: return launch_x<64>(tq, tk, tp, p, s);
+    case 96: return launch_x<96>(tq, tk, tp, p, s);
+    default: return launch_x<128>(tq, tk, tp, p, s);
   }
 }

@@ -1,0 +1,69 @@
+"""Failure detection without a GPU fault: with the debug wait limit at 0 the
+pipelined kernels' bounded waits give up at once; each CTA then raises its
+abort flag, drains its in-flight TMA loads and MMAs, frees TMEM and returns,
+and the status word reports SAFEDIT_ERR_TIMEOUT.  The context must stay
+usable: the next call with the normal limit reproduces the reference output
+bit for bit."""
+import pytest
+import torch
+
+from tests.gpu_util import expect_status, sd
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _attn_case():
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(1, 4, 1024, 96, generator=g).to(torch.bfloat16).to(DEV)
+    k = torch.randn(1, 4, 1024, 96, generator=g).to(torch.bfloat16).to(DEV)
+    v = torch.randn(1, 4, 1024, 96, generator=g).to(torch.bfloat16).to(DEV)
+    idx = torch.arange(0, 1024, 3, dtype=torch.int32, device=DEV)
+    return q, k, v, idx
+
+
+def _run_attn(q, k, v, idx):
+    out = torch.zeros(1, 4, idx.numel(), 96, dtype=torch.bfloat16, device=DEV)
+    sd().safedit_attn_subset(q, k, v, idx, idx.numel(), None, None, 0.0, out, 0)
+    return out
+
+
+def _run_xattn():
+    g = torch.Generator().manual_seed(6)
+    qi = torch.randn(1, 4, 2048, 96, generator=g).to(torch.bfloat16).to(DEV)
+    kt = torch.randn(1, 4, 256, 96, generator=g).to(torch.bfloat16).to(DEV)
+    valid = torch.ones(1, 256, dtype=torch.uint8, device=DEV)
+    P = torch.zeros(4, 2048, 256, device=DEV)
+    sd().safedit_cross_attn_probs(qi, kt, valid, 0, 0.0, P)
+    return P
+
+
+def test_bounded_wait_timeout_is_reported_and_context_survives():
+    q, k, v, idx = _attn_case()
+    ref = _run_attn(q, k, v, idx)
+    ref_p = _run_xattn()
+    expect_status(0)
+    old = sd().safedit_debug_set_wait_limit_ns(0)
+    try:
+        _run_attn(q, k, v, idx)
+        expect_status(sd().ERR_TIMEOUT)
+        _run_xattn()
+        expect_status(sd().ERR_TIMEOUT)
+    finally:
+        sd().safedit_debug_set_wait_limit_ns(old)
+    again = _run_attn(q, k, v, idx)
+    again_p = _run_xattn()
+    expect_status(0)
+    assert torch.equal(again, ref)
+    assert torch.equal(again_p, ref_p)
+
+
+def test_device_errors_do_not_poison_later_calls():
+    q, k, v, idx = _attn_case()
+    ref = _run_attn(q, k, v, idx)
+    bad = idx.clone()
+    bad[0] = 10 ** 6
+    _run_attn(q, k, v, bad)
+    expect_status(sd().ERR_INDEX)
+    assert torch.equal(_run_attn(q, k, v, idx), ref)
+    expect_status(0)
