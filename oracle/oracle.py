@@ -232,6 +232,53 @@ def is_anchor_step(t: int, warmup: int, period: int) -> bool:
     return t < warmup or (t % period == 0)
 
 
+def trajectory(steps, warmup, period, k, gamma_ctx, gamma_sens):
+    """The SRSU / CAR schedule [SAFE-DiT summary, 방법론 2-4], composed from
+    C1-C8.  `steps` is a list of per-step dicts of inputs (numpy / torch):
+      q, k_full, v_full: [B,H,N,d]; k_s, v_s: [B,H,k,d] (fresh sensitive rows);
+      q_img, k_txt: [B,H,N,d] / [B,H,L,d], key_valid [B,L], content [L]
+      (warm-up steps); eps_c, eps_u: [N,F].
+    Warm-up steps (t < warmup) are dense and accumulate the PCSP score from
+    the cond branch (b = 0); the split follows the last warm-up step; then
+    step t is an anchor when t % period == 0 (full refresh of K/V/O state),
+    otherwise SRSU: K_state[S] <- K_S, V_state[S] <- V_S, O_state[S] <-
+    attention of the S rows over the merged state.  Every step ends with the
+    guidance combine (global gamma_ctx until the split exists).
+    Returns dict(idx_s, s, score, k_state, v_state, o_state, cfg=[per step])."""
+    score = None
+    idx_s = s = None
+    k_state = v_state = o_state = None
+    cfg = []
+    for t, st in enumerate(steps):
+        if t < warmup:
+            kv = _u8(st["key_valid"])
+            P = cross_attn_probs(_f64(st["q_img"])[0], _f64(st["k_txt"])[0], kv[0])
+            score = partition_accumulate(P, st["content"], score)
+        if t == warmup - 1:
+            idx_s, _, s = partition_select(score, k)
+        q = _f64(st["q"])
+        B, H, N, d = q.shape
+        if is_anchor_step(t, warmup, period):
+            k_state = _f64(st["k_full"]).copy()
+            v_state = _f64(st["v_full"]).copy()
+            o_state = np.empty_like(q)
+            for b in range(B):
+                for h in range(H):
+                    o_state[b, h] = attn_dense(q[b, h], k_state[b, h], v_state[b, h])
+        else:
+            ks, vs = _f64(st["k_s"]), _f64(st["v_s"])
+            for b in range(B):
+                for h in range(H):
+                    k_state[b, h] = scatter_rows(ks[b, h], k_state[b, h], idx_s)
+                    v_state[b, h] = scatter_rows(vs[b, h], v_state[b, h], idx_s)
+                    rows = attn_subset(q[b, h], k_state[b, h], v_state[b, h], idx_s)
+                    o_state[b, h] = scatter_rows(rows, o_state[b, h], idx_s)
+        sv = s if s is not None else np.zeros(N, dtype=np.float32)
+        g_sens = gamma_sens if t >= warmup else gamma_ctx
+        cfg.append(sw_cfg(st["eps_c"], st["eps_u"], sv, gamma_ctx, g_sens))
+    return dict(idx_s=idx_s, s=s, score=score, k_state=k_state, v_state=v_state, o_state=o_state, cfg=cfg)
+
+
 __all__ = ["OracleError", "lib", "num_threads", "default_scale", "cross_attn_probs",
            "partition_accumulate", "partition_select", "mask_row_constant", "attn_subset",
-           "attn_dense", "scatter_rows", "gather_rows", "sw_cfg", "is_anchor_step"]
+           "attn_dense", "scatter_rows", "gather_rows", "sw_cfg", "is_anchor_step", "trajectory"]

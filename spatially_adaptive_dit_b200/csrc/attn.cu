@@ -292,13 +292,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // row max of the tile (in log2 units)
       float mt;
       {
-        float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
+        // four independent max chains (latency), three-input max (issue)
+        float m0 = fmaxf(x[0], x[1]), m1 = fmaxf(x[2], x[3]), m2 = fmaxf(x[4], x[5]),
+              m3 = fmaxf(x[6], x[7]);
 #pragma unroll
-        for (int c = 6; c < 126; c += 4) {
+        for (int c = 8; c < 128; c += 8) {
           m0 = max3(m0, x[c], x[c + 1]);
           m1 = max3(m1, x[c + 2], x[c + 3]);
+          m2 = max3(m2, x[c + 4], x[c + 5]);
+          m3 = max3(m3, x[c + 6], x[c + 7]);
         }
-        mt = max3(m0, m1, fmaxf(x[126], x[127]));
+        mt = fmaxf(max3(m0, m1, m2), m3);
         if (!MASKED) mt *= sl2;  // sl2 > 0: the max commutes with the scale
       }
       // lazy rescale: the running max moves only when it grows by > 2^8
@@ -324,7 +328,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
       const float mul = MASKED ? 1.f : sl2;
       const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(neg_m, neg_m);
-      uint64_t sum2 = f2_pack(0.f, 0.f);
+      // four independent partial sums: the row sum is not one serial chain
+      uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -339,14 +344,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             p0 = ex2_approx(a0);
             p1 = ex2_approx(a1);
           }
-          sum2 = f2_add(sum2, f2_pack(p0, p1));
+          sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + uint32_t(c * 16), pk);
       }
       {
         float s0, s1;
-        f2_unpack(sum2, s0, s1);
+        f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
         l_run += s0 + s1;
       }
       tmem_wait_st();

@@ -7,7 +7,7 @@
 // One CTA = 128 image rows of one head, 128 threads (thread = row = TMEM
 // lane).  TMA brings the Q tile and the whole text-key block (L <= 256) into
 // swizzled shared memory; one elected thread issues tcgen05.mma for
-// S = Q K^T (M=128, N=L rounded up to 16) into TMEM; the softmax runs in
+// S = Q K^T (M=128, N=L rounded up to 32) into TMEM; the softmax runs in
 // three TMEM passes (max; exp + sum with the exponentials written back to
 // TMEM; scale) and the probabilities leave through a double-buffered,
 // 128B-swizzled shared-memory stage and TMA tensor stores, so the 4-byte
@@ -30,10 +30,14 @@ struct XCfg {
   static constexpr int K_CHUNK = 256 * ROWB;  // room for L <= 256 rows
   static constexpr int K_BYTES = NCH * K_CHUNK;
   static constexpr int STAGE_BYTES = Q_BYTES + K_BYTES;  // one Q tile + one text block
-  static constexpr int NSTAGE = (D == 128) ? 1 : 2;
+  // One load stage: the next unit's loads still overlap the current unit's
+  // softmax (the MMA frees the stage long before the softmax ends); the smem
+  // goes to staging so that more TMA stores stay in flight.
+  static constexpr int NSTAGE = 1;
+  static constexpr int NOUT = 4;                       // staging buffers per warpgroup
   static constexpr int OUT_BYTES = 128 * 128;          // 128 rows x 32 f32
   static constexpr int SMEM_BYTES =
-      1024 + NSTAGE * STAGE_BYTES + 4 * OUT_BYTES + 256 + 1024;
+      1024 + NSTAGE * STAGE_BYTES + 2 * NOUT * OUT_BYTES + 256 + 1024;
 };
 
 struct XParams {
@@ -64,8 +68,8 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sStage = smem_u32(smem);
-  const uint32_t sOut = sStage + C::NSTAGE * C::STAGE_BYTES;  // 4 staging buffers
-  uint8_t* tail = smem + C::NSTAGE * C::STAGE_BYTES + 4 * C::OUT_BYTES;
+  const uint32_t sOut = sStage + C::NSTAGE * C::STAGE_BYTES;  // 2 x NOUT staging buffers
+  uint8_t* tail = smem + C::NSTAGE * C::STAGE_BYTES + 2 * C::NOUT * C::OUT_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
   // bars: [0,2) stage_full, [2,4) stage_empty, [4,6) s_full, [6,8) s_empty, 8 drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + 96);
@@ -105,9 +109,17 @@ __global__ void __launch_bounds__(320, 1)
     // ============================================= softmax warpgroups
     const int w = warp >> 2, wq = warp & 3, r = tid & 127;
     const uint32_t tl = tmem + uint32_t(w * 256) + (uint32_t(wq * 32) << 16);
-    const int nc = p.Lpad / 32 + ((p.Lpad % 32) ? 1 : 0);
+    const int nc = p.Lpad / 32;  // 32-column chunks (Lpad is a multiple of 32)
+    // chunks with at least one valid key; all-padding chunks are written as
+    // zeros without touching TMEM or the exponential unit
+    uint32_t vmask = 0;
+    for (int c = 0; c < nc; ++c) {
+      bool any = false;
+      for (int e = 0; e < 32; ++e) any |= (vadd[c * 32 + e] == 0.f);
+      if (any) vmask |= 1u << c;
+    }
     const float sl2 = p.scale_log2;
-    int nstore = 0;  // TMA stores issued by this warpgroup (staging buffer = nstore & 1)
+    int nstore = 0;  // TMA stores issued by this warpgroup (staging buffer = nstore % NOUT)
     for (int i = w; i < n_local; i += 2) {
       const int u = u0 + i, h = u / p.tiles, tile = u - h * p.tiles;
       const int row0 = tile * 128;
@@ -115,88 +127,96 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       // pass 1: row max over valid keys
       float m = -INFINITY;
-      for (int c = 0; c < nc; ++c) {
-        const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
-        uint32_t v[32];
-        if (ncol == 32) {
-          tmem_ld32(tl + uint32_t(c * 32), v);
-        } else {
-          uint32_t v16[16];
-          tmem_ld16(tl + uint32_t(c * 32), v16);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = v16[e];
-        }
+#pragma unroll 1
+      for (int c = 0; c < nc; c += 2) {
+        const bool a = (vmask >> c) & 1u, b2 = (c + 1 < nc) && ((vmask >> (c + 1)) & 1u);
+        if (!a && !b2) continue;
+        uint32_t v0[32], v1[32];
+        // both chunks are loaded (a pair never leaves the 256-column accumulator)
+        tmem_ld32(tl + uint32_t(c * 32), v0);
+        tmem_ld32(tl + uint32_t((c + 1) * 32), v1);
         tmem_wait_ld();
+        if (a) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (e < ncol) m = fmaxf(m, fmaf(__uint_as_float(v[e]), sl2, vadd[c * 32 + e]));
+          for (int e = 0; e < 32; ++e)
+            m = fmaxf(m, fmaf(__uint_as_float(v0[e]), sl2, vadd[c * 32 + e]));
+        }
+        if (b2) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            m = fmaxf(m, fmaf(__uint_as_float(v1[e]), sl2, vadd[(c + 1) * 32 + e]));
+        }
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
       // pass 2: exponentials (written back to TMEM) and their sum
-      float sum = 0.f;
-      for (int c = 0; c < nc; ++c) {
-        const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
-        uint32_t v[32];
-        if (ncol == 32) {
-          tmem_ld32(tl + uint32_t(c * 32), v);
-        } else {
-          uint32_t v16[16];
-          tmem_ld16(tl + uint32_t(c * 32), v16);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = v16[e];
-        }
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < nc; c += 2) {
+        const bool a = (vmask >> c) & 1u, b2 = (c + 1 < nc) && ((vmask >> (c + 1)) & 1u);
+        if (!a && !b2) continue;
+        uint32_t v0[32], v1[32];
+        // both chunks are loaded (a pair never leaves the 256-column accumulator)
+        tmem_ld32(tl + uint32_t(c * 32), v0);
+        tmem_ld32(tl + uint32_t((c + 1) * 32), v1);
         tmem_wait_ld();
+        if (a) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float ev =
-              (e < ncol) ? ex2_approx(fmaf(__uint_as_float(v[e]), sl2, vadd[c * 32 + e]) - m_use)
-                         : 0.f;
-          sum += ev;
-          v[e] = __float_as_uint(ev);
+          for (int e = 0; e < 32; ++e) {
+            const float ev = ex2_approx(fmaf(__uint_as_float(v0[e]), sl2, vadd[c * 32 + e]) - m_use);
+            sum0 += ev;
+            v0[e] = __float_as_uint(ev);
+          }
+          tmem_st32(tl + uint32_t(c * 32), v0);
         }
-        if (ncol == 32) {
-          tmem_st32(tl + uint32_t(c * 32), v);
-        } else {
-          uint32_t v16[16];
+        if (b2) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v16[e] = v[e];
-          tmem_st16(tl + uint32_t(c * 32), v16);
+          for (int e = 0; e < 32; ++e) {
+            const float ev =
+                ex2_approx(fmaf(__uint_as_float(v1[e]), sl2, vadd[(c + 1) * 32 + e]) - m_use);
+            sum1 += ev;
+            v1[e] = __float_as_uint(ev);
+          }
+          tmem_st32(tl + uint32_t((c + 1) * 32), v1);
         }
       }
       tmem_wait_st();
+      const float sum = sum0 + sum1;
       if (!(sum > 0.f) && row0 + r < p.N) set_status(p.status, SAFEDIT_ERR_MASKED_ROW);
       const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
       // pass 3: normalise, stage (128B swizzle) and store 128 x 32 boxes
+      int last_valid = -1;
+      for (int c = 0; c < nc; ++c)
+        if ((vmask >> c) & 1u) last_valid = c;
+      if (last_valid < 0) {  // no TMEM read in this pass: the accumulator is free now
+        tc_fence_before();
+        mbar_arrive(BAR(6 + w));
+      }
+#pragma unroll 1
       for (int c = 0; c < nc; ++c) {
-        const int ncol = (p.Lpad - c * 32) >= 32 ? 32 : 16;
         uint32_t v[32];
-        if (ncol == 32) {
+        if ((vmask >> c) & 1u) {
           tmem_ld32(tl + uint32_t(c * 32), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv);
+          if (c == last_valid) {  // the accumulator is free for the next unit
+            tc_fence_before();
+            mbar_arrive(BAR(6 + w));
+          }
         } else {
-          uint32_t v16[16];
-          tmem_ld16(tl + uint32_t(c * 32), v16);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = v16[e];
-#pragma unroll
-          for (int e = 16; e < 32; ++e) v[e] = 0u;
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
         }
-        tmem_wait_ld();
-        if (c == nc - 1) {  // the accumulator is free for the next unit
-          tc_fence_before();
-          mbar_arrive(BAR(6 + w));
-        }
-        const uint32_t buf = sOut + uint32_t((w * 2 + (nstore & 1)) * C::OUT_BYTES);
-        if (nstore >= 2) {
-          if (r == 0) bulk_wait_read<1>();
+        const uint32_t buf = sOut + uint32_t((w * C::NOUT + (nstore % C::NOUT)) * C::OUT_BYTES);
+        if (nstore >= C::NOUT) {
+          if (r == 0) bulk_wait_read<C::NOUT - 1>();
           named_bar_sync(1 + w, 128);
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const uint32_t off = uint32_t(r * 128 + ((q ^ (r & 7)) * 16));
-          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(buf + off),
-                       "f"(__uint_as_float(v[4 * q]) * inv), "f"(__uint_as_float(v[4 * q + 1]) * inv),
-                       "f"(__uint_as_float(v[4 * q + 2]) * inv),
-                       "f"(__uint_as_float(v[4 * q + 3]) * inv)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + off), "r"(v[4 * q]),
+                       "r"(v[4 * q + 1]), "r"(v[4 * q + 2]), "r"(v[4 * q + 3])
                        : "memory");
         }
         fence_proxy_async_smem();
@@ -214,7 +234,7 @@ __global__ void __launch_bounds__(320, 1)
           for (int e = 0; e < 32; ++e) {
             const int j = c * 32 + e;
             if (j >= p.L4 && j < p.L)
-              p.P[h * p.p_sh + int64_t(row0 + r) * p.p_sn + j] = __uint_as_float(v[e]) * inv;
+              p.P[h * p.p_sh + int64_t(row0 + r) * p.p_sn + j] = __uint_as_float(v[e]);
           }
         }
       }
@@ -342,7 +362,7 @@ extern "C" safedit_status safedit_cross_attn_probs(const safedit_tensor* q_img,
   p.P = static_cast<float*>(p_out->data);
   p.p_sh = p_out->strides[0];
   p.p_sn = p_out->strides[1];
-  p.Lpad = static_cast<int>((L + 15) / 16 * 16);
+  p.Lpad = static_cast<int>((L + 31) / 32 * 32);  // MMA N and TMEM chunks of 32 columns
   p.N = static_cast<int>(N);
   p.H = static_cast<int>(H);
   p.b = batch_index;
