@@ -69,11 +69,11 @@ struct AttnParams {
 
 // 12 warps: two softmax warpgroups (warps 0-7), then TMA producer (8), MMA
 // issuer (9) and two spare warps (10, 11) completing the third warpgroup, so
-// that setmaxnreg can move registers from the control warpgroup (72 each) to
-// the softmax warpgroups (216 each): 256*216 + 128*72 = 384*168.
+// that setmaxnreg can move registers from the control warpgroup (88 each) to
+// the softmax warpgroups (208 each): 256*208 + 128*88 = 384*168.
 constexpr int kAttnThreads = 384;
-constexpr uint32_t kSoftmaxRegs = 216;
-constexpr uint32_t kControlRegs = 72;
+constexpr uint32_t kSoftmaxRegs = 208;
+constexpr uint32_t kControlRegs = 88;
 // Column pairs (bit e of the mask = pair e of each 16-pair group) whose
 // exponentials go to the FMA-pipe polynomial instead of the MUFU unit, on the
 // mask-free path.  Balances the two pipes (measured on B200 at the 2560^2
@@ -425,31 +425,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t tS0 = tmem, tS1 = tmem + 128u;
         const uint32_t tO0 = tmem + 256u, tO1 = tmem + 256u + uint32_t(D);
         constexpr uint32_t SBO = 8u * C::ROWB;
-        auto issue_qk = [&](uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+        // Descriptors are built once; per MMA only the 16-byte address field
+        // of the low word advances (all smem offsets here stay below 256 KB,
+        // so the field never carries into the other fields).
+        const uint64_t qd0 = smem_desc(sQ, 16u, SBO, C::LAYOUT);
+        const uint64_t qd1 = smem_desc(sQ + C::TILE_BYTES, 16u, SBO, C::LAYOUT);
+        const uint64_t kd0 = smem_desc(sK, 16u, SBO, C::LAYOUT);
+        const uint64_t vd0 = smem_desc(sV, uint32_t(C::CHUNK_BYTES), SBO, C::LAYOUT);
+        auto adv = [](uint64_t d, uint32_t bytes) {
+          return (d & 0xFFFFFFFF00000000ull) | uint64_t(uint32_t(d) + (bytes >> 4));
+        };
+        auto issue_qk = [&](uint32_t d_tmem, uint64_t qd, uint64_t kd) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const int chunk = (kk * 16) / C::CH;
-            const uint32_t within = uint32_t(((kk * 16) % C::CH) * 2);
-            const uint32_t off = uint32_t(chunk * C::CHUNK_BYTES) + within;
-            mma_ss(d_tmem, smem_desc(q_smem + off, 16u, SBO, C::LAYOUT),
-                   smem_desc(k_smem + off, 16u, SBO, C::LAYOUT), idesc_qk, kk > 0 ? 1u : 0u);
+            const uint32_t off = uint32_t(((kk * 16) / C::CH) * C::CHUNK_BYTES + ((kk * 16) % C::CH) * 2);
+            mma_ss(d_tmem, adv(qd, off), adv(kd, off), idesc_qk, kk > 0 ? 1u : 0u);
           }
         };
-        auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, bool acc) {
+        auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint64_t vd, bool acc) {
 #pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk) {
-            const uint64_t bdesc = smem_desc(v_smem + uint32_t(kk * 16 * C::ROWB),
-                                             uint32_t(C::CHUNK_BYTES), SBO, C::LAYOUT);
-            mma_ts(d_tmem, p_tmem + uint32_t(kk * 8), bdesc, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < C::BN / 16; ++kk)
+            mma_ts(d_tmem, p_tmem + uint32_t(kk * 8), adv(vd, uint32_t(kk * 16 * C::ROWB)), idesc_pv,
+                   (acc || kk > 0) ? 1u : 0u);
         };
         bool ok = wait_bounded(BAR(Q_FULL + 0), 0u, ctl) &&
                   wait_bounded(BAR(Q_FULL + 1), 0u, ctl) && wait_bounded(BAR(K_FULL + 0), 0u, ctl);
         if (ok) {
           tc_fence_after();
-          issue_qk(tS0, sQ, sK);
+          issue_qk(tS0, qd0, kd0);
           tc_commit(BAR(S_FULL + 0));
-          issue_qk(tS1, sQ + C::TILE_BYTES, sK);
+          issue_qk(tS1, qd1, kd0);
           tc_commit(BAR(S_FULL + 1));
           tc_commit(BAR(K_EMPTY + 0));
         }
@@ -462,19 +467,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!(ok = wait_bounded(BAR(V_FULL + s), ph, ctl))) break;
           if (!(ok = wait_bounded(BAR(P_FULL + 0), uint32_t(j & 1), ctl))) break;
           tc_fence_after();
-          issue_pv(tO0, tS0, sV + s * C::TILE_BYTES, j > 0);
+          issue_pv(tO0, tS0, adv(vd0, uint32_t(s * C::TILE_BYTES)), j > 0);
           if (more) {
             if (!(ok = wait_bounded(BAR(K_FULL + s1), ph1, ctl))) break;
             tc_fence_after();
-            issue_qk(tS0, sQ, sK + s1 * C::TILE_BYTES);
+            issue_qk(tS0, qd0, adv(kd0, uint32_t(s1 * C::TILE_BYTES)));
             tc_commit(BAR(S_FULL + 0));
           }
           if (!(ok = wait_bounded(BAR(P_FULL + 1), uint32_t(j & 1), ctl))) break;
           tc_fence_after();
-          issue_pv(tO1, tS1, sV + s * C::TILE_BYTES, j > 0);
+          issue_pv(tO1, tS1, adv(vd0, uint32_t(s * C::TILE_BYTES)), j > 0);
           tc_commit(BAR(V_EMPTY + s));
           if (more) {
-            issue_qk(tS1, sQ + C::TILE_BYTES, sK + s1 * C::TILE_BYTES);
+            issue_qk(tS1, qd1, adv(kd0, uint32_t(s1 * C::TILE_BYTES)));
             tc_commit(BAR(S_FULL + 1));
             tc_commit(BAR(K_EMPTY + s1));
           }

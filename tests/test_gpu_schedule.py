@@ -66,7 +66,9 @@ def test_tiny_trajectory_matches_oracle_schedule(w):
     steps = _inputs(w)
     gpu = _gpu_trajectory(w, steps)
     ref = oracle.trajectory(steps, w.warmup, w.period, w.k, w.gamma_ctx, w.gamma_sens)
-    assert np.abs(gpu["score"] - ref["score"]).max() <= 1e-12 * np.abs(ref["score"]).max()
+    # the GPU aggregates its own fp32 probabilities (bf16 inputs, fp32 MMA and
+    # exponentials), the oracle its fp64 ones: the scores agree to ~1e-7
+    assert np.abs(gpu["score"] - ref["score"]).max() <= 1e-5 * np.abs(ref["score"]).max()
     # the split: exact except tokens within 1e-6 relative of the threshold score
     tau = np.sort(ref["score"])[::-1][w.k - 1]
     near = set(np.nonzero(np.abs(ref["score"] - tau) <= 1e-6 * abs(tau))[0].tolist())
