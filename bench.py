@@ -493,6 +493,8 @@ def run_only(args):
                   None, tr.bytes["cross_attn_probs"]),
         "accumulate": (lambda: sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream), None,
                        tr.bytes["partition_accumulate"]),
+        "pcsp": (lambda: sd.safedit_pcsp_score(tr.q_img, tr.k_txt, tr.valid, tr.content, 0, 0.0, tr.score,
+                                               stream), None, W.H * W.N * W.d * 2 + W.H * W.L * W.d * 2),
         "finalize": (lambda: sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s,
                                                            stream), None, None),
         "scatter": (lambda: sd.safedit_scatter_state([tr.k_s, tr.v_s], [tr.k_state, tr.v_state], tr.idx_s,
@@ -537,7 +539,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,
-                    choices=["srsu", "anchor", "xattn", "accumulate", "finalize", "scatter", "cfg", "mask"],
+                    choices=["srsu", "anchor", "xattn", "accumulate", "pcsp", "finalize", "scatter", "cfg",
+                             "mask"],
                     help="run one kernel of the path in isolation (profiling target)")
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--cfg-f", type=int, default=W.F, help="prediction width for --only cfg")

@@ -125,6 +125,27 @@ safedit_status safedit_partition_finalize(const double *d_score, int32_t n,
                                           void *stream);
 
 /* ------------------------------------------------------------------------
+ * Fused PCSP score: cross-attention probabilities and their aggregation in
+ * one pass, without materialising P.  [P1 방법론 2 / P4 Metodologia 2];
+ * [P3 B.1 step 3].  Same result as safedit_cross_attn_probs followed by
+ * safedit_partition_accumulate (up to fp32 rounding of the probabilities):
+ *
+ *   d_score[i] += sum_h ( sum_{j valid, content} e_hij / sum_{j valid} e_hij ),
+ *   e_hij = exp(scale q_img[b,h,i,:] . k_txt[b,h,j,:] - max_j(...)),  b = batch_index.
+ *
+ * q_img [B,H,N,d] bf16, d in {64,96,128}; k_txt [B,H,L,d] bf16, L <= 256;
+ * d_key_valid [B*L] u8; d_content [L] u8; d_score [N] f64 (in/out, fp64
+ * accumulation, each row's heads summed inside one CTA: deterministic).
+ * scale: 0 selects 1/sqrt(d).  A row with no valid key sets
+ * SAFEDIT_ERR_MASKED_ROW and adds nothing.
+ */
+safedit_status safedit_pcsp_score(const safedit_tensor *q_img,
+                                  const safedit_tensor *k_txt,
+                                  const uint8_t *d_key_valid,
+                                  const uint8_t *d_content, int32_t batch_index,
+                                  float scale, double *d_score, void *stream);
+
+/* ------------------------------------------------------------------------
  * Exact mask-elision criterion.  [P1 방법론 1 / P4 Metodologia 1]: an additive
  * mask whose effect on the logits is a per-row constant c_i (L_{i,:} + c_i)
  * leaves softmax unchanged and may be removed; text padding, causal and

@@ -29,7 +29,7 @@ F32, BF16, F16, BOOL, I32, F64, U8 = range(7)
 _DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16, torch.bool: BOOL,
           torch.int32: I32, torch.float64: F64, torch.uint8: U8}
 
-EXPORTED = ("safedit_cross_attn_probs", "safedit_partition_accumulate",
+EXPORTED = ("safedit_cross_attn_probs", "safedit_partition_accumulate", "safedit_pcsp_score",
             "safedit_partition_finalize", "safedit_mask_is_row_constant", "safedit_attn_subset",
             "safedit_scatter_state", "safedit_gather_rows", "safedit_sw_cfg",
             "safedit_get_device_status", "safedit_status_string", "safedit_kernel_launch_count",
@@ -55,6 +55,7 @@ _f32 = ctypes.c_float
 _lib.safedit_cross_attn_probs.argtypes = [_T, _T, _vp, _i32, _f32, _T, _vp]
 _lib.safedit_partition_accumulate.argtypes = [_T, _vp, _vp, _vp]
 _lib.safedit_partition_finalize.argtypes = [_vp, _i32, _i32, _vp, _vp, _vp, _vp]
+_lib.safedit_pcsp_score.argtypes = [_T, _T, _vp, _vp, _i32, _f32, _vp, _vp]
 _lib.safedit_mask_is_row_constant.argtypes = [_T, _vp, _vp, _vp]
 _lib.safedit_attn_subset.argtypes = [_T, _T, _T, _vp, _i32, _T, _T, _f32, _T, _i32, _vp]
 _lib.safedit_scatter_state.argtypes = [_T, _T, _i32, _vp, _i32, _vp]
@@ -123,6 +124,12 @@ def safedit_cross_attn_probs(q_img, k_txt, key_valid, batch_index, scale, p_out,
 def safedit_partition_accumulate(p, content, score, stream=None):
     _check(_lib.safedit_partition_accumulate(_ref(p), _ptr(content), _ptr(score), _stream(stream)),
            "safedit_partition_accumulate")
+
+
+def safedit_pcsp_score(q_img, k_txt, key_valid, content, batch_index, scale, score, stream=None):
+    _check(_lib.safedit_pcsp_score(_ref(q_img), _ref(k_txt), _ptr(key_valid), _ptr(content),
+                                   int(batch_index), float(scale), _ptr(score), _stream(stream)),
+           "safedit_pcsp_score")
 
 
 def safedit_partition_finalize(score, n, k, idx_s, idx_c, s, stream=None):
