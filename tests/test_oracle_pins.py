@@ -307,3 +307,58 @@ def test_sw_cfg_special_cases():
     got = oracle.sw_cfg(c, u, sb, 2.0, 7.5)
     gam = np.where(sb > 0, 7.5, 2.0)[:, None]
     assert np.abs(got - (u + gam * (c.astype(np.float64) - u))).max() <= 1e-14
+
+
+# ---------------------------------------------------------------------------
+# Schedule (C9): SAFE-DiT summary 방법론 2-3 (warm-up, fixed split, SRSU/CAR).
+# ---------------------------------------------------------------------------
+def _tiny_steps(B, H, N, d, L, k, steps, same_kv):
+    out = []
+    for t in range(steps):
+        q, kf, vf = rng.standard_normal((B, H, N, d)), rng.standard_normal((B, H, N, d)), \
+            rng.standard_normal((B, H, N, d))
+        if same_kv:  # every step sees the same K/V: the cached context is never stale
+            kf, vf = out[0]["k_full"] if out else kf, out[0]["v_full"] if out else vf
+        out.append(dict(q=q, k_full=kf, v_full=vf, k_s=None, v_s=None,
+                        q_img=rng.standard_normal((B, H, N, d)), k_txt=rng.standard_normal((B, H, L, d)),
+                        key_valid=np.ones((B, L), dtype=np.uint8), content=np.ones(L, dtype=np.uint8),
+                        eps_c=rng.standard_normal((N, 4)), eps_u=rng.standard_normal((N, 4))))
+    return out
+
+
+def test_trajectory_srsu_rows_equal_dense_when_context_is_fresh():
+    """If the cached context equals the current K/V, an SRSU step's S rows are
+    the dense anchor's rows (S queries attend to the global K/V), and C rows
+    keep the previous anchor's output."""
+    B, H, N, d, L, k = 1, 2, 40, 8, 6, 12
+    steps = _tiny_steps(B, H, N, d, L, k, 3, same_kv=True)
+    warm = oracle.trajectory(steps[:1], 1, 5, k, 2.0, 4.0)
+    idx = warm["idx_s"]
+    for st in steps:
+        st["k_s"] = st["k_full"][:, :, idx]
+        st["v_s"] = st["v_full"][:, :, idx]
+    res = oracle.trajectory(steps[:2], 1, 5, k, 2.0, 4.0)  # t=0 anchor, t=1 SRSU
+    for h in range(H):
+        dense1 = oracle.attn_dense(steps[1]["q"][0, h], steps[1]["k_full"][0, h], steps[1]["v_full"][0, h])
+        dense0 = oracle.attn_dense(steps[0]["q"][0, h], steps[0]["k_full"][0, h], steps[0]["v_full"][0, h])
+        assert np.abs(res["o_state"][0, h][idx] - dense1[idx]).max() <= 1e-13
+        c = np.setdiff1d(np.arange(N), idx)
+        assert np.array_equal(res["o_state"][0, h][c], dense0[c])
+    # guidance: global before the split exists, sensitivity-weighted after it
+    s = res["s"].astype(np.float64)
+    g = 2.0 + 2.0 * s
+    u, cc = steps[1]["eps_u"], steps[1]["eps_c"]
+    assert np.abs(res["cfg"][1] - (u + g[:, None] * (cc - u))).max() <= 1e-14
+    assert np.abs(res["cfg"][0] - (steps[0]["eps_u"] + 2.0 * (steps[0]["eps_c"] - steps[0]["eps_u"]))).max() <= 1e-14
+
+
+def test_trajectory_anchor_refreshes_everything():
+    B, H, N, d, L, k = 1, 1, 24, 4, 5, 6
+    steps = _tiny_steps(B, H, N, d, L, k, 3, same_kv=False)
+    for st in steps:
+        st["k_s"] = rng.standard_normal((B, H, k, d))
+        st["v_s"] = rng.standard_normal((B, H, k, d))
+    res = oracle.trajectory(steps, 1, 2, k, 1.0, 1.0)  # t=0 anchor, t=1 SRSU, t=2 anchor
+    assert np.array_equal(res["k_state"], steps[2]["k_full"])
+    dense = oracle.attn_dense(steps[2]["q"][0, 0], steps[2]["k_full"][0, 0], steps[2]["v_full"][0, 0])
+    assert np.array_equal(res["o_state"][0, 0], dense)
