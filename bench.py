@@ -231,6 +231,7 @@ def run_ours(args):
         torch.distributed.barrier()
     clk = clocks.stop()
     status = sd.safedit_get_device_status(stream)
+    peak_gb = torch.cuda.max_memory_allocated(dev) / 1e9
     total_ms = t0.elapsed_time(t1)
     per = {n: [a.elapsed_time(b) for a, b in lst] for n, lst in ev.items()}
     srsu_ms = sum(per["attn_subset_srsu"])
@@ -274,6 +275,10 @@ def run_ours(args):
                          "peak": bf16_sust, "peak_kind": f"bf16_tflops_sustained ({src})",
                          "unit": "TFLOP/s", "frac": round(achieved / bf16_sust, 4), "traffic": traffic},
             "gpu_launches": launches,
+            "memory": {"peak_allocated_gb": round(peak_gb, 2),
+                       "note": "all buffers of the attention path incl. the 0.63 GB probability tensor; "
+                               "a dense masked path that materialises bf16 scores [B,H,N,N] would need "
+                               f"{W.B * W.H * W.N * W.N * 2 / 1e9:.1f} GB for them alone"},
             "device_status": status,
             "e2e": {"value": round(whole_job_tflops(tr.flop_srsu * n_srsu / args.steps, ws, e2e["ms"]), 3),
                     "unit": "TFLOP/s", "ms_per_step": round(e2e["ms"], 3),
@@ -322,25 +327,32 @@ def _ncu_traffic():
 
 
 def run_e2e(tr, stream, args):
-    """Same trajectory through the C ABI with host buffers: every denoising
-    step's inputs are copied from pinned host memory (Q, eps_c, eps_u; the
-    text tensors on the warm-up step; fresh S-row K/V on SRSU steps, full K/V
-    on anchor steps) and each step's guided prediction is copied back, all
-    inside the timed region.  A copy stream fills a second buffer set for
-    step t+1 while step t computes; events order every reuse."""
+    """Same trajectory through the C ABI with host buffers.  Every denoising
+    step's inputs are copied from pinned host memory and its guided
+    prediction copied back, inside the timed region: on the warm-up step the
+    text tensors, on anchor steps the full Q, K, V, and on SRSU steps only the
+    fresh S rows -- Q_S, K_S, V_S compact [B,H,k,d] (the projections of an
+    SRSU step run on the S rows alone) -- plus eps_c, eps_u every step.  An
+    SRSU step is then: scatter K_S, V_S into the cached state, attention of the
+    compact Q_S over all N keys, scatter O_S into O_state.  A copy stream fills
+    a second buffer set for step t+1 while step t computes; events order every
+    buffer reuse."""
     w = tr.w
-    names = ("q", "k_s", "v_s", "q_img", "k_txt", "eps_c", "eps_u")
+    names = ("q", "q_s", "k_s", "v_s", "q_img", "k_txt", "eps_c", "eps_u")
+    q_s = tr.q[:, :, : tr.k].contiguous()
+    o_s = torch.empty_like(q_s)
+    dev_t = {"q_s": q_s}
     host = {}
     for n in names + ("k_full", "v_full"):
-        t = getattr(tr, n)
+        t = dev_t.get(n, getattr(tr, n, None))
         host[n] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
         host[n].copy_(t)
-    sets = [{n: getattr(tr, n) for n in names}, {n: torch.empty_like(getattr(tr, n)) for n in names}]
+    sets = [{n: dev_t.get(n, getattr(tr, n, None)) for n in names},
+            {n: torch.empty_like(host[n], device=tr.dev) for n in names}]
     out_h = [torch.empty(tr.cfg_out.shape, dtype=tr.cfg_out.dtype, pin_memory=True) for _ in range(2)]
     copy_stream = torch.cuda.Stream(device=tr.dev)
     sd = tr.sd
     counts = {"h2d": 0, "d2h": 0}
-
     freed = [None, None]  # per buffer set: event after the last step that used it
 
     def trajectory(count):
@@ -349,8 +361,8 @@ def run_e2e(tr, stream, args):
         for t in range(w.steps):
             anchor = (t % w.period == 0)
             cur = sets[t % 2]
-            need = ["q", "eps_c", "eps_u"] + (["q_img", "k_txt"] if t < w.warmup else []) + \
-                ([] if anchor else ["k_s", "v_s"])
+            need = ["eps_c", "eps_u"] + (["q_img", "k_txt"] if t < w.warmup else []) + \
+                (["q"] if anchor else ["q_s", "k_s", "v_s"])
             ready = torch.cuda.Event()
             with torch.cuda.stream(copy_stream):
                 if freed[t % 2] is not None:
@@ -382,8 +394,9 @@ def run_e2e(tr, stream, args):
                 else:
                     sd.safedit_scatter_state([cur["k_s"], cur["v_s"]], [tr.k_state, tr.v_state], tr.idx_s,
                                              tr.k, stream)
-                    sd.safedit_attn_subset(cur["q"], tr.k_state, tr.v_state, tr.idx_s, tr.k, None, None,
-                                           0.0, tr.o_state, 1, stream)
+                    sd.safedit_attn_subset(cur["q_s"], tr.k_state, tr.v_state, None, 0, None, None, 0.0,
+                                           o_s, 0, stream)
+                    sd.safedit_scatter_state([o_s], [tr.o_state], tr.idx_s, tr.k, stream)
                 g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx
                 sd.safedit_sw_cfg(cur["eps_c"], cur["eps_u"], tr.s, w.gamma_ctx, g_sens, tr.cfg_out, stream)
                 out_h[t % 2].copy_(tr.cfg_out, non_blocking=True)
@@ -477,11 +490,13 @@ def run_only(args):
         sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s, stream)
     stream.synchronize()
     extra = {}
-    if args.only == "cfg" and args.cfg_f != w.F:
+    if args.only in ("cfg", "stepcache") and args.cfg_f != w.F:
         # bandwidth sweep of the guidance combine at a wider prediction (synthetic)
         tr.eps_c, tr.eps_u = wl.cfg_preds(w, device=dev, F=args.cfg_f)
         tr.cfg_out = torch.empty_like(tr.eps_c)
         tr.bytes["sw_cfg"] = 3 * w.N * args.cfg_f * 4 + 4 * w.N
+    if args.only == "stepcache":  # predictions of the previous full step: distinct tensors
+        extra["prev_c"], extra["prev_u"] = wl.cfg_preds(w, step=1, device=dev, F=tr.eps_c.shape[1])
     if args.only == "mask":
         extra["mask"] = torch.zeros(1, 1, wl.STRESS.N, wl.STRESS.N, dtype=torch.bfloat16, device=dev)
     fns = {
@@ -503,6 +518,10 @@ def run_only(args):
                                           stream), None, tr.bytes["sw_cfg"]),
         "mask": (lambda: sd.safedit_mask_is_row_constant(extra["mask"], tr.verdict, None, stream), None,
                  wl.STRESS.N * wl.STRESS.N * 2),
+        "stepcache": (lambda: sd.safedit_stepcache_sw_cfg(extra["prev_c"], tr.eps_c, extra["prev_u"], tr.eps_u,
+                                                          tr.s, 0.5, w.gamma_ctx, w.gamma_sens, tr.cfg_out,
+                                                          stream),
+                      None, 5 * tr.eps_c.numel() * 4 + 4 * w.N),
     }
     fn, flop, nbytes = fns[args.only]
     times = []
@@ -518,7 +537,7 @@ def run_only(args):
     ms = [a.elapsed_time(b) for a, b in times]
     status = sd.safedit_get_device_status(stream)
     out = {"only": args.only, "reps": args.reps, "ms": [round(x, 4) for x in ms], "status": status}
-    if args.only == "cfg":
+    if args.only in ("cfg", "stepcache"):
         out["F"] = args.cfg_f
     best = min(ms[1:] if len(ms) > 1 else ms)
     if flop:
@@ -540,7 +559,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,
                     choices=["srsu", "anchor", "xattn", "accumulate", "pcsp", "finalize", "scatter", "cfg",
-                             "mask"],
+                             "stepcache", "mask"],
                     help="run one kernel of the path in isolation (profiling target)")
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--cfg-f", type=int, default=W.F, help="prediction width for --only cfg")

@@ -233,6 +233,23 @@ safedit_status safedit_sw_cfg(const safedit_tensor *eps_c,
                               const safedit_tensor *out, void *stream);
 
 /* ------------------------------------------------------------------------
+ * StepCache with sensitivity-weighted CFG.  [P3 B.3]: full inference runs
+ * only every Delta steps and the noise prediction is reused in between by
+ * linear extrapolation; combined here with the guidance of [P1 방법론 4]:
+ *   c = c_b + w (c_b - c_a),   u = u_b + w (u_b - u_a),
+ *   out = u + gamma_i (c - u),  gamma_i = gamma_ctx + (gamma_sens - gamma_ctx) s_i
+ * where a, b are the last two full steps (b later) and w = (t - t_b)/(t_b - t_a).
+ * All tensors [N, F] f32, inner stride 1 (out may alias an input); d_s [N] f32.
+ */
+safedit_status safedit_stepcache_sw_cfg(const safedit_tensor *eps_c_a,
+                                        const safedit_tensor *eps_c_b,
+                                        const safedit_tensor *eps_u_a,
+                                        const safedit_tensor *eps_u_b,
+                                        const float *d_s, float w,
+                                        float gamma_ctx, float gamma_sens,
+                                        const safedit_tensor *out, void *stream);
+
+/* ------------------------------------------------------------------------
  * Device status word: waits for `stream`, copies the word of the current
  * device into *host_status (a safedit_status value, SAFEDIT_OK if nothing
  * was flagged since the last read) and clears it.

@@ -454,3 +454,30 @@ void oracle_sw_cfg(int64_t N, int64_t F, const double *eps_c,
     }
   }
 }
+
+/* ------------------------------------------------------------------------ */
+/* C10  StepCache: linear extrapolation of the noise prediction between full
+ * steps, combined with the guidance.
+ *
+ * [P3 B.3 StepCache]: full transformer inference runs only every Delta
+ * steps; in between, the noise prediction is reused through linear
+ * extrapolation.  Reading: from the last two full steps a and b (b later),
+ *   eps(t) = eps_b + w (eps_b - eps_a),  w = (t - t_b) / (t_b - t_a),
+ * per branch, then the sensitivity-weighted combine C8 of the extrapolated
+ * branches (CFG is linear, so this equals extrapolating the guided output).
+ * All arrays [N][F]; s [N].
+ */
+void oracle_stepcache_sw_cfg(int64_t N, int64_t F, const double *c_a,
+                             const double *c_b, const double *u_a,
+                             const double *u_b, const double *s, double w,
+                             double gamma_ctx, double gamma_sens, double *out) {
+  for (int64_t i = 0; i < N; ++i) {
+    double g = gamma_ctx + (gamma_sens - gamma_ctx) * s[i];
+    for (int64_t f = 0; f < F; ++f) {
+      int64_t e = i * F + f;
+      double c = c_b[e] + w * (c_b[e] - c_a[e]);
+      double u = u_b[e] + w * (u_b[e] - u_a[e]);
+      out[e] = u + g * (c - u);
+    }
+  }
+}

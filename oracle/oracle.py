@@ -50,6 +50,9 @@ def lib():
         L.oracle_gather_rows.argtypes = [_i64, _i64, _i64, _up, _up, _ip]
         L.oracle_sw_cfg.argtypes = [_i64, _i64, _dp, _dp, _dp, ctypes.c_double, ctypes.c_double, _dp]
         L.oracle_sw_cfg.restype = None
+        L.oracle_stepcache_sw_cfg.argtypes = [_i64, _i64, _dp, _dp, _dp, _dp, _dp, ctypes.c_double,
+                                              ctypes.c_double, ctypes.c_double, _dp]
+        L.oracle_stepcache_sw_cfg.restype = None
         _lib = L
     return _lib
 
@@ -225,6 +228,18 @@ def sw_cfg(eps_c, eps_u, s, gamma_ctx, gamma_sens):
     return out
 
 
+# ---- C10 ------------------------------------------------------------------
+def stepcache_sw_cfg(c_a, c_b, u_a, u_b, s, w, gamma_ctx, gamma_sens):
+    """Extrapolated branches eps_b + w (eps_b - eps_a), then the weighted combine."""
+    arrs = [_f64(x) for x in (c_a, c_b, u_a, u_b)]
+    sv = _f64(s)
+    N, F = arrs[0].shape
+    out = np.empty((N, F), dtype=np.float64)
+    lib().oracle_stepcache_sw_cfg(N, F, *[_p(a, _dp) for a in arrs], _p(sv, _dp), float(w),
+                                  float(gamma_ctx), float(gamma_sens), _p(out, _dp))
+    return out
+
+
 # ---- C9 -------------------------------------------------------------------
 def is_anchor_step(t: int, warmup: int, period: int) -> bool:
     """Schedule reading: warm-up steps are dense; afterwards step t is a dense
@@ -281,4 +296,4 @@ def trajectory(steps, warmup, period, k, gamma_ctx, gamma_sens):
 
 __all__ = ["OracleError", "lib", "num_threads", "default_scale", "cross_attn_probs",
            "partition_accumulate", "partition_select", "mask_row_constant", "attn_subset",
-           "attn_dense", "scatter_rows", "gather_rows", "sw_cfg", "is_anchor_step", "trajectory"]
+           "attn_dense", "scatter_rows", "gather_rows", "sw_cfg", "is_anchor_step", "trajectory", "stepcache_sw_cfg"]

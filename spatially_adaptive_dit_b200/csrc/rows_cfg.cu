@@ -188,6 +188,62 @@ __global__ void __launch_bounds__(256) sw_cfg_scalar_kernel(CfgParams p) {
   }
 }
 
+// ------------------------------------------------------------ StepCache ---
+// AccelAes summary B.3: between full steps the noise prediction is reused by
+// linear extrapolation; fused with the guidance combine:
+//   c = c_b + w (c_b - c_a),  u = u_b + w (u_b - u_a),  out = u + gamma_i (c - u).
+struct StepCacheParams {
+  const float* ca;
+  const float* cb;
+  const float* ua;
+  const float* ub;
+  const float* s;
+  float* out;
+  int64_t N, F;
+  int64_t sca, scb, sua, sub, so;  // row strides (elements)
+  float w, g_ctx, g_diff;
+};
+
+__device__ __forceinline__ float stepcache_one(float ca, float cb, float ua, float ub, float w,
+                                               float g) {
+  const float c = fmaf(w, cb - ca, cb);
+  const float u = fmaf(w, ub - ua, ub);
+  return fmaf(g, c - u, u);
+}
+
+__global__ void __launch_bounds__(256) stepcache_vec4_kernel(StepCacheParams p) {
+  const int64_t F4 = p.F >> 2;
+  const int64_t total = p.N * F4;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t i = e / F4;
+    const int64_t f = (e - i * F4) << 2;
+    const float g = fmaf(p.g_diff, __ldg(p.s + i), p.g_ctx);
+    const float4 ca = __ldcs(reinterpret_cast<const float4*>(p.ca + i * p.sca + f));
+    const float4 cb = __ldcs(reinterpret_cast<const float4*>(p.cb + i * p.scb + f));
+    const float4 ua = __ldcs(reinterpret_cast<const float4*>(p.ua + i * p.sua + f));
+    const float4 ub = __ldcs(reinterpret_cast<const float4*>(p.ub + i * p.sub + f));
+    float4 o;
+    o.x = stepcache_one(ca.x, cb.x, ua.x, ub.x, p.w, g);
+    o.y = stepcache_one(ca.y, cb.y, ua.y, ub.y, p.w, g);
+    o.z = stepcache_one(ca.z, cb.z, ua.z, ub.z, p.w, g);
+    o.w = stepcache_one(ca.w, cb.w, ua.w, ub.w, p.w, g);
+    __stcs(reinterpret_cast<float4*>(p.out + i * p.so + f), o);
+  }
+}
+
+__global__ void __launch_bounds__(256) stepcache_scalar_kernel(StepCacheParams p) {
+  const int64_t total = p.N * p.F;
+  for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t i = e / p.F;
+    const int64_t f = e - i * p.F;
+    const float g = fmaf(p.g_diff, p.s[i], p.g_ctx);
+    p.out[i * p.so + f] = stepcache_one(p.ca[i * p.sca + f], p.cb[i * p.scb + f],
+                                        p.ua[i * p.sua + f], p.ub[i * p.sub + f], p.w, g);
+  }
+}
+
 }  // namespace sd
 
 using namespace sd;
@@ -248,6 +304,59 @@ safedit_status safedit_sw_cfg(const safedit_tensor* eps_c, const safedit_tensor*
     sw_cfg_vec4_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
   else
     sw_cfg_scalar_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+  return after_launch(1);
+}
+
+safedit_status safedit_stepcache_sw_cfg(const safedit_tensor* eps_c_a, const safedit_tensor* eps_c_b,
+                                        const safedit_tensor* eps_u_a, const safedit_tensor* eps_u_b,
+                                        const float* d_s, float w, float gamma_ctx, float gamma_sens,
+                                        const safedit_tensor* out, void* stream) {
+  safedit_status st;
+  const safedit_tensor* ins[4] = {eps_c_a, eps_c_b, eps_u_a, eps_u_b};
+  for (const safedit_tensor* t : ins)
+    if ((st = check_tensor(t, 2)) != SAFEDIT_OK) return st;
+  if ((st = check_tensor(out, 2)) != SAFEDIT_OK) return st;
+  if (!d_s) return SAFEDIT_ERR_INVALID_ARG;
+  const int64_t N = out->dims[0], F = out->dims[1];
+  for (const safedit_tensor* t : ins) {
+    if (t->dtype != SAFEDIT_F32) return SAFEDIT_ERR_DTYPE;
+    if (t->dims[0] != N || t->dims[1] != F) return SAFEDIT_ERR_SHAPE;
+    if (t->strides[1] != 1) return SAFEDIT_ERR_ALIGNMENT;
+  }
+  if (out->dtype != SAFEDIT_F32) return SAFEDIT_ERR_DTYPE;
+  if (out->strides[1] != 1) return SAFEDIT_ERR_ALIGNMENT;
+  if (N == 0 || F == 0) return SAFEDIT_OK;
+  StepCacheParams p;
+  p.ca = static_cast<const float*>(eps_c_a->data);
+  p.cb = static_cast<const float*>(eps_c_b->data);
+  p.ua = static_cast<const float*>(eps_u_a->data);
+  p.ub = static_cast<const float*>(eps_u_b->data);
+  p.s = d_s;
+  p.out = static_cast<float*>(out->data);
+  p.N = N;
+  p.F = F;
+  p.sca = eps_c_a->strides[0];
+  p.scb = eps_c_b->strides[0];
+  p.sua = eps_u_a->strides[0];
+  p.sub = eps_u_b->strides[0];
+  p.so = out->strides[0];
+  p.w = w;
+  p.g_ctx = gamma_ctx;
+  p.g_diff = gamma_sens - gamma_ctx;
+  bool vec = (F % 4 == 0) && aligned16(p.out) && (p.so % 4 == 0);
+  for (const safedit_tensor* t : ins) vec = vec && aligned16(t->data) && (t->strides[0] % 4 == 0);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t work = vec ? N * (F / 4) : N * F;
+  int64_t blocks = (work + 255) / 256;
+  const int64_t cap = int64_t(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (vec)
+    stepcache_vec4_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+  else
+    stepcache_scalar_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
   return after_launch(1);
 }
 

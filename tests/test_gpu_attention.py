@@ -217,3 +217,16 @@ def test_3072_sweep_sampled():
         ref = oracle_rows(q, k, v, idx.cpu().numpy(), 1, 5, rows=rows)
         check_attn(f64(out[1, 5, torch.as_tensor(rows, device=DEV)]), ref, f"rho={rho}")
         del out
+
+
+def test_compact_query_rows_over_all_keys():
+    """Fresh S-row queries given compact ([B,H,k,d], idx = NULL) attend over
+    the N-row state: the form an SRSU step takes when only the S rows were
+    projected."""
+    B, H, N, D, kr = 2, 3, 900, 96, 271
+    q, k, v = _qkv(B, H, kr, N, D, seed=91)
+    out = run(q.to(DEV), k.to(DEV), v.to(DEV))
+    for b in range(B):
+        for h in range(H):
+            ref = oracle.attn_subset(f64(q[b, h]), f64(k[b, h]), f64(v[b, h]))
+            check_attn(f64(out[b, h]), ref, f"b{b}h{h}")

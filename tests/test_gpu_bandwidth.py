@@ -240,3 +240,19 @@ def test_mask_stress_config_full_size():
         assert np.array_equal(fl.cpu().numpy()[rows], rf)
         assert int(v.item()) == (1 if kind in ("zero", "rowconst") else 0)
         del m
+
+
+# ----------------------------------------------------------------- StepCache
+@pytest.mark.parametrize("N,F,w", [(4096, 16, 0.5), (25600, 16, 1.0), (1000, 13, -0.25), (257, 4096, 2.0)])
+def test_stepcache_sw_cfg(N, F, w):
+    g = _gen(N * 3 + F)
+    ca, cb, ua, ub = (torch.randn(N, F, generator=g) for _ in range(4))
+    s = torch.rand(N, generator=g)
+    out = torch.empty(N, F, device=DEV)
+    sd().safedit_stepcache_sw_cfg(ca.to(DEV), cb.to(DEV), ua.to(DEV), ub.to(DEV), s.to(DEV), w, 3.0, 5.0, out)
+    expect_status(0)
+    ref = oracle.stepcache_sw_cfg(ca, cb, ua, ub, s, w, 3.0, 5.0)
+    gam = (3.0 + 2.0 * s.double().numpy())[:, None]
+    mag = (1 + abs(w)) * (ca.abs() + cb.abs() + ua.abs() + ub.abs()).double().numpy()
+    err = np.abs(out.cpu().double().numpy() - ref)
+    assert np.all(err <= CFG_REL * (1 + gam) * mag + 1e-30)

@@ -362,3 +362,25 @@ def test_trajectory_anchor_refreshes_everything():
     assert np.array_equal(res["k_state"], steps[2]["k_full"])
     dense = oracle.attn_dense(steps[2]["q"][0, 0], steps[2]["k_full"][0, 0], steps[2]["v_full"][0, 0])
     assert np.array_equal(res["o_state"][0, 0], dense)
+
+
+# ---------------------------------------------------------------------------
+# StepCache (C10): AccelAes summary B.3 (linear extrapolation between full steps).
+# ---------------------------------------------------------------------------
+def test_stepcache_extrapolation_closed_forms():
+    N, F = 23, 8
+    c_a, c_b, u_a, u_b = (rng.standard_normal((N, F)) for _ in range(4))
+    s = rng.random(N)
+    # w = 0 reuses the last full step, w = -1 the one before: the plain combine of that step
+    assert np.abs(oracle.stepcache_sw_cfg(c_a, c_b, u_a, u_b, s, 0.0, 3.0, 5.0)
+                  - oracle.sw_cfg(c_b, u_b, s, 3.0, 5.0)).max() <= 1e-14
+    assert np.abs(oracle.stepcache_sw_cfg(c_a, c_b, u_a, u_b, s, -1.0, 3.0, 5.0)
+                  - oracle.sw_cfg(c_a, u_a, s, 3.0, 5.0)).max() <= 1e-14
+    # predictions linear in t are reproduced exactly at any later t
+    slope_c, slope_u = rng.standard_normal((N, F)), rng.standard_normal((N, F))
+    t_a, t_b, t = 10.0, 12.0, 15.0
+    ca, cb, ct = c_b + slope_c * t_a, c_b + slope_c * t_b, c_b + slope_c * t
+    ua, ub, ut = u_b + slope_u * t_a, u_b + slope_u * t_b, u_b + slope_u * t
+    w = (t - t_b) / (t_b - t_a)
+    assert np.abs(oracle.stepcache_sw_cfg(ca, cb, ua, ub, s, w, 3.0, 5.0)
+                  - oracle.sw_cfg(ct, ut, s, 3.0, 5.0)).max() <= 1e-12
