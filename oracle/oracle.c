@@ -481,3 +481,54 @@ void oracle_stepcache_sw_cfg(int64_t N, int64_t F, const double *c_a,
     }
   }
 }
+
+/* ------------------------------------------------------------------------ */
+/* C11  SkipSparse FFN caching.
+ *
+ * [P3 B.2 SkipSparse]: the FFN is skipped for background tokens, whose most
+ * recent cached output is reused; focus tokens are recomputed.  Reading: the
+ * DiT feed-forward block y = W2 gelu(W1 x + b1) + b2 with the tanh form of
+ * GELU (the DiT convention; Hendrycks & Gimpel's approximation
+ * 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))), weights in the
+ * nn.Linear layout [out][in].
+ *   y_cache[idx[r]] = ffn(x[idx[r]]) for r < n_idx; every other row keeps its
+ *   cached value.
+ * x, y_cache: [N][D]; w1: [F][D], b1: [F] (nullable); w2: [D][F], b2: [D]
+ * (nullable); act = 0 (identity) or 1 (gelu-tanh).
+ */
+static double gelu_tanh(double v) {
+  const double c = 0.7978845608028654; /* sqrt(2/pi) */
+  return 0.5 * v * (1.0 + tanh(c * (v + 0.044715 * v * v * v)));
+}
+
+int oracle_ffn_cached(int64_t N, int64_t D, int64_t F, const double *x,
+                      const int32_t *idx, int64_t n_idx, const double *w1,
+                      const double *b1, const double *w2, const double *b2,
+                      int act, double *y_cache) {
+  if (N < 0 || D <= 0 || F <= 0 || n_idx < 0 || !x || !w1 || !w2 || !y_cache)
+    return OR_EINVAL;
+  int rc = idx ? check_index(idx, n_idx, N, 1) : OR_OK;
+  if (rc) return rc;
+  int64_t n = idx ? n_idx : N;
+#pragma omp parallel
+  {
+    double *hid = (double *)malloc(sizeof(double) * (size_t)F);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; ++r) {
+      int64_t i = idx ? idx[r] : r;
+      const double *xi = x + i * D;
+      for (int64_t f = 0; f < F; ++f) {
+        double a = b1 ? b1[f] : 0.0;
+        for (int64_t c = 0; c < D; ++c) a += w1[f * D + c] * xi[c];
+        hid[f] = act ? gelu_tanh(a) : a;
+      }
+      for (int64_t c = 0; c < D; ++c) {
+        double a = b2 ? b2[c] : 0.0;
+        for (int64_t f = 0; f < F; ++f) a += w2[c * F + f] * hid[f];
+        y_cache[i * D + c] = a;
+      }
+    }
+    free(hid);
+  }
+  return OR_OK;
+}

@@ -53,6 +53,7 @@ def lib():
         L.oracle_stepcache_sw_cfg.argtypes = [_i64, _i64, _dp, _dp, _dp, _dp, _dp, ctypes.c_double,
                                               ctypes.c_double, ctypes.c_double, _dp]
         L.oracle_stepcache_sw_cfg.restype = None
+        L.oracle_ffn_cached.argtypes = [_i64, _i64, _i64, _dp, _ip, _i64, _dp, _dp, _dp, _dp, ctypes.c_int, _dp]
         _lib = L
     return _lib
 
@@ -240,6 +241,22 @@ def stepcache_sw_cfg(c_a, c_b, u_a, u_b, s, w, gamma_ctx, gamma_sens):
     return out
 
 
+# ---- C11 ------------------------------------------------------------------
+def ffn_cached(x, idx, w1, b1, w2, b2, y_cache, act=1):
+    """Returns a copy of y_cache [N,D] with rows idx recomputed as
+    W2 gelu(W1 x + b1) + b2 (act=0: no activation).  Weights [out, in]."""
+    x, w1, w2 = _f64(x), _f64(w1), _f64(w2)
+    b1a, b2a = _f64(b1), _f64(b2)
+    y = np.array(_f64(y_cache), copy=True)
+    N, D = x.shape
+    F = w1.shape[0]
+    idx_a = _i32(idx)
+    n = N if idx_a is None else idx_a.shape[0]
+    _check(lib().oracle_ffn_cached(N, D, F, _p(x, _dp), _p(idx_a, _ip), n, _p(w1, _dp), _p(b1a, _dp),
+                                   _p(w2, _dp), _p(b2a, _dp), int(act), _p(y, _dp)))
+    return y
+
+
 # ---- C9 -------------------------------------------------------------------
 def is_anchor_step(t: int, warmup: int, period: int) -> bool:
     """Schedule reading: warm-up steps are dense; afterwards step t is a dense
@@ -296,4 +313,4 @@ def trajectory(steps, warmup, period, k, gamma_ctx, gamma_sens):
 
 __all__ = ["OracleError", "lib", "num_threads", "default_scale", "cross_attn_probs",
            "partition_accumulate", "partition_select", "mask_row_constant", "attn_subset",
-           "attn_dense", "scatter_rows", "gather_rows", "sw_cfg", "is_anchor_step", "trajectory", "stepcache_sw_cfg"]
+           "attn_dense", "scatter_rows", "gather_rows", "sw_cfg", "is_anchor_step", "trajectory", "stepcache_sw_cfg", "ffn_cached"]

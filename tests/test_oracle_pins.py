@@ -384,3 +384,28 @@ def test_stepcache_extrapolation_closed_forms():
     w = (t - t_b) / (t_b - t_a)
     assert np.abs(oracle.stepcache_sw_cfg(ca, cb, ua, ub, s, w, 3.0, 5.0)
                   - oracle.sw_cfg(ct, ut, s, 3.0, 5.0)).max() <= 1e-12
+
+
+# ---------------------------------------------------------------------------
+# SkipSparse FFN caching (C11): AccelAes summary B.2.
+# ---------------------------------------------------------------------------
+def test_ffn_cached_against_library_and_cache_rule():
+    N, D, F = 37, 16, 40
+    x = rng.standard_normal((N, D))
+    w1, b1 = rng.standard_normal((F, D)) / 4, rng.standard_normal(F)
+    w2, b2 = rng.standard_normal((D, F)) / 6, rng.standard_normal(D)
+    cache = rng.standard_normal((N, D))
+    idx = np.sort(rng.choice(N, size=11, replace=False)).astype(np.int32)
+    y = oracle.ffn_cached(x, idx, w1, b1, w2, b2, cache, act=1)
+    # library routine: torch's tanh-approximate GELU and float64 matmuls
+    xt = torch.tensor(x[idx])
+    h = torch.nn.functional.gelu(xt @ torch.tensor(w1).T + torch.tensor(b1), approximate="tanh")
+    ref = (h @ torch.tensor(w2).T + torch.tensor(b2)).numpy()
+    assert np.abs(y[idx] - ref).max() <= 1e-12
+    keep = np.setdiff1d(np.arange(N), idx)
+    assert np.array_equal(y[keep], cache[keep])  # background rows reuse the cache
+    # no activation: the block is affine, so it is a single matrix
+    y0 = oracle.ffn_cached(x, None, w1, None, w2, None, cache, act=0)
+    assert np.abs(y0 - x @ (w2 @ w1).T).max() <= 1e-12
+    with pytest.raises(oracle.OracleError):
+        oracle.ffn_cached(x, np.array([1, 1], dtype=np.int32), w1, b1, w2, b2, cache)
