@@ -532,3 +532,24 @@ int oracle_ffn_cached(int64_t N, int64_t D, int64_t F, const double *x,
   }
   return OR_OK;
 }
+
+/* C12  One projection of that block, on its own: out = act(a w^T + b).
+ *
+ * [P3 B.2 SkipSparse] runs the FFN's projections (and the Q/K/V projections of
+ * an SRSU step) on the gathered focus rows only; this is one such projection.
+ *   out[r][n] = act(b[n] + sum_k w[n][k] a[r][k]),  a: [M][K], w: [N][K]
+ * (nn.Linear layout), b: [N] (nullable), act as in C11.
+ */
+int oracle_linear_act(int64_t M, int64_t K, int64_t N, const double *a,
+                      const double *w, const double *b, int act, double *out) {
+  if (M < 0 || K <= 0 || N < 0 || !a || !w || !out) return OR_EINVAL;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < M; ++r) {
+    for (int64_t n = 0; n < N; ++n) {
+      double acc = b ? b[n] : 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += w[n * K + k] * a[r * K + k];
+      out[r * N + n] = act ? gelu_tanh(acc) : acc;
+    }
+  }
+  return OR_OK;
+}

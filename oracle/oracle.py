@@ -54,6 +54,7 @@ def lib():
                                               ctypes.c_double, ctypes.c_double, _dp]
         L.oracle_stepcache_sw_cfg.restype = None
         L.oracle_ffn_cached.argtypes = [_i64, _i64, _i64, _dp, _ip, _i64, _dp, _dp, _dp, _dp, ctypes.c_int, _dp]
+        L.oracle_linear_act.argtypes = [_i64, _i64, _i64, _dp, _dp, _dp, ctypes.c_int, _dp]
         _lib = L
     return _lib
 
@@ -257,6 +258,20 @@ def ffn_cached(x, idx, w1, b1, w2, b2, y_cache, act=1):
     return y
 
 
+# ---- C12 ------------------------------------------------------------------
+def linear_act(a, w, b=None, act=0):
+    """out [M,N] = act(a [M,K] w[N,K]^T + b[N]) in fp64 (act 1 = gelu-tanh)."""
+    a, w = _f64(a), _f64(w)
+    ba = None if b is None else _f64(b)
+    M, K = a.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise OracleError("shape mismatch")
+    out = np.empty((M, N), dtype=np.float64)
+    _check(lib().oracle_linear_act(M, K, N, _p(a, _dp), _p(w, _dp), _p(ba, _dp), int(act), _p(out, _dp)))
+    return out
+
+
 # ---- C9 -------------------------------------------------------------------
 def is_anchor_step(t: int, warmup: int, period: int) -> bool:
     """Schedule reading: warm-up steps are dense; afterwards step t is a dense
@@ -313,4 +328,5 @@ def trajectory(steps, warmup, period, k, gamma_ctx, gamma_sens):
 
 __all__ = ["OracleError", "lib", "num_threads", "default_scale", "cross_attn_probs",
            "partition_accumulate", "partition_select", "mask_row_constant", "attn_subset",
-           "attn_dense", "scatter_rows", "gather_rows", "sw_cfg", "is_anchor_step", "trajectory", "stepcache_sw_cfg", "ffn_cached"]
+           "attn_dense", "scatter_rows", "gather_rows", "sw_cfg", "is_anchor_step", "trajectory", "stepcache_sw_cfg", "ffn_cached",
+           "linear_act"]

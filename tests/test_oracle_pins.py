@@ -409,3 +409,27 @@ def test_ffn_cached_against_library_and_cache_rule():
     assert np.abs(y0 - x @ (w2 @ w1).T).max() <= 1e-12
     with pytest.raises(oracle.OracleError):
         oracle.ffn_cached(x, np.array([1, 1], dtype=np.int32), w1, b1, w2, b2, cache)
+
+
+def test_linear_act_against_library_and_closed_forms():
+    M, K, N = 23, 19, 31
+    a = rng.standard_normal((M, K))
+    w, b = rng.standard_normal((N, K)) / 3, rng.standard_normal(N)
+    out = oracle.linear_act(a, w, b, act=1)
+    ref = torch.nn.functional.gelu(torch.nn.functional.linear(torch.tensor(a), torch.tensor(w), torch.tensor(b)),
+                                   approximate="tanh").numpy()
+    assert np.abs(out - ref).max() <= 1e-12
+    # identity weights, no bias, no activation: the input itself
+    assert np.array_equal(oracle.linear_act(a, np.eye(K), None, act=0), a)
+    # GELU closed forms: gelu(0) = 0, odd part x/2, gelu(x) -> x for large x, -> 0 for very negative x
+    z = oracle.linear_act(np.array([[0.0], [1.0], [-1.0], [12.0], [-12.0]]), np.ones((1, 1)), None, act=1)[:, 0]
+    assert z[0] == 0.0
+    assert abs((z[1] - z[2]) - 1.0) <= 1e-15  # gelu(x) - gelu(-x) = x
+    assert abs(z[3] - 12.0) <= 1e-12 and abs(z[4]) <= 1e-12
+    # 0.5 (1 + tanh(sqrt(2/pi) (1 + 0.044715))) at x = 1, from math.tanh directly
+    assert abs(z[1] - 0.5 * (1 + math.tanh(math.sqrt(2 / math.pi) * 1.044715))) <= 1e-15
+    # the block of C11 is two such projections
+    x = rng.standard_normal((7, K))
+    w2, b2 = rng.standard_normal((K, N)) / 5, rng.standard_normal(K)
+    y = oracle.ffn_cached(x, None, w, b, w2, b2, np.zeros((7, K)), act=1)
+    assert np.abs(y - oracle.linear_act(oracle.linear_act(x, w, b, 1), w2, b2, 0)).max() <= 1e-12
