@@ -499,6 +499,23 @@ def run_only(args):
         extra["prev_c"], extra["prev_u"] = wl.cfg_preds(w, step=1, device=dev, F=tr.eps_c.shape[1])
     if args.only == "mask":
         extra["mask"] = torch.zeros(1, 1, wl.STRESS.N, wl.STRESS.N, dtype=torch.bfloat16, device=dev)
+    ffn_flop = 2 * w.B * tr.k * w.D_model * w.D_ff  # one projection of the cached FFN
+    if args.only in ("ffn1", "ffn2", "ffn"):
+        # SkipSparse FFN caching on the focus rows: gather, W1 (+b1, GELU), W2 (+b2) scattered
+        w1, b1, w2, b2 = (t.to(dev) for t in wl.ffn_weights(w))
+        x, y = (t.to(dev) for t in wl.ffn_states(w))
+        xs = torch.empty(w.B, 1, tr.k, w.D_model, dtype=torch.bfloat16, device=dev)
+        h = torch.empty(w.B, tr.k, w.D_ff, dtype=torch.bfloat16, device=dev)
+        sd.safedit_gather_rows([x.view(w.B, 1, w.N, w.D_model)], [xs], tr.idx_s, tr.k, stream)
+        xs3 = xs.view(w.B, tr.k, w.D_model)
+        extra["ffn1"] = lambda: sd.safedit_gemm_bias_act(xs3, w1, b1, 1, None, h, stream)
+        extra["ffn2"] = lambda: sd.safedit_gemm_bias_act(h, w2, b2, 0, tr.idx_s, y, stream)
+
+        def ffn_block():
+            sd.safedit_gather_rows([x.view(w.B, 1, w.N, w.D_model)], [xs], tr.idx_s, tr.k, stream)
+            extra["ffn1"]()
+            extra["ffn2"]()
+        extra["ffn"] = ffn_block
     fns = {
         "srsu": (lambda: sd.safedit_attn_subset(tr.q, tr.k_state, tr.v_state, tr.idx_s, tr.k, None, None,
                                                 0.0, tr.o_state, 1, stream), tr.flop_srsu, None),
@@ -522,6 +539,9 @@ def run_only(args):
                                                           tr.s, 0.5, w.gamma_ctx, w.gamma_sens, tr.cfg_out,
                                                           stream),
                       None, 5 * tr.eps_c.numel() * 4 + 4 * w.N),
+        "ffn1": (lambda: extra["ffn1"](), ffn_flop, None),
+        "ffn2": (lambda: extra["ffn2"](), ffn_flop, None),
+        "ffn": (lambda: extra["ffn"](), 2 * ffn_flop, None),
     }
     fn, flop, nbytes = fns[args.only]
     times = []
@@ -559,7 +579,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,
                     choices=["srsu", "anchor", "xattn", "accumulate", "pcsp", "finalize", "scatter", "cfg",
-                             "stepcache", "mask"],
+                             "stepcache", "mask", "ffn1", "ffn2", "ffn"],
                     help="run one kernel of the path in isolation (profiling target)")
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--cfg-f", type=int, default=W.F, help="prediction width for --only cfg")

@@ -250,6 +250,36 @@ safedit_status safedit_stepcache_sw_cfg(const safedit_tensor *eps_c_a,
                                         const safedit_tensor *out, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Dense projection with fused bias and activation, and optional row scatter:
+ * the GEMM of SkipSparse FFN caching [P3 B.2], where the FFN runs on the
+ * sensitive (focus) tokens only and every other token keeps its cached FFN
+ * output.  With X_S the gathered sensitive rows:
+ *   H   = GELU(X_S W1^T + b1)                       (act = 1, d_idx_out NULL)
+ *   Y[idx[r], :] = (H W2^T + b2)[r, :]             (act = 0, d_idx_out = idx)
+ * and the same call with act = 0 serves the gathered Q/K/V projections.
+ *
+ *   out[row(r), n] = act( sum_k a[r,k] * w[n,k] + bias[n] ),  r < M, n < N
+ *   row(r) = d_idx_out ? d_idx_out[r] : r
+ *
+ * a [M, K] or batched [B, M, K], w [N, K] (nn.Linear layout: out_features x
+ * in_features), bf16, inner stride 1, row and batch strides multiples of 8
+ * elements, 16-byte aligned bases.  out [M_out, N] or [B, M_out, N] (same
+ * rank as a, same rules); w and d_idx_out are shared by every batch; without
+ * d_idx_out M_out must equal M.  N must be a multiple of 8.  d_bias: NULL or
+ * N f32 on the device.  act: 0 identity, 1 GELU (tanh form, fp32).
+ * Accumulation is fp32 over all of K (tensor cores), rounded to bf16 once.
+ * d_idx_out: NULL or M int32 on the device, unique (not checked); an entry
+ * outside [0, M_out) sets SAFEDIT_ERR_INDEX on the device status word and
+ * that row is skipped.  Rows of out that no r maps to are untouched.
+ * M == 0 or N == 0 is a no-op; K == 0 is SAFEDIT_ERR_SHAPE.
+ */
+safedit_status safedit_gemm_bias_act(const safedit_tensor *a,
+                                     const safedit_tensor *w,
+                                     const float *d_bias, int32_t act,
+                                     const int32_t *d_idx_out,
+                                     const safedit_tensor *out, void *stream);
+
+/* ------------------------------------------------------------------------
  * Device status word: waits for `stream`, copies the word of the current
  * device into *host_status (a safedit_status value, SAFEDIT_OK if nothing
  * was flagged since the last read) and clears it.

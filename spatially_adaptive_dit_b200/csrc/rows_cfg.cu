@@ -22,6 +22,7 @@ struct RowCopyParams {
   int64_t x_sb[kMaxRowTensors], x_sh[kMaxRowTensors], x_sr[kMaxRowTensors];
   int H[kMaxRowTensors], BH[kMaxRowTensors], units[kMaxRowTensors];
   int rows_per_pass[kMaxRowTensors];
+  int slices[kMaxRowTensors];  // column slices of kRowThreads units (rows wider than a block)
   int n_idx;       // compact rows
   int n_rows_x;    // rows of the indexed side
   const int* idx;
@@ -32,22 +33,26 @@ struct RowCopyParams {
 constexpr int kRowThreads = 256;
 constexpr int kRowIters = 4;  // independent 16-byte copies in flight per thread
 
-// grid: x = row blocks, y = b*H + h, z = tensor.
+// grid: x = row blocks x column slices, y = b*H + h, z = tensor.  A row of
+// at most kRowThreads 16-byte units is one slice, and a block copies several
+// such rows per pass; a wider row is cut into slices of kRowThreads units.
 __global__ void __launch_bounds__(kRowThreads) row_copy_kernel(RowCopyParams p) {
   const int t = blockIdx.z;
   const int bh = blockIdx.y;
   if (bh >= p.BH[t]) return;
-  const int U = p.units[t];
+  const int S = p.slices[t];
+  const int xb = blockIdx.x / S, sl = blockIdx.x - xb * S;
+  const int Uw = min(p.units[t] - sl * kRowThreads, kRowThreads);
   const int rpp = p.rows_per_pass[t];
-  const int sub = threadIdx.x / U;
-  const int unit = threadIdx.x - sub * U;
+  const int sub = threadIdx.x / Uw;
+  const int unit = sl * kRowThreads + (threadIdx.x - sub * Uw);
   if (sub >= rpp) return;
   const int b = bh / p.H[t], h = bh - b * p.H[t];
   const char* cb_src;
   char* cb_dst;
   const int64_t c_off = b * p.c_sb[t] + h * p.c_sh[t] + int64_t(unit) * 16;
   const int64_t x_off = b * p.x_sb[t] + h * p.x_sh[t] + int64_t(unit) * 16;
-  const int r_base = blockIdx.x * (rpp * kRowIters) + sub;
+  const int r_base = xb * (rpp * kRowIters) + sub;
 
   uint4 v[kRowIters];
   int64_t dst_off[kRowIters];
@@ -115,7 +120,6 @@ static safedit_status row_copy(const safedit_tensor* src, const safedit_tensor* 
       if ((s.strides[k] * es) % 16 != 0 || (d.strides[k] * es) % 16 != 0)
         return SAFEDIT_ERR_ALIGNMENT;
     if (!aligned16(s.data) || !aligned16(d.data)) return SAFEDIT_ERR_ALIGNMENT;
-    if (row_bytes / 16 > kRowThreads) return SAFEDIT_ERR_UNSUPPORTED;
     if (s.dims[0] * s.dims[1] > 65535) return SAFEDIT_ERR_UNSUPPORTED;
     p.src[t] = static_cast<const char*>(s.data);
     p.dst[t] = static_cast<char*>(d.data);
@@ -128,9 +132,13 @@ static safedit_status row_copy(const safedit_tensor* src, const safedit_tensor* 
     p.H[t] = static_cast<int>(s.dims[1]);
     p.BH[t] = static_cast<int>(s.dims[0] * s.dims[1]);
     p.units[t] = static_cast<int>(row_bytes / 16);
-    p.rows_per_pass[t] = kRowThreads / p.units[t];
+    if (row_bytes / 16 > INT32_MAX / 2) return SAFEDIT_ERR_UNSUPPORTED;
+    p.slices[t] = (p.units[t] + kRowThreads - 1) / kRowThreads;
+    p.rows_per_pass[t] = p.slices[t] > 1 ? 1 : kRowThreads / p.units[t];
     const int rows_per_block = p.rows_per_pass[t] * kRowIters;
-    const int blocks = (n_idx + rows_per_block - 1) / rows_per_block;
+    const int64_t blocks64 = int64_t((n_idx + rows_per_block - 1) / rows_per_block) * p.slices[t];
+    if (blocks64 > INT32_MAX) return SAFEDIT_ERR_UNSUPPORTED;
+    const int blocks = static_cast<int>(blocks64);
     if (p.BH[t] > max_bh) max_bh = p.BH[t];
     if (blocks > max_blocks) max_blocks = blocks;
   }

@@ -32,7 +32,7 @@ _DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16, torch.bo
 EXPORTED = ("safedit_cross_attn_probs", "safedit_partition_accumulate", "safedit_pcsp_score",
             "safedit_partition_finalize", "safedit_mask_is_row_constant", "safedit_attn_subset",
             "safedit_scatter_state", "safedit_gather_rows", "safedit_sw_cfg", "safedit_stepcache_sw_cfg",
-            "safedit_get_device_status", "safedit_status_string", "safedit_kernel_launch_count",
+            "safedit_gemm_bias_act", "safedit_get_device_status", "safedit_status_string", "safedit_kernel_launch_count",
             "safedit_debug_set_wait_limit_ns")
 
 
@@ -62,6 +62,7 @@ _lib.safedit_scatter_state.argtypes = [_T, _T, _i32, _vp, _i32, _vp]
 _lib.safedit_gather_rows.argtypes = [_T, _T, _i32, _vp, _i32, _vp]
 _lib.safedit_sw_cfg.argtypes = [_T, _T, _vp, _f32, _f32, _T, _vp]
 _lib.safedit_stepcache_sw_cfg.argtypes = [_T, _T, _T, _T, _vp, _f32, _f32, _f32, _T, _vp]
+_lib.safedit_gemm_bias_act.argtypes = [_T, _T, _vp, _i32, _vp, _T, _vp]
 _lib.safedit_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32), _vp]
 _lib.safedit_status_string.argtypes = [ctypes.c_int]
 _lib.safedit_status_string.restype = ctypes.c_char_p
@@ -177,6 +178,12 @@ def safedit_stepcache_sw_cfg(c_a, c_b, u_a, u_b, s, w, gamma_ctx, gamma_sens, ou
     _check(_lib.safedit_stepcache_sw_cfg(_ref(c_a), _ref(c_b), _ref(u_a), _ref(u_b), _ptr(s), float(w),
                                          float(gamma_ctx), float(gamma_sens), _ref(out), _stream(stream)),
            "safedit_stepcache_sw_cfg")
+
+
+def safedit_gemm_bias_act(a, w, bias, act, idx_out, out, stream=None):
+    _check(_lib.safedit_gemm_bias_act(_ref(a), _ref(w), _ptr(bias), int(act), _ptr(idx_out), _ref(out),
+                                      _stream(stream)),
+           "safedit_gemm_bias_act")
 
 
 def safedit_get_device_status(stream=None) -> int:

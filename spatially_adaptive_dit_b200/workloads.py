@@ -18,7 +18,11 @@ per-tensor offset so that tensors are independent):
     (trailing 1/8 of the keys -inf, else 0); non-uniform bias N(0, 1);
   * clustered scores: 8 Gaussian blobs on the sqrt(N) x sqrt(N) grid, centres
     U over the grid, sigma ~ U(4, 16) patches, amplitude U(0.5, 1), plus
-    1e-3 * U(0, 1) noise.
+    1e-3 * U(0, 1) noise;
+  * FFN block (model width D = H d, hidden width F = ffn_mult D): token
+    states N(0,1) [B, N, D] bf16; W1 [F, D] and W2 [D, F] N(0,1) / sqrt(fan_in)
+    (random init, nn.Linear layout), biases N(0, 0.02^2) fp32; the cached FFN
+    output of the previous step N(0,1) [B, N, D] bf16.
 """
 from dataclasses import dataclass, field
 from fractions import Fraction
@@ -49,6 +53,15 @@ class Workload:
     steps: int = 10     # denoising steps in one trajectory
     fp32_inputs: bool = False
     rho_sweep: tuple = field(default_factory=tuple)
+    ffn_mult: int = 4   # FFN hidden width / model width
+
+    @property
+    def D_model(self) -> int:
+        return self.H * self.d
+
+    @property
+    def D_ff(self) -> int:
+        return self.ffn_mult * self.H * self.d
 
     @property
     def k(self) -> int:
@@ -95,6 +108,7 @@ def uniform(shape, lo, hi, w: Workload, offset: int, device="cpu", dtype=torch.f
 # Tensor offsets (kept distinct so every tensor is an independent draw).
 OFF_Q, OFF_K, OFF_V, OFF_QX, OFF_KTXT, OFF_KS, OFF_VS, OFF_EPSC, OFF_EPSU = range(1, 10)
 OFF_MASK_ROW, OFF_MASK_BIAS, OFF_BLOB = 20, 21, 22
+OFF_X, OFF_W1, OFF_B1, OFF_W2, OFF_B2, OFF_YCACHE = 30, 31, 32, 33, 34, 35
 STEP_STRIDE = 100
 
 
@@ -182,3 +196,24 @@ def blob_scores(w: Workload, device="cpu"):
     for b in range(nb):
         field += amp[b] * torch.exp(-((xx - cx[b]) ** 2 + (yy - cy[b]) ** 2) / (2 * sig[b] ** 2))
     return (field.reshape(-1) + noise).to(device)
+
+
+def ffn_weights(w: Workload, device="cpu", D=None, F=None):
+    """FFN parameters: W1 [F, D], W2 [D, F] bf16 (N(0,1)/sqrt(fan_in), rounded
+    after scaling), b1 [F], b2 [D] fp32 N(0, 0.02^2)."""
+    D = w.D_model if D is None else D
+    F = w.D_ff if F is None else F
+    w1 = (normal((F, D), w, OFF_W1, device, torch.float32) / math.sqrt(D)).to(torch.bfloat16)
+    w2 = (normal((D, F), w, OFF_W2, device, torch.float32) / math.sqrt(F)).to(torch.bfloat16)
+    b1 = 0.02 * normal((F,), w, OFF_B1, device, torch.float32)
+    b2 = 0.02 * normal((D,), w, OFF_B2, device, torch.float32)
+    return w1, b1, w2, b2
+
+
+def ffn_states(w: Workload, step: int = 0, device="cpu", D=None):
+    """Token states entering the FFN [B, N, D] bf16 and the FFN cache of the
+    previous step [B, N, D] bf16."""
+    D = w.D_model if D is None else D
+    o = STEP_STRIDE * step
+    return (normal((w.B, w.N, D), w, OFF_X + o, device),
+            normal((w.B, w.N, D), w, OFF_YCACHE + o, device))

@@ -29,7 +29,9 @@ def _rand_idx(n_total, k, seed):
 @pytest.mark.parametrize("D,dtype,B,H,N,k", [(96, torch.bfloat16, 2, 3, 1000, 300),
                                               (64, torch.bfloat16, 1, 2, 256, 64),
                                               (128, torch.bfloat16, 1, 4, 517, 517),
-                                              (16, torch.float32, 2, 2, 333, 1)])
+                                              (16, torch.float32, 2, 2, 333, 1),
+                                              (2304, torch.bfloat16, 2, 1, 700, 300),  # rows wider than a block
+                                              (1100, torch.float32, 1, 2, 90, 45)])
 def test_scatter_gather_bit_exact(D, dtype, B, H, N, k):
     g = _gen(D + N)
     idx = _rand_idx(N, k, N + k)

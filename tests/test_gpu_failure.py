@@ -38,10 +38,20 @@ def _run_xattn():
     return P
 
 
+def _run_gemm():
+    g = torch.Generator().manual_seed(7)
+    a = torch.randn(1000, 512, generator=g).to(torch.bfloat16).to(DEV)
+    w = torch.randn(768, 512, generator=g).to(torch.bfloat16).to(DEV)
+    out = torch.zeros(1000, 768, dtype=torch.bfloat16, device=DEV)
+    sd().safedit_gemm_bias_act(a, w, None, 1, None, out)
+    return out
+
+
 def test_bounded_wait_timeout_is_reported_and_context_survives():
     q, k, v, idx = _attn_case()
     ref = _run_attn(q, k, v, idx)
     ref_p = _run_xattn()
+    ref_g = _run_gemm()
     expect_status(0)
     old = sd().safedit_debug_set_wait_limit_ns(0)
     try:
@@ -49,13 +59,17 @@ def test_bounded_wait_timeout_is_reported_and_context_survives():
         expect_status(sd().ERR_TIMEOUT)
         _run_xattn()
         expect_status(sd().ERR_TIMEOUT)
+        _run_gemm()
+        expect_status(sd().ERR_TIMEOUT)
     finally:
         sd().safedit_debug_set_wait_limit_ns(old)
     again = _run_attn(q, k, v, idx)
     again_p = _run_xattn()
+    again_g = _run_gemm()
     expect_status(0)
     assert torch.equal(again, ref)
     assert torch.equal(again_p, ref_p)
+    assert torch.equal(again_g, ref_g)
 
 
 def test_device_errors_do_not_poison_later_calls():
