@@ -241,6 +241,8 @@ def run_ours(args):
     # ---- end to end through the public API with host buffers (pinned)
     e2e = run_e2e(tr, stream, args)
     e2e["ms"] = max_over_ranks([e2e["ms"]], dev)[0]
+    unfused = statistics.mean(per["cross_attn_probs"]) + statistics.mean(per["partition_accumulate"])
+    ext = measure_extensions(tr, stream, dev, unfused)
 
     if rank == 0:
         hbm, bf16_burst, bf16_sust, src = _peaks()
@@ -280,6 +282,7 @@ def run_ours(args):
                                "a dense masked path that materialises bf16 scores [B,H,N,N] would need "
                                f"{W.B * W.H * W.N * W.N * 2 / 1e9:.1f} GB for them alone"},
             "device_status": status,
+            "extensions": ext,
             "e2e": {"value": round(whole_job_tflops(tr.flop_srsu * n_srsu / args.steps, ws, e2e["ms"]), 3),
                     "unit": "TFLOP/s", "ms_per_step": round(e2e["ms"], 3),
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
@@ -291,6 +294,71 @@ def run_ours(args):
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def measure_extensions(tr, stream, dev, unfused_pcsp_ms, reps=5):
+    """The steps around the per-step path, each launched alone on the same
+    workload (best of `reps` CUDA-event timings after 2 warm-ups): the fused
+    PCSP score, SkipSparse's projections on the focus rows (gathered Q|K|V;
+    FFN W1 with bias and GELU; FFN W2 with bias, rows scattered into the FFN
+    cache) and the StepCache guidance combine."""
+    sd, w = tr.sd, tr.w
+    hbm, bf16_burst, _, src = _peaks()
+    k, D, F, B = tr.k, w.D_model, w.D_ff, w.B
+    w1, b1, w2, b2 = (t.to(dev) for t in wl.ffn_weights(w))
+    wqkv, bqkv = (t.to(dev) for t in wl.qkv_proj_weights(w))
+    x, y = (t.to(dev) for t in wl.ffn_states(w))
+    xs = torch.empty(B, 1, k, D, dtype=torch.bfloat16, device=dev)
+    xs3 = xs.view(B, k, D)
+    h = torch.empty(B, k, F, dtype=torch.bfloat16, device=dev)
+    qkv = torch.empty(B, k, 3 * D, dtype=torch.bfloat16, device=dev)
+    prev_c, prev_u = wl.cfg_preds(w, step=1, device=dev)
+
+    def best_ms(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                fn()
+            evs = []
+            for _ in range(reps):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                evs.append((a, b))
+        stream.synchronize()
+        return min(a.elapsed_time(b) for a, b in evs)
+
+    def gemm_entry(ms, flop):
+        tf = flop / (ms * 1e-3) / 1e12
+        return {"ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / bf16_burst, 3),
+                "peak": bf16_burst, "peak_kind": f"bf16_tflops burst ({src})"}
+
+    gather = lambda: sd.safedit_gather_rows([x.view(B, 1, w.N, D)], [xs], tr.idx_s, k, stream)
+    ffn1 = lambda: sd.safedit_gemm_bias_act(xs3, w1, b1, 1, None, h, stream)
+    ffn2 = lambda: sd.safedit_gemm_bias_act(h, w2, b2, 0, tr.idx_s, y, stream)
+    proj = lambda: sd.safedit_gemm_bias_act(xs3, wqkv, bqkv, 0, None, qkv, stream)
+    gather()
+    ffn_flop = 2.0 * B * k * D * F
+    out = {
+        "pcsp_fused": {"ms": round(best_ms(lambda: sd.safedit_pcsp_score(
+            tr.q_img, tr.k_txt, tr.valid, tr.content, 0, 0.0, tr.score, stream)), 4),
+            "unfused_ms": round(unfused_pcsp_ms, 4)},
+        "qkv_projection_gathered": gemm_entry(best_ms(proj), 2.0 * B * k * D * 3 * D),
+        "ffn_w1_bias_gelu": gemm_entry(best_ms(ffn1), ffn_flop),
+        "ffn_w2_bias_scatter": gemm_entry(best_ms(ffn2), ffn_flop),
+        "ffn_block_ms": round(best_ms(lambda: (gather(), ffn1(), ffn2())), 4),
+    }
+    sc_ms = best_ms(lambda: sd.safedit_stepcache_sw_cfg(prev_c, tr.eps_c, prev_u, tr.eps_u, tr.s, 0.5,
+                                                        w.gamma_ctx, w.gamma_sens, tr.cfg_out, stream))
+    sc_bytes = 5 * tr.eps_c.numel() * 4 + 4 * w.N
+    out["stepcache_sw_cfg"] = {"ms": round(sc_ms, 4), "gbs": round(sc_bytes / (sc_ms * 1e-3) / 1e9, 1),
+                               "note": f"F={tr.eps_c.shape[1]}: {sc_bytes / 1e6:.1f} MB, launch-bound"}
+    out["workload"] = (f"B={B}, |S|={k} focus rows per batch, D={D}, F={F}; "
+                       "synthetic weights N(0,1)/sqrt(fan_in)")
+    if sd.safedit_get_device_status(stream) != 0:
+        raise RuntimeError("device status set during the extension measurements")
+    return out
 
 
 def max_over_ranks(values, device):
@@ -500,7 +568,7 @@ def run_only(args):
     if args.only == "mask":
         extra["mask"] = torch.zeros(1, 1, wl.STRESS.N, wl.STRESS.N, dtype=torch.bfloat16, device=dev)
     ffn_flop = 2 * w.B * tr.k * w.D_model * w.D_ff  # one projection of the cached FFN
-    if args.only in ("ffn1", "ffn2", "ffn"):
+    if args.only in ("ffn1", "ffn2", "ffn", "qkv"):
         # SkipSparse FFN caching on the focus rows: gather, W1 (+b1, GELU), W2 (+b2) scattered
         w1, b1, w2, b2 = (t.to(dev) for t in wl.ffn_weights(w))
         x, y = (t.to(dev) for t in wl.ffn_states(w))
@@ -510,6 +578,9 @@ def run_only(args):
         xs3 = xs.view(w.B, tr.k, w.D_model)
         extra["ffn1"] = lambda: sd.safedit_gemm_bias_act(xs3, w1, b1, 1, None, h, stream)
         extra["ffn2"] = lambda: sd.safedit_gemm_bias_act(h, w2, b2, 0, tr.idx_s, y, stream)
+        wqkv, bqkv = (t.to(dev) for t in wl.qkv_proj_weights(w))
+        qkv = torch.empty(w.B, tr.k, 3 * w.D_model, dtype=torch.bfloat16, device=dev)
+        extra["qkv"] = lambda: sd.safedit_gemm_bias_act(xs3, wqkv, bqkv, 0, None, qkv, stream)
 
         def ffn_block():
             sd.safedit_gather_rows([x.view(w.B, 1, w.N, w.D_model)], [xs], tr.idx_s, tr.k, stream)
@@ -542,6 +613,7 @@ def run_only(args):
         "ffn1": (lambda: extra["ffn1"](), ffn_flop, None),
         "ffn2": (lambda: extra["ffn2"](), ffn_flop, None),
         "ffn": (lambda: extra["ffn"](), 2 * ffn_flop, None),
+        "qkv": (lambda: extra["qkv"](), 3 * ffn_flop / w.ffn_mult, None),
     }
     fn, flop, nbytes = fns[args.only]
     times = []
@@ -579,7 +651,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,
                     choices=["srsu", "anchor", "xattn", "accumulate", "pcsp", "finalize", "scatter", "cfg",
-                             "stepcache", "mask", "ffn1", "ffn2", "ffn"],
+                             "stepcache", "mask", "ffn1", "ffn2", "ffn", "qkv"],
                     help="run one kernel of the path in isolation (profiling target)")
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--cfg-f", type=int, default=W.F, help="prediction width for --only cfg")

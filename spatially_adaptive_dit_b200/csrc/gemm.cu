@@ -33,7 +33,10 @@ struct GemmParams {
   int64_t out_rs, out_bs;  // row / batch strides (elements)
   const int* idx;          // nullable: output row of A row r is idx[r] (every batch)
   int M, N, K, M_out, act;
-  int tiles_m, tiles_bm, tiles;  // row tiles per batch, x batches, x column tiles
+  // row tiles per batch, column tiles, all tiles (B x tiles_m x tiles_n).  The
+  // column index runs fastest, so the CTAs in flight share a few row blocks
+  // of A and sweep all of W: W stays in L2 and A is read from HBM once.
+  int tiles_m, tiles_n, tiles;
   int* status;
   uint64_t wait_limit;
 };
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       int g = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
-        const int bm = t % p.tiles_bm, n0 = (t / p.tiles_bm) * kGBN;
+        const int bm = t / p.tiles_n, n0 = (t % p.tiles_n) * kGBN;
         const int bb = bm / p.tiles_m, m0 = (bm % p.tiles_m) * kGBM;
         for (int j = 0; j < nk; ++j, ++g) {
           const int s = g % kGNS;
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     int i = 0;
     for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++i) {
       const int b = i & 1;
-      const int bm = t % p.tiles_bm, n0 = (t / p.tiles_bm) * kGBN + hh * (kGBN / 2);
+      const int bm = t / p.tiles_n, n0 = (t % p.tiles_n) * kGBN + hh * (kGBN / 2);
       const int bb = bm / p.tiles_m, r = (bm % p.tiles_m) * kGBM + q * 32 + lane;
       // row destination and this warp's 128 bias values, fetched while the
       // accumulator is still being computed
@@ -295,8 +298,8 @@ extern "C" safedit_status safedit_gemm_bias_act(const safedit_tensor* a, const s
   if (N % 8 != 0) return SAFEDIT_ERR_ALIGNMENT;  // whole 16-byte output units
   if (M == 0 || N == 0 || B == 0) return SAFEDIT_OK;
   if (K == 0) return SAFEDIT_ERR_SHAPE;
-  const int64_t tiles_m = (M + kGBM - 1) / kGBM, tiles_bm = tiles_m * B;
-  const int64_t tiles = tiles_bm * ((N + kGBN - 1) / kGBN);
+  const int64_t tiles_m = (M + kGBM - 1) / kGBM, tiles_n = (N + kGBN - 1) / kGBN;
+  const int64_t tiles = tiles_m * B * tiles_n;
   if (tiles > INT32_MAX) return SAFEDIT_ERR_SHAPE;
   GemmParams p{};
   p.bias = d_bias;
@@ -310,7 +313,7 @@ extern "C" safedit_status safedit_gemm_bias_act(const safedit_tensor* a, const s
   p.M_out = static_cast<int>(M_out);
   p.act = act;
   p.tiles_m = static_cast<int>(tiles_m);
-  p.tiles_bm = static_cast<int>(tiles_bm);
+  p.tiles_n = static_cast<int>(tiles_n);
   p.tiles = static_cast<int>(tiles);
   p.wait_limit = wait_limit_ns();
   CUtensorMap tA, tW;

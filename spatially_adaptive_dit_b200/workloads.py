@@ -22,7 +22,8 @@ per-tensor offset so that tensors are independent):
   * FFN block (model width D = H d, hidden width F = ffn_mult D): token
     states N(0,1) [B, N, D] bf16; W1 [F, D] and W2 [D, F] N(0,1) / sqrt(fan_in)
     (random init, nn.Linear layout), biases N(0, 0.02^2) fp32; the cached FFN
-    output of the previous step N(0,1) [B, N, D] bf16.
+    output of the previous step N(0,1) [B, N, D] bf16; the fused Q|K|V
+    projection W_qkv [3D, D] N(0,1) / sqrt(D) bf16 with bias N(0, 0.02^2).
 """
 from dataclasses import dataclass, field
 from fractions import Fraction
@@ -108,7 +109,7 @@ def uniform(shape, lo, hi, w: Workload, offset: int, device="cpu", dtype=torch.f
 # Tensor offsets (kept distinct so every tensor is an independent draw).
 OFF_Q, OFF_K, OFF_V, OFF_QX, OFF_KTXT, OFF_KS, OFF_VS, OFF_EPSC, OFF_EPSU = range(1, 10)
 OFF_MASK_ROW, OFF_MASK_BIAS, OFF_BLOB = 20, 21, 22
-OFF_X, OFF_W1, OFF_B1, OFF_W2, OFF_B2, OFF_YCACHE = 30, 31, 32, 33, 34, 35
+OFF_X, OFF_W1, OFF_B1, OFF_W2, OFF_B2, OFF_YCACHE, OFF_WQKV, OFF_BQKV = 30, 31, 32, 33, 34, 35, 36, 37
 STEP_STRIDE = 100
 
 
@@ -217,3 +218,12 @@ def ffn_states(w: Workload, step: int = 0, device="cpu", D=None):
     o = STEP_STRIDE * step
     return (normal((w.B, w.N, D), w, OFF_X + o, device),
             normal((w.B, w.N, D), w, OFF_YCACHE + o, device))
+
+
+def qkv_proj_weights(w: Workload, device="cpu", D=None):
+    """Fused Q|K|V projection: W_qkv [3D, D] bf16 (N(0,1)/sqrt(D)), b [3D]
+    fp32 N(0, 0.02^2); output features ordered (q|k|v, head, d)."""
+    D = w.D_model if D is None else D
+    wq = (normal((3 * D, D), w, OFF_WQKV, device, torch.float32) / math.sqrt(D)).to(torch.bfloat16)
+    bq = 0.02 * normal((3 * D,), w, OFF_BQKV, device, torch.float32)
+    return wq, bq

@@ -197,3 +197,45 @@ def test_projection_argument_and_device_errors():
     expect_status(0)
     rows = torch.tensor([r for r in range(64) if r != 5], device=DEV)
     assert torch.equal(out[rows], ref[rows])
+
+
+def test_gathered_qkv_projection_feeds_srsu():
+    """SkipSparse on one attention layer: only the focus rows are projected
+    (x_S W_qkv^T + b, fused q|k|v output with heads inner), their K/V replace
+    the cached rows of the state, and their Q attends over the whole state,
+    read through strided views of the projection output.  Against the oracle
+    composed from gather, linear_act, scatter and attn_subset in fp64.
+    Tolerance: two bf16 roundings in sequence (projection outputs, then the
+    attention's P and O), each about 2e-3 relative: relative Frobenius <= 1e-2."""
+    B, H, d, N, k = 2, 2, 64, 384, 100
+    D = H * d
+    g = _gen(61)
+    x = torch.randn(B, N, D, generator=g).to(torch.bfloat16)
+    wqkv = (torch.randn(3 * D, D, generator=g) / D ** 0.5).to(torch.bfloat16)
+    bqkv = 0.02 * torch.randn(3 * D, generator=g)
+    k_state = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    v_state = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    idx = _rand_idx(N, k, 62)
+    # GPU: gather -> projection -> scatter K/V -> compact-query attention
+    d_idx = idx.to(DEV)
+    xs = torch.empty(B, 1, k, D, dtype=torch.bfloat16, device=DEV)
+    sd().safedit_gather_rows([x.to(DEV).view(B, 1, N, D)], [xs], d_idx, k)
+    qkv = torch.empty(B, k, 3 * D, dtype=torch.bfloat16, device=DEV)
+    sd().safedit_gemm_bias_act(xs.view(B, k, D), wqkv.to(DEV), bqkv.to(DEV), 0, None, qkv)
+    q_s, k_s, v_s = (qkv.view(B, k, 3, H, d)[:, :, j].permute(0, 2, 1, 3) for j in range(3))
+    ks_d, vs_d = k_state.to(DEV), v_state.to(DEV)
+    sd().safedit_scatter_state([k_s, v_s], [ks_d, vs_d], d_idx, k)
+    out = torch.empty(B, H, k, d, dtype=torch.bfloat16, device=DEV)
+    sd().safedit_attn_subset(q_s, ks_d, vs_d, None, 0, None, None, 0.0, out, 0)
+    expect_status(0)
+    # oracle composition
+    for bb in range(B):
+        x_s = oracle.gather_rows(x[bb].view(torch.int16).numpy(), idx)
+        x_s = torch.from_numpy(x_s).view(torch.bfloat16)
+        proj = oracle.linear_act(x_s, wqkv, bqkv, act=0).reshape(k, 3, H, d)
+        for h in range(H):
+            kst = oracle.scatter_rows(proj[:, 1, h], f64(k_state[bb, h]), idx)
+            vst = oracle.scatter_rows(proj[:, 2, h], f64(v_state[bb, h]), idx)
+            ref = oracle.attn_subset(proj[:, 0, h], kst, vst)
+            rf = rel_fro(f64(out[bb, h]), ref)
+            assert rf <= 1e-2, f"b{bb}h{h}: relFro={rf:.3e}"
