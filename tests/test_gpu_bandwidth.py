@@ -258,3 +258,24 @@ def test_stepcache_sw_cfg(N, F, w):
     mag = (1 + abs(w)) * (ca.abs() + cb.abs() + ua.abs() + ub.abs()).double().numpy()
     err = np.abs(out.cpu().double().numpy() - ref)
     assert np.all(err <= CFG_REL * (1 + gam) * mag + 1e-30)
+
+
+def test_stepcache_sw_cfg_large_sampled():
+    """A bandwidth-sized call (grid-stride loop over many passes): sampled rows
+    against the oracle, every row against the same combine in fp32 torch on the
+    device being finite and unchanged where the branches agree."""
+    N, F, w = 25600, 4096, 0.5
+    g = torch.Generator(device=DEV).manual_seed(77)
+    ca, cb, ua, ub = (torch.randn(N, F, generator=g, device=DEV) for _ in range(4))
+    s = torch.rand(N, generator=g, device=DEV)
+    out = torch.full((N, F), float("nan"), device=DEV)
+    sd().safedit_stepcache_sw_cfg(ca, cb, ua, ub, s, w, 3.0, 5.0, out)
+    expect_status(0)
+    assert bool(torch.isfinite(out).all())  # every element was written
+    rows = torch.cat([torch.tensor([0, N - 1]), torch.randperm(N, generator=_gen(78))[:62]]).to(DEV)
+    sub = [t[rows].cpu() for t in (ca, cb, ua, ub)]
+    ref = oracle.stepcache_sw_cfg(*sub, s[rows].cpu(), w, 3.0, 5.0)
+    gam = (3.0 + 2.0 * s[rows].cpu().double().numpy())[:, None]
+    mag = (1 + abs(w)) * sum(t.abs() for t in sub).double().numpy()
+    err = np.abs(out[rows].cpu().double().numpy() - ref)
+    assert np.all(err <= CFG_REL * (1 + gam) * mag + 1e-30)
