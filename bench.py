@@ -402,10 +402,12 @@ def run_e2e(tr, stream, args):
     fresh S rows -- Q_S, K_S, V_S compact [B,H,k,d] (the projections of an
     SRSU step run on the S rows alone) -- plus eps_c, eps_u every step.  An
     SRSU step is then: scatter K_S, V_S into the cached state, attention of the
-    compact Q_S over all N keys, scatter O_S into O_state.  A copy stream fills
-    a second buffer set for step t+1 while step t computes; events order every
-    buffer reuse."""
+    compact Q_S over all N keys, scatter O_S into O_state.  A copy stream runs
+    ahead of the compute stream: three input buffer sets, and two K/V state
+    sets that alternate between anchors, so that an anchor's full K/V upload
+    never waits for the step before it; events order every buffer reuse."""
     w = tr.w
+    NSET = 3
     names = ("q", "q_s", "k_s", "v_s", "q_img", "k_txt", "eps_c", "eps_u")
     q_s = tr.q[:, :, : tr.k].contiguous()
     o_s = torch.empty_like(q_s)
@@ -415,38 +417,43 @@ def run_e2e(tr, stream, args):
         t = dev_t.get(n, getattr(tr, n, None))
         host[n] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
         host[n].copy_(t)
-    sets = [{n: dev_t.get(n, getattr(tr, n, None)) for n in names},
-            {n: torch.empty_like(host[n], device=tr.dev) for n in names}]
-    out_h = [torch.empty(tr.cfg_out.shape, dtype=tr.cfg_out.dtype, pin_memory=True) for _ in range(2)]
+    sets = [{n: dev_t.get(n, getattr(tr, n, None)) for n in names}] + \
+        [{n: torch.empty_like(host[n], device=tr.dev) for n in names} for _ in range(NSET - 1)]
+    states = [(tr.k_state, tr.v_state), (torch.empty_like(tr.k_state), torch.empty_like(tr.v_state))]
+    out_h = [torch.empty(tr.cfg_out.shape, dtype=tr.cfg_out.dtype, pin_memory=True) for _ in range(NSET)]
     copy_stream = torch.cuda.Stream(device=tr.dev)
     sd = tr.sd
     counts = {"h2d": 0, "d2h": 0}
-    freed = [None, None]  # per buffer set: event after the last step that used it
+    freed = [None] * NSET          # per input set: event after the last step that used it
+    state_freed = [None, None]     # per state set: event after the last step that read it
+    cur_state = [1]                # the state set in use (flips at every anchor)
 
     def trajectory(count):
         with torch.cuda.stream(stream):
             tr.score.zero_()
         for t in range(w.steps):
             anchor = (t % w.period == 0)
-            cur = sets[t % 2]
+            cur = sets[t % NSET]
             need = ["eps_c", "eps_u"] + (["q_img", "k_txt"] if t < w.warmup else []) + \
                 (["q"] if anchor else ["q_s", "k_s", "v_s"])
             ready = torch.cuda.Event()
             with torch.cuda.stream(copy_stream):
-                if freed[t % 2] is not None:
-                    copy_stream.wait_event(freed[t % 2])  # step t-2 is done with this set
+                if freed[t % NSET] is not None:
+                    copy_stream.wait_event(freed[t % NSET])  # step t-NSET is done with this set
                 for n in need:
                     cur[n].copy_(host[n], non_blocking=True)
                     if count:
                         counts["h2d"] += host[n].numel() * host[n].element_size()
                 if anchor:
-                    if freed[(t + 1) % 2] is not None:
-                        copy_stream.wait_event(freed[(t + 1) % 2])  # step t-1 still reads the state
-                    for n, dst in (("k_full", tr.k_state), ("v_full", tr.v_state)):
+                    cur_state[0] ^= 1
+                    if state_freed[cur_state[0]] is not None:
+                        copy_stream.wait_event(state_freed[cur_state[0]])  # the previous anchor period
+                    for n, dst in zip(("k_full", "v_full"), states[cur_state[0]]):
                         dst.copy_(host[n], non_blocking=True)
                         if count:
                             counts["h2d"] += host[n].numel() * host[n].element_size()
                 ready.record(copy_stream)
+            k_st, v_st = states[cur_state[0]]
             stream.wait_event(ready)
             with torch.cuda.stream(stream):
                 if t < w.warmup:
@@ -457,22 +464,21 @@ def run_e2e(tr, stream, args):
                 if t == 0:
                     sd.safedit_mask_is_row_constant(tr.mask, tr.verdict, None, stream)
                 if anchor:
-                    sd.safedit_attn_subset(cur["q"], tr.k_state, tr.v_state, None, 0, None, None, 0.0,
+                    sd.safedit_attn_subset(cur["q"], k_st, v_st, None, 0, None, None, 0.0,
                                            tr.o_state, 0, stream)
                 else:
-                    sd.safedit_scatter_state([cur["k_s"], cur["v_s"]], [tr.k_state, tr.v_state], tr.idx_s,
-                                             tr.k, stream)
-                    sd.safedit_attn_subset(cur["q_s"], tr.k_state, tr.v_state, None, 0, None, None, 0.0,
-                                           o_s, 0, stream)
+                    sd.safedit_scatter_state([cur["k_s"], cur["v_s"]], [k_st, v_st], tr.idx_s, tr.k, stream)
+                    sd.safedit_attn_subset(cur["q_s"], k_st, v_st, None, 0, None, None, 0.0, o_s, 0, stream)
                     sd.safedit_scatter_state([o_s], [tr.o_state], tr.idx_s, tr.k, stream)
                 g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx
                 sd.safedit_sw_cfg(cur["eps_c"], cur["eps_u"], tr.s, w.gamma_ctx, g_sens, tr.cfg_out, stream)
-                out_h[t % 2].copy_(tr.cfg_out, non_blocking=True)
+                out_h[t % NSET].copy_(tr.cfg_out, non_blocking=True)
                 if count:
-                    counts["d2h"] += out_h[t % 2].numel() * out_h[t % 2].element_size()
+                    counts["d2h"] += out_h[t % NSET].numel() * out_h[t % NSET].element_size()
                 ev = torch.cuda.Event()
                 ev.record(stream)
-                freed[t % 2] = ev
+                freed[t % NSET] = ev
+                state_freed[cur_state[0]] = ev
 
     trajectory(False)
     torch.cuda.synchronize()

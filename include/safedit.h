@@ -15,7 +15,10 @@
  * - Memory.  Every pointer named d_* and every safedit_tensor.data is DEVICE
  *   memory on the current CUDA device; host_* pointers are host memory.  The
  *   caller owns and allocates every buffer.  The library allocates nothing
- *   except one static device status word per device.
+ *   except one static device status word per device.  A pointer to an array
+ *   with no elements (an empty tensor, a zero-length vector) may be NULL.
+ * - Empty work.  A call whose work is empty (no rows, no tokens, no
+ *   columns) checks its arguments, launches nothing and returns SAFEDIT_OK.
  * - Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream).
  *   Every call only enqueues work on that stream and returns without
  *   synchronising, except safedit_get_device_status.

@@ -268,25 +268,11 @@ extern "C" safedit_status safedit_gemm_bias_act(const safedit_tensor* a, const s
   const int rank = a->ndim;
   if (rank != 2 && rank != 3) return SAFEDIT_ERR_SHAPE;
   safedit_status st;
-  // an empty operand may come with a null data pointer: check it as if it had one
-  auto check = [](const safedit_tensor* t, int nd) {
-    bool empty = false;
-    for (int i = 0; i < nd && i < 4; ++i) empty = empty || t->dims[i] == 0;
-    safedit_tensor c = *t;
-    if (empty && !c.data) c.data = reinterpret_cast<void*>(uintptr_t(256));
-    return check_tensor(&c, nd);
-  };
-  if ((st = check(a, rank)) != SAFEDIT_OK) return st;
-  if ((st = check(w, 2)) != SAFEDIT_OK) return st;
-  if ((st = check(out, rank)) != SAFEDIT_OK) return st;
-  for (const safedit_tensor* t : {a, w, out}) {
+  if ((st = check_tensor(a, rank)) != SAFEDIT_OK) return st;
+  if ((st = check_tensor(w, 2)) != SAFEDIT_OK) return st;
+  if ((st = check_tensor(out, rank)) != SAFEDIT_OK) return st;
+  for (const safedit_tensor* t : {a, w, out})
     if (t->dtype != SAFEDIT_BF16) return SAFEDIT_ERR_DTYPE;
-    const int r = t->ndim;
-    if (t->strides[r - 1] != 1 || t->strides[r - 2] <= 0 || t->strides[r - 2] % 8 != 0 ||
-        (t->data && !aligned16(t->data)))
-      return SAFEDIT_ERR_ALIGNMENT;
-    if (r == 3 && (t->strides[0] <= 0 || t->strides[0] % 8 != 0)) return SAFEDIT_ERR_ALIGNMENT;
-  }
   const int64_t B = rank == 3 ? a->dims[0] : 1;
   const int64_t M = a->dims[rank - 2], K = a->dims[rank - 1], N = w->dims[0];
   const int64_t M_out = out->dims[rank - 2];
@@ -296,8 +282,15 @@ extern "C" safedit_status safedit_gemm_bias_act(const safedit_tensor* a, const s
   if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || M_out > INT32_MAX) return SAFEDIT_ERR_SHAPE;
   if (act != 0 && act != 1) return SAFEDIT_ERR_INVALID_ARG;
   if (N % 8 != 0) return SAFEDIT_ERR_ALIGNMENT;  // whole 16-byte output units
-  if (M == 0 || N == 0 || B == 0) return SAFEDIT_OK;
+  if (M == 0 || N == 0 || B == 0) return SAFEDIT_OK;  // strides of empty tensors are not checked
   if (K == 0) return SAFEDIT_ERR_SHAPE;
+  for (const safedit_tensor* t : {a, w, out}) {
+    const int r = t->ndim;
+    if (t->strides[r - 1] != 1 || t->strides[r - 2] <= 0 || t->strides[r - 2] % 8 != 0 ||
+        !aligned16(t->data))
+      return SAFEDIT_ERR_ALIGNMENT;
+    if (r == 3 && (t->strides[0] <= 0 || t->strides[0] % 8 != 0)) return SAFEDIT_ERR_ALIGNMENT;
+  }
   const int64_t tiles_m = (M + kGBM - 1) / kGBM, tiles_n = (N + kGBN - 1) / kGBN;
   const int64_t tiles = tiles_m * B * tiles_n;
   if (tiles > INT32_MAX) return SAFEDIT_ERR_SHAPE;

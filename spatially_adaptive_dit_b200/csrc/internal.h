@@ -26,14 +26,20 @@ inline int elt_size(int dtype) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Basic structural check of a tensor argument: non-null, known dtype,
-// ndim in range, non-negative dims.
+// Basic structural check of a tensor argument: non-null descriptor, known
+// dtype, ndim as expected, non-negative dims, and a data pointer unless the
+// tensor is empty (an empty tensor may carry a null pointer; every entry point
+// returns before launching anything when its work is empty).
 inline safedit_status check_tensor(const safedit_tensor* t, int ndim) {
-  if (!t || !t->data) return SAFEDIT_ERR_INVALID_ARG;
+  if (!t) return SAFEDIT_ERR_INVALID_ARG;
   if (elt_size(t->dtype) == 0) return SAFEDIT_ERR_DTYPE;
-  if (t->ndim != ndim) return SAFEDIT_ERR_SHAPE;
-  for (int i = 0; i < ndim; ++i)
+  if (t->ndim != ndim || ndim < 1 || ndim > 4) return SAFEDIT_ERR_SHAPE;
+  bool empty = false;
+  for (int i = 0; i < ndim; ++i) {
     if (t->dims[i] < 0) return SAFEDIT_ERR_SHAPE;
+    empty = empty || t->dims[i] == 0;
+  }
+  if (!t->data && !empty) return SAFEDIT_ERR_INVALID_ARG;
   return SAFEDIT_OK;
 }
 

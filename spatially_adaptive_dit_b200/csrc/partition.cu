@@ -275,7 +275,8 @@ safedit_status safedit_partition_accumulate(const safedit_tensor* p, const uint8
                                             double* d_score, void* stream) {
   safedit_status st;
   if ((st = check_tensor(p, 3)) != SAFEDIT_OK) return st;
-  if (!d_content || !d_score) return SAFEDIT_ERR_INVALID_ARG;
+  if ((p->dims[2] > 0 && !d_content) || (p->dims[1] > 0 && !d_score))
+    return SAFEDIT_ERR_INVALID_ARG;
   if (p->dtype != SAFEDIT_F32) return SAFEDIT_ERR_DTYPE;
   if (p->strides[2] != 1) return SAFEDIT_ERR_ALIGNMENT;
   AccParams a;
@@ -317,8 +318,9 @@ safedit_status safedit_partition_accumulate(const safedit_tensor* p, const uint8
 safedit_status safedit_partition_finalize(const double* d_score, int32_t n, int32_t k,
                                           int32_t* d_idx_s, int32_t* d_idx_c, float* d_s,
                                           void* stream) {
-  if (!d_score || n < 0 || k < 0 || k > n || n > (1 << 24)) return SAFEDIT_ERR_INVALID_ARG;
+  if (n < 0 || k < 0 || k > n || n > (1 << 24)) return SAFEDIT_ERR_INVALID_ARG;
   if (n == 0) return SAFEDIT_OK;
+  if (!d_score) return SAFEDIT_ERR_INVALID_ARG;
   int* status = status_ptr();
   if (!status) return SAFEDIT_ERR_CUDA;
   finalize_kernel<<<1, kFinThreads, 0, static_cast<cudaStream_t>(stream)>>>(d_score, n, k, d_idx_s,

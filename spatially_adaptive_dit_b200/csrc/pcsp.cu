@@ -302,8 +302,9 @@ extern "C" safedit_status safedit_pcsp_score(const safedit_tensor* q_img, const 
     for (int i = 0; i < 3; ++i)
       if (t->strides[i] % 8 != 0 || t->strides[i] < 0) return SAFEDIT_ERR_ALIGNMENT;
   }
-  if (!d_key_valid || !d_content || !d_score) return SAFEDIT_ERR_INVALID_ARG;
+  if (!d_key_valid || !d_content) return SAFEDIT_ERR_INVALID_ARG;
   const int64_t B = q_img->dims[0], H = q_img->dims[1], N = q_img->dims[2], D = q_img->dims[3];
+  if (N > 0 && !d_score) return SAFEDIT_ERR_INVALID_ARG;
   const int64_t L = k_txt->dims[2];
   if (k_txt->dims[0] != B || k_txt->dims[1] != H || k_txt->dims[3] != D) return SAFEDIT_ERR_SHAPE;
   if (batch_index < 0 || batch_index >= B) return SAFEDIT_ERR_INVALID_ARG;

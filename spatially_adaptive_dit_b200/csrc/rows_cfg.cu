@@ -277,7 +277,6 @@ safedit_status safedit_sw_cfg(const safedit_tensor* eps_c, const safedit_tensor*
   if ((st = check_tensor(eps_c, 2)) != SAFEDIT_OK) return st;
   if ((st = check_tensor(eps_u, 2)) != SAFEDIT_OK) return st;
   if ((st = check_tensor(out, 2)) != SAFEDIT_OK) return st;
-  if (!d_s) return SAFEDIT_ERR_INVALID_ARG;
   if (eps_c->dtype != SAFEDIT_F32 || eps_u->dtype != SAFEDIT_F32 || out->dtype != SAFEDIT_F32)
     return SAFEDIT_ERR_DTYPE;
   const int64_t N = eps_c->dims[0], F = eps_c->dims[1];
@@ -286,6 +285,7 @@ safedit_status safedit_sw_cfg(const safedit_tensor* eps_c, const safedit_tensor*
   if (eps_c->strides[1] != 1 || eps_u->strides[1] != 1 || out->strides[1] != 1)
     return SAFEDIT_ERR_ALIGNMENT;
   if (N == 0 || F == 0) return SAFEDIT_OK;
+  if (!d_s) return SAFEDIT_ERR_INVALID_ARG;
   CfgParams p;
   p.c = static_cast<const float*>(eps_c->data);
   p.u = static_cast<const float*>(eps_u->data);
@@ -324,7 +324,6 @@ safedit_status safedit_stepcache_sw_cfg(const safedit_tensor* eps_c_a, const saf
   for (const safedit_tensor* t : ins)
     if ((st = check_tensor(t, 2)) != SAFEDIT_OK) return st;
   if ((st = check_tensor(out, 2)) != SAFEDIT_OK) return st;
-  if (!d_s) return SAFEDIT_ERR_INVALID_ARG;
   const int64_t N = out->dims[0], F = out->dims[1];
   for (const safedit_tensor* t : ins) {
     if (t->dtype != SAFEDIT_F32) return SAFEDIT_ERR_DTYPE;
@@ -334,6 +333,7 @@ safedit_status safedit_stepcache_sw_cfg(const safedit_tensor* eps_c_a, const saf
   if (out->dtype != SAFEDIT_F32) return SAFEDIT_ERR_DTYPE;
   if (out->strides[1] != 1) return SAFEDIT_ERR_ALIGNMENT;
   if (N == 0 || F == 0) return SAFEDIT_OK;
+  if (!d_s) return SAFEDIT_ERR_INVALID_ARG;
   StepCacheParams p;
   p.ca = static_cast<const float*>(eps_c_a->data);
   p.cb = static_cast<const float*>(eps_c_b->data);

@@ -144,9 +144,21 @@ def safedit_mask_is_row_constant(mask, verdict, row_flags=None, stream=None):
                                              _stream(stream)), "safedit_mask_is_row_constant")
 
 
+# A NULL row index means "every row" to safedit_attn_subset, while torch hands
+# out a null data pointer for an empty tensor: an empty index is passed as this
+# non-null address instead (never dereferenced, since n_idx is then 0).
+_EMPTY_INDEX = ctypes.c_void_p(16)
+
+
+def _idx_ptr(idx):
+    if idx is not None and idx.numel() == 0:
+        return _EMPTY_INDEX
+    return _ptr(idx)
+
+
 def safedit_attn_subset(q, k, v, idx, n_idx, key_pad, bias, scale, out, out_scattered,
                         stream=None):
-    _check(_lib.safedit_attn_subset(_ref(q), _ref(k), _ref(v), _ptr(idx), int(n_idx), _ref(key_pad),
+    _check(_lib.safedit_attn_subset(_ref(q), _ref(k), _ref(v), _idx_ptr(idx), int(n_idx), _ref(key_pad),
                                     _ref(bias), float(scale), _ref(out), int(out_scattered),
                                     _stream(stream)), "safedit_attn_subset")
 
