@@ -548,6 +548,48 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """The 3072^2 sensitive-fraction sweep (B=2, H=24, N=36864, d=96): SRSU
+    attention of |S| = rho N gathered rows over all N keys, scattered into the
+    output state, for rho in {0.1, 0.2, 0.3, 0.5}, and the dense anchor
+    (rho = 1).  Best of `--reps` CUDA-event timings per point; one JSON line
+    per point (not a bench line)."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    from spatially_adaptive_dit_b200 import safedit as sd
+    w = wl.W3072
+    _, bf16_burst, _, src = _peaks()
+    q, k, v = wl.qkv(w, device=dev)
+    o = torch.zeros_like(q)
+    stream = torch.cuda.Stream(device=dev)
+    g = torch.Generator().manual_seed(3072)
+    perm = torch.randperm(w.N, generator=g)
+    for rho in w.rho_sweep:
+        kk = wl.k_of(rho, w.N)
+        dense = kk == w.N
+        idx = None if dense else torch.sort(perm[:kk]).values.to(torch.int32).to(dev)
+        times = []
+        with torch.cuda.stream(stream):
+            for _ in range(args.reps + 1):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                sd.safedit_attn_subset(q, k, v, idx, 0 if dense else kk, None, None, 0.0, o,
+                                       0 if dense else 1, stream)
+                b.record(stream)
+                times.append((a, b))
+        stream.synchronize()
+        ms = min(a.elapsed_time(b) for a, b in times[1:])
+        flop = 4.0 * kk * w.N * w.d * w.B * w.H
+        tf = flop / (ms * 1e-3) / 1e12
+        status = sd.safedit_get_device_status(stream)
+        print(json.dumps({"sweep": "3072", "rho": float(rho), "rows": kk, "dense": dense, "ms": round(ms, 4),
+                          "tflops": round(tf, 1), "frac_of_burst": round(tf / bf16_burst, 3),
+                          "peak": f"bf16_tflops {bf16_burst} ({src})", "status": status}), flush=True)
+        if status != 0:
+            sys.exit(3)
+
+
 def run_only(args):
     """One kernel of the path in isolation, `--reps` times on the bench
     workload's buffers (the target of ncu captures and quick timing).  Prints
@@ -657,11 +699,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,
                     choices=["srsu", "anchor", "xattn", "accumulate", "pcsp", "finalize", "scatter", "cfg",
-                             "stepcache", "mask", "ffn1", "ffn2", "ffn", "qkv"],
+                             "stepcache", "mask", "ffn1", "ffn2", "ffn", "qkv", "sweep"],
                     help="run one kernel of the path in isolation (profiling target)")
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--cfg-f", type=int, default=W.F, help="prediction width for --only cfg")
     args = ap.parse_args()
+    if args.only == "sweep":
+        run_sweep(args)
+        return
     if args.only:
         run_only(args)
         return
