@@ -410,12 +410,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         c * C::CH, j * C::BN, h, b);
           issued_v = j + 1;
         }
-        if (*abort_flag) {  // drain the loads still in flight before leaving
-          for (int j = (issued_k > C::NS ? issued_k - C::NS : 0); j < issued_k; ++j)
-            wait_drain(BAR(K_FULL + j % C::NS), uint32_t((j / C::NS) & 1), kDrainNs);
-          for (int j = (issued_v > C::NS ? issued_v - C::NS : 0); j < issued_v; ++j)
-            wait_drain(BAR(V_FULL + j % C::NS), uint32_t((j / C::NS) & 1), kDrainNs);
-        }
+        // every copy has landed before the CTA leaves (already true unless a
+        // role aborted before consuming it)
+        for (int j = (issued_k > C::NS ? issued_k - C::NS : 0); j < issued_k; ++j)
+          wait_drain(BAR(K_FULL + j % C::NS), uint32_t((j / C::NS) & 1), kDrainNs);
+        for (int j = (issued_v > C::NS ? issued_v - C::NS : 0); j < issued_v; ++j)
+          wait_drain(BAR(V_FULL + j % C::NS), uint32_t((j / C::NS) & 1), kDrainNs);
       }
     } else if (warp == 9) {
       // ================================================ MMA issuer
@@ -484,12 +484,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_commit(BAR(K_EMPTY + s1));
           }
         }
-        if (ok) {
-          tc_commit(BAR(O_FULL));
-        } else {  // wait for every MMA already issued before TMEM is freed
-          tc_commit(BAR(DRAIN));
-          wait_drain(BAR(DRAIN), 0u, kDrainNs);
-        }
+        if (ok) tc_commit(BAR(O_FULL));
+        // every MMA has completed before TMEM is freed, whoever aborted
+        tc_commit(BAR(DRAIN));
+        wait_drain(BAR(DRAIN), 0u, kDrainNs);
       }
     }
   }

@@ -227,10 +227,10 @@ __global__ void __launch_bounds__(320, 1)
         }
         issued = n + 1;
       }
-      if (*abort_flag) {
-        for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
-          wait_drain(BAR(0 + (n & 1)), uint32_t((n >> 1) & 1), kPDrainNs);
-      }
+      // every copy has landed before the CTA leaves (already true unless a
+      // role aborted before consuming it)
+      for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
+        wait_drain(BAR(0 + (n & 1)), uint32_t((n >> 1) & 1), kPDrainNs);
     }
   } else {
     // ============================================= MMA issuer
@@ -256,10 +256,9 @@ __global__ void __launch_bounds__(320, 1)
         tc_commit(BAR(4 + st));
         tc_commit(BAR(2 + st));
       }
-      if (!ok) {
-        tc_commit(BAR(10));
-        wait_drain(BAR(10), 0u, kPDrainNs);
-      }
+      // every MMA has completed before TMEM is freed, whoever aborted
+      tc_commit(BAR(10));
+      wait_drain(BAR(10), 0u, kPDrainNs);
     }
   }
 

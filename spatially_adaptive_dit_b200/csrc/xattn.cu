@@ -34,10 +34,12 @@ struct XCfg {
   // softmax (the MMA frees the stage long before the softmax ends); the smem
   // goes to staging so that more TMA stores stay in flight.
   static constexpr int NSTAGE = 1;
-  static constexpr int NOUT = 4;                       // staging buffers per warpgroup
+  static constexpr int NOUT = (D == 128) ? 3 : 4;      // staging buffers per warpgroup
   static constexpr int OUT_BYTES = 128 * 128;          // 128 rows x 32 f32
+  // + one all-zero box that every all-padding chunk is stored from
   static constexpr int SMEM_BYTES =
-      1024 + NSTAGE * STAGE_BYTES + 2 * NOUT * OUT_BYTES + 256 + 1024;
+      1024 + NSTAGE * STAGE_BYTES + (2 * NOUT + 1) * OUT_BYTES + 256 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 struct XParams {
@@ -69,7 +71,8 @@ __global__ void __launch_bounds__(320, 1)
                                              ~uintptr_t(1023));
   const uint32_t sStage = smem_u32(smem);
   const uint32_t sOut = sStage + C::NSTAGE * C::STAGE_BYTES;  // 2 x NOUT staging buffers
-  uint8_t* tail = smem + C::NSTAGE * C::STAGE_BYTES + 2 * C::NOUT * C::OUT_BYTES;
+  const uint32_t sZero = sOut + 2 * C::NOUT * C::OUT_BYTES;   // zeros, never rewritten
+  uint8_t* tail = smem + C::NSTAGE * C::STAGE_BYTES + (2 * C::NOUT + 1) * C::OUT_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(tail);
   // bars: [0,2) stage_full, [2,4) stage_empty, [4,6) s_full, [6,8) s_empty, 8 drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + 96);
@@ -95,6 +98,10 @@ __global__ void __launch_bounds__(320, 1)
   }
   for (int j = tid; j < 256; j += blockDim.x)
     vadd[j] = (j < p.L && p.key_valid[j] != 0) ? 0.f : -INFINITY;
+  for (int j = tid; j < C::OUT_BYTES / 16; j += blockDim.x)
+    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(sZero + 16u * uint32_t(j)), "r"(0u)
+                 : "memory");
+  fence_proxy_async_smem();  // the zero box is read by TMA stores
   if (warp == 8) {
     tmem_alloc(smem_u32(tmem_slot), 512u);
     tmem_relinquish();
@@ -193,19 +200,26 @@ __global__ void __launch_bounds__(320, 1)
       }
 #pragma unroll 1
       for (int c = 0; c < nc; ++c) {
-        uint32_t v[32];
-        if ((vmask >> c) & 1u) {
-          tmem_ld32(tl + uint32_t(c * 32), v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv);
-          if (c == last_valid) {  // the accumulator is free for the next unit
-            tc_fence_before();
-            mbar_arrive(BAR(6 + w));
+        if (!((vmask >> c) & 1u)) {
+          // an all-padding chunk: stored from the zero box, no staging
+          if (c * 32 < p.L4 && r == 0) {
+            tma_store_3d(&tmP, sZero, c * 32, row0, h);
+            bulk_commit();
           }
-        } else {
+          if (p.L4 < p.L && row0 + r < p.N) {
+            for (int j = max(c * 32, p.L4); j < min(c * 32 + 32, p.L); ++j)
+              p.P[h * p.p_sh + int64_t(row0 + r) * p.p_sn + j] = 0.f;
+          }
+          continue;
+        }
+        uint32_t v[32];
+        tmem_ld32(tl + uint32_t(c * 32), v);
+        tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv);
+        if (c == last_valid) {  // the accumulator is free for the next unit
+          tc_fence_before();
+          mbar_arrive(BAR(6 + w));
         }
         const uint32_t buf = sOut + uint32_t((w * C::NOUT + (nstore % C::NOUT)) * C::OUT_BYTES);
         if (nstore >= C::NOUT) {
@@ -264,10 +278,10 @@ __global__ void __launch_bounds__(320, 1)
         khead[st] = h;
         issued = i + 1;
       }
-      if (*abort_flag) {
-        for (int i = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); i < issued; ++i)
-          wait_drain(BAR(0 + i % C::NSTAGE), uint32_t((i / C::NSTAGE) & 1), kXDrainNs);
-      }
+      // every copy has landed before the CTA leaves (already true unless a
+      // role aborted before consuming it)
+      for (int i = (issued > C::NSTAGE ? issued - C::NSTAGE : 0); i < issued; ++i)
+        wait_drain(BAR(0 + i % C::NSTAGE), uint32_t((i / C::NSTAGE) & 1), kXDrainNs);
     }
   } else {
     // ============================================= MMA issuer
@@ -293,10 +307,9 @@ __global__ void __launch_bounds__(320, 1)
         tc_commit(BAR(4 + buf));
         tc_commit(BAR(2 + st));
       }
-      if (!ok) {
-        tc_commit(BAR(8));
-        wait_drain(BAR(8), 0u, kXDrainNs);
-      }
+      // every MMA has completed before TMEM is freed, whoever aborted
+      tc_commit(BAR(8));
+      wait_drain(BAR(8), 0u, kXDrainNs);
     }
   }
 
