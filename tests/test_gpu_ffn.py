@@ -59,9 +59,11 @@ def _check_close(out, ref, what):
     assert rf <= ATTN_REL_FRO and mx <= ATTN_MAX_ABS, f"{what}: relFro={rf:.3e} maxabs={mx:.3e}"
 
 
-@pytest.mark.parametrize("M,K,N", [(300, 200, 520),     # ragged rows, k-block and column tails
-                                   (128, 64, 256),      # exactly one tile
-                                   (2560, 512, 2048),   # 160 tiles: CTAs loop, both accumulators cycle
+@pytest.mark.parametrize("M,K,N", [(300, 200, 520),     # CTA pairs: ragged rows, k-block and column tails
+                                   (128, 64, 256),      # single CTA, exactly one tile
+                                   (255, 64, 264),      # single CTA, largest M below the pair tiles
+                                   (256, 8, 8),         # CTA pair, one tile, W half of the pair empty
+                                   (2560, 512, 2048),   # CTA pairs: 80 tiles, pairs loop, accumulators cycle
                                    (1, 8, 8)])          # smallest legal shape
 @pytest.mark.parametrize("bias", [True, False])
 def test_projection_plain(M, K, N, bias):
@@ -82,10 +84,12 @@ def test_projection_gelu(M, K, N):
     _check_close(f64(out), oracle.linear_act(a, w, b, act=1), "gelu projection")
 
 
-def test_projection_batched_scattered_rows():
+@pytest.mark.parametrize("M,M_out", [(77, 150),     # single-CTA tiles (M < 256)
+                                     (300, 700)])   # CTA-pair tiles with a ragged second row tile
+def test_projection_batched_scattered_rows(M, M_out):
     """[B, M, K] input, rows scattered by a shared index into [B, M_out, N];
     rows no index points at keep their bytes."""
-    B, M, K, N, M_out = 2, 77, 136, 264, 150
+    B, K, N = 2, 136, 264
     a, w, b = _linear_inputs(M, K, N, 11, B=B)
     idx = torch.randperm(M_out, generator=_gen(12))[:M].to(torch.int32)  # unique, unsorted
     init = torch.randn(B, M_out, N, generator=_gen(13)).to(torch.bfloat16)
