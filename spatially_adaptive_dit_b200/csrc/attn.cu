@@ -9,18 +9,25 @@
 //
 //   o_r = sum_j softmax_j(scale q_{idx[r]} . k_j + pad_j + bias_{idx[r],j}) v_j
 //
-// Design (one CTA per SM, 320 threads = 10 warps):
+// Design (one CTA per SM, 384 threads = 3 warpgroups):
 //   * 2 query tiles of 128 rows (256 rows per CTA).  The softmax warpgroup of
 //     tile t (warps 4t..4t+3) gathers its rows q[idx[r]] with 16-byte loads
 //     straight into the swizzled K-major shared-memory layout the tensor core
 //     reads (the indexed gather replaces a copy of Q_S).
-//   * warp 8 streams K and V tiles (128 keys) through an NS-stage TMA ring.
-//   * warp 9 issues tcgen05.mma: S_t = Q_t K_j^T into TMEM (fp32, 128 cols per
-//     tile) and O_t += P_t V_j with P_t read back from TMEM (the bf16 softmax
-//     probabilities overwrite S_t in place), so P never touches shared memory.
+//   * the third warpgroup: warp 8 streams K and V tiles (128 keys) through an
+//     NS-stage TMA ring, warp 9 issues tcgen05.mma, warps 10-11 only lend
+//     their registers (setmaxnreg: 208 per softmax thread, 88 per control
+//     thread).
+//   * MMAs: S_t = Q_t K_j^T into TMEM (fp32, 128 columns per tile) and
+//     O_t += P_t V_j with P_t read back from TMEM (the bf16 probabilities
+//     overwrite S_t in place), so P never touches shared memory; issue order
+//     per key tile PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so one tile's
+//     softmax overlaps the other tile's MMAs.  Descriptors are built once.
 //   * softmax: thread = query row = TMEM lane.  Online softmax in base 2 with
 //     a lazy rescale (the running max only moves when it grows by more than
-//     2^8, which is exact after the final division by the row sum).
+//     2^8, which is exact after the final division by the row sum); packed
+//     f32x2 FMAs and adds, three-input max; a quarter of the exponentials on
+//     the FMA pipe (degree-3 polynomial), the rest on the MUFU unit.
 // Every mbarrier wait is bounded; an expired wait raises the CTA's abort
 // flag, drains in-flight TMA loads and MMAs, frees TMEM and returns.
 #include <cmath>

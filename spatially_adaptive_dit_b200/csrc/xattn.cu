@@ -4,14 +4,17 @@
 // step 3).  Text padding is a kept semantic mask (방법론 1 보존): padding keys
 // receive exactly 0.
 //
-// One CTA = 128 image rows of one head, 128 threads (thread = row = TMEM
-// lane).  TMA brings the Q tile and the whole text-key block (L <= 256) into
-// swizzled shared memory; one elected thread issues tcgen05.mma for
-// S = Q K^T (M=128, N=L rounded up to 32) into TMEM; the softmax runs in
-// three TMEM passes (max; exp + sum with the exponentials written back to
-// TMEM; scale) and the probabilities leave through a double-buffered,
-// 128B-swizzled shared-memory stage and TMA tensor stores, so the 4-byte
-// P writes reach HBM as full lines.
+// Persistent: one 320-thread CTA per SM over (head, 128-row tile) units.  TMA
+// brings the Q tile and the whole text-key block (L <= 256, reloaded only on a
+// head change) into swizzled shared memory; one elected thread issues
+// tcgen05.mma for S = Q K^T (M=128, N=L rounded up to 32) into one of two
+// 256-column TMEM accumulators; two softmax warpgroups (thread = row = TMEM
+// lane) take alternate units and run three TMEM passes (max; exp + sum with
+// the exponentials written back to TMEM; scale).  The probabilities leave
+// through 4-deep 128B-swizzled shared-memory staging per warpgroup and TMA
+// tensor stores, so the 4-byte P writes reach HBM as full lines; text chunks
+// that are all padding skip TMEM and the exponential unit and are stored from
+// one shared all-zero box.
 #include <cmath>
 
 #include "common.cuh"
