@@ -295,6 +295,11 @@ def run_ours(args):
         }
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+            gms = {n: e["ms_mean"] for n, e in kern.items()}
+            gms.update({"ffn_block": ext["ffn_block_ms"], "mask_is_row_constant": ext["mask_stress"]["ms"],
+                        "qkv_projection_gathered": ext["qkv_projection_gathered"]["ms"],
+                        "stepcache_sw_cfg": ext["stepcache_sw_cfg"]["ms"]})
+            line["oracle_rows"] = oracle_rows(gms)
         print(json.dumps(line), flush=True)
     if ws > 1:
         torch.distributed.barrier()
@@ -359,6 +364,12 @@ def measure_extensions(tr, stream, dev, unfused_pcsp_ms, reps=5):
     sc_bytes = 5 * tr.eps_c.numel() * 4 + 4 * w.N
     out["stepcache_sw_cfg"] = {"ms": round(sc_ms, 4), "gbs": round(sc_bytes / (sc_ms * 1e-3) / 1e9, 1),
                                "note": f"F={tr.eps_c.shape[1]}: {sc_bytes / 1e6:.1f} MB, launch-bound"}
+    del x, y, xs, h, qkv, w1, w2
+    mask = torch.zeros(1, 1, wl.STRESS.N, wl.STRESS.N, dtype=torch.bfloat16, device=dev)
+    out["mask_stress"] = {"ms": round(best_ms(lambda: sd.safedit_mask_is_row_constant(mask, tr.verdict, None,
+                                                                                      stream)), 4),
+                          "note": f"[1,1,{wl.STRESS.N},{wl.STRESS.N}] bf16 all-zero mask (removable: read fully)"}
+    del mask
     out["workload"] = (f"B={B}, |S|={k} focus rows per batch, D={D}, F={F}; "
                        "synthetic weights N(0,1)/sqrt(fan_in)")
     if sd.safedit_get_device_status(stream) != 0:
@@ -494,6 +505,73 @@ def run_e2e(tr, stream, args):
     torch.cuda.synchronize()
     ms = (time.perf_counter() - t0) * 1e3 / n
     return {"ms": ms, "h2d": counts["h2d"] // n, "d2h": counts["d2h"] // n}
+
+
+def oracle_rows(gpu_ms):
+    """Every row of the path and of its extensions run by the fp64 oracle, as
+    it stands, on the host cores, on a bounded sample of the bench workload;
+    the per-call time is extrapolated linearly to the full call (the sample
+    and the factor are stated per row) and set beside the GPU's per-call time
+    of this run (`gpu_ms`, ms per call by CUDA events)."""
+    import numpy as np
+    import oracle
+    w = W
+    out = {}
+
+    def row(name, fn, factor, sample):
+        t0 = time.perf_counter()
+        fn()
+        dt = (time.perf_counter() - t0) * 1e3
+        est = dt * factor
+        g = gpu_ms.get(name)
+        out[name] = {"oracle_ms": round(est, 2), "gpu_ms": None if g is None else round(g, 4),
+                     "oracle_over_gpu": None if not g else round(est / g, 1), "sample": sample,
+                     "sample_ms": round(dt, 1)}
+
+    q_img, k_txt, valid, content = wl.text(w)
+    hs = 2
+    P = oracle.cross_attn_probs(q_img[0, :1, :64], k_txt[0, :1], valid[0])  # warm the library
+    row("cross_attn_probs", lambda: oracle.cross_attn_probs(q_img[0, :hs], k_txt[0, :hs], valid[0]),
+        w.H / hs, f"{hs} of {w.H} heads, all {w.N} rows (x{w.H // hs})")
+    P = oracle.cross_attn_probs(q_img[0, :hs], k_txt[0, :hs], valid[0])
+    row("partition_accumulate", lambda: oracle.partition_accumulate(P, content), w.H / hs,
+        f"{hs} of {w.H} heads (x{w.H // hs})")
+    score = wl.blob_scores(wl.Workload("2560 blobs", 2, B=2, H=24, N=w.N, d=96, L=256, n_valid=128,
+                                       rho=w.rho, grid=w.grid)).numpy()
+    row("partition_finalize", lambda: oracle.partition_select(score, w.k), 1.0,
+        f"the full split of N={w.N} (all-pairs rank count)")
+    nr = 256
+    m = wl.mask(wl.STRESS, "zero", dtype=torch.bfloat16, rows=list(range(nr)))[0, 0]
+    row("mask_is_row_constant", lambda: oracle.mask_row_constant(m), wl.STRESS.N / nr,
+        f"{nr} of {wl.STRESS.N} rows of the [1,1,{wl.STRESS.N},{wl.STRESS.N}] all-zero mask "
+        f"(x{wl.STRESS.N // nr})")
+    q, k, v = (t[0, 0].double().numpy() for t in wl.qkv(w))
+    ra = 128
+    row("attn_dense_anchor", lambda: oracle.attn_subset(q, k, v, np.arange(ra, dtype=np.int32)),
+        w.N * w.B * w.H / ra, f"{ra} query rows of one (b,h) over all {w.N} keys (x{w.N * w.B * w.H // ra})")
+    row("attn_subset_srsu", lambda: oracle.attn_subset(q, k, v, np.arange(ra, dtype=np.int32)),
+        w.k * w.B * w.H / ra, f"{ra} query rows of one (b,h) over all {w.N} keys (x{w.k * w.B * w.H // ra})")
+    idx = np.sort(np.random.default_rng(5).choice(w.N, w.k, replace=False)).astype(np.int32)
+    ks = wl.fresh_sensitive_kv(w, w.k, step=1)[0][0, 0].view(torch.int16).numpy()
+    kst = wl.qkv(w)[1][0, 0].view(torch.int16).numpy()
+    row("scatter_state", lambda: oracle.scatter_rows(ks, kst, idx), 2 * w.B * w.H,
+        f"one (b,h) slice of K (x{2 * w.B * w.H}: K and V of every slice)")
+    ec, eu = wl.cfg_preds(w)
+    sv = torch.rand(w.N).numpy()
+    row("sw_cfg", lambda: oracle.sw_cfg(ec, eu, sv, w.gamma_ctx, w.gamma_sens), 1.0, f"full [{w.N}, {w.F}]")
+    pc, pu = wl.cfg_preds(w, step=1)
+    row("stepcache_sw_cfg", lambda: oracle.stepcache_sw_cfg(pc, ec, pu, eu, sv, 0.5, w.gamma_ctx, w.gamma_sens),
+        1.0, f"full [{w.N}, {w.F}]")
+    D, F = w.D_model, w.D_ff
+    w1, b1, w2, b2 = wl.ffn_weights(w)
+    x = wl.ffn_states(w)[0][0, :8]
+    rf = 8
+    row("ffn_block", lambda: oracle.ffn_cached(x, None, w1, b1, w2, b2, np.zeros((rf, D)), act=1),
+        w.B * w.k / rf, f"{rf} focus rows (x{w.B * w.k // rf})")
+    wq, bq = wl.qkv_proj_weights(w)
+    row("qkv_projection_gathered", lambda: oracle.linear_act(x, wq, bq, act=0), w.B * w.k / rf,
+        f"{rf} focus rows (x{w.B * w.k // rf})")
+    return {"cores": oracle.num_threads(), "kind": "oracle", "rows": out}
 
 
 def cpu_baseline(seconds=12.0, rows=None):
