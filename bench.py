@@ -410,6 +410,19 @@ def _ncu_traffic():
         return None
 
 
+def _packed(tensors, device=None, pin=False):
+    """One byte block holding tensors shaped like `tensors` back to back
+    (256-byte aligned), and those views of it."""
+    sizes = [t.numel() * t.element_size() for t in tensors]
+    offs, o = [], 0
+    for sz in sizes:
+        offs.append(o)
+        o += (sz + 255) // 256 * 256
+    blk = torch.empty(o, dtype=torch.uint8, device=device, pin_memory=pin)
+    views = [blk[off:off + sz].view(t.dtype).view(t.shape) for t, off, sz in zip(tensors, offs, sizes)]
+    return blk, views
+
+
 def run_e2e(tr, stream, args):
     """Same trajectory through the C ABI with host buffers.  Every denoising
     step's inputs are copied from pinned host memory and its guided
@@ -418,82 +431,98 @@ def run_e2e(tr, stream, args):
     fresh S rows -- Q_S, K_S, V_S compact [B,H,k,d] (the projections of an
     SRSU step run on the S rows alone) -- plus eps_c, eps_u every step.  An
     SRSU step is then: scatter K_S, V_S into the cached state, attention of the
-    compact Q_S over all N keys, scatter O_S into O_state.  A copy stream runs
-    ahead of the compute stream: three input buffer sets, and two K/V state
-    sets that alternate between anchors, so that an anchor's full K/V upload
-    never waits for the step before it; events order every buffer reuse."""
+    compact Q_S over all N keys, scatter O_S into O_state.  Each step's inputs
+    sit back to back in one pinned block and cross the link as one copy (large
+    copies reach the link's rate, 70 MB ones do not).  A copy stream runs
+    ahead of the compute stream: three SRSU input blocks, and two anchor blocks
+    (Q, K, V, predictions) whose K and V then serve as the cached state until
+    the next anchor, so an anchor's upload never waits for the step before it;
+    events order every buffer reuse."""
     w = tr.w
     NSET = 3
-    names = ("q", "q_s", "k_s", "v_s", "q_img", "k_txt", "eps_c", "eps_u")
     q_s = tr.q[:, :, : tr.k].contiguous()
     o_s = torch.empty_like(q_s)
-    dev_t = {"q_s": q_s}
-    host = {}
-    for n in names + ("k_full", "v_full"):
-        t = dev_t.get(n, getattr(tr, n, None))
-        host[n] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-        host[n].copy_(t)
-    sets = [{n: dev_t.get(n, getattr(tr, n, None)) for n in names}] + \
-        [{n: torch.empty_like(host[n], device=tr.dev) for n in names} for _ in range(NSET - 1)]
-    states = [(tr.k_state, tr.v_state), (torch.empty_like(tr.k_state), torch.empty_like(tr.v_state))]
+    srsu_src = [q_s, tr.k_s, tr.v_s, tr.eps_c, tr.eps_u]
+    anchor_src = [tr.q, tr.k_full, tr.v_full, tr.eps_c, tr.eps_u]
+    text_src = [tr.q_img, tr.k_txt]
+    h_srsu, hv = _packed(srsu_src, pin=True)
+    for v, t in zip(hv, srsu_src):
+        v.copy_(t)
+    h_anchor, hv = _packed(anchor_src, pin=True)
+    for v, t in zip(hv, anchor_src):
+        v.copy_(t)
+    h_text, hv = _packed(text_src, pin=True)
+    for v, t in zip(hv, text_src):
+        v.copy_(t)
+    sets = [_packed(srsu_src, device=tr.dev) for _ in range(NSET)]      # (block, [q_s, k_s, v_s, c, u])
+    states = [_packed(anchor_src, device=tr.dev) for _ in range(2)]    # (block, [q, k, v, c, u])
+    d_text = _packed(text_src, device=tr.dev)
     out_h = [torch.empty(tr.cfg_out.shape, dtype=tr.cfg_out.dtype, pin_memory=True) for _ in range(NSET)]
     copy_stream = torch.cuda.Stream(device=tr.dev)
     sd = tr.sd
     counts = {"h2d": 0, "d2h": 0}
-    freed = [None] * NSET          # per input set: event after the last step that used it
-    state_freed = [None, None]     # per state set: event after the last step that read it
-    cur_state = [1]                # the state set in use (flips at every anchor)
+    freed = [None] * NSET          # per SRSU block: event after the last step that used it
+    state_freed = [None, None]     # per anchor block: event after the last step that read it
+    text_freed = [None]
+    cur_state = [1]                # the anchor block in use (flips at every anchor)
 
     def trajectory(count):
         with torch.cuda.stream(stream):
             tr.score.zero_()
         for t in range(w.steps):
             anchor = (t % w.period == 0)
-            cur = sets[t % NSET]
-            need = ["eps_c", "eps_u"] + (["q_img", "k_txt"] if t < w.warmup else []) + \
-                (["q"] if anchor else ["q_s", "k_s", "v_s"])
             ready = torch.cuda.Event()
             with torch.cuda.stream(copy_stream):
-                if freed[t % NSET] is not None:
-                    copy_stream.wait_event(freed[t % NSET])  # step t-NSET is done with this set
-                for n in need:
-                    cur[n].copy_(host[n], non_blocking=True)
+                if t < w.warmup:
+                    if text_freed[0] is not None:
+                        copy_stream.wait_event(text_freed[0])
+                    d_text[0].copy_(h_text, non_blocking=True)
                     if count:
-                        counts["h2d"] += host[n].numel() * host[n].element_size()
+                        counts["h2d"] += h_text.numel()
                 if anchor:
                     cur_state[0] ^= 1
                     if state_freed[cur_state[0]] is not None:
                         copy_stream.wait_event(state_freed[cur_state[0]])  # the previous anchor period
-                    for n, dst in zip(("k_full", "v_full"), states[cur_state[0]]):
-                        dst.copy_(host[n], non_blocking=True)
-                        if count:
-                            counts["h2d"] += host[n].numel() * host[n].element_size()
+                    blk, src = states[cur_state[0]][0], h_anchor
+                else:
+                    if freed[t % NSET] is not None:
+                        copy_stream.wait_event(freed[t % NSET])  # step t-NSET is done with this block
+                    blk, src = sets[t % NSET][0], h_srsu
+                blk.copy_(src, non_blocking=True)
+                if count:
+                    counts["h2d"] += src.numel()
                 ready.record(copy_stream)
-            k_st, v_st = states[cur_state[0]]
+            aq, k_st, v_st, a_c, a_u = states[cur_state[0]][1]
             stream.wait_event(ready)
             with torch.cuda.stream(stream):
                 if t < w.warmup:
-                    sd.safedit_cross_attn_probs(cur["q_img"], cur["k_txt"], tr.valid, 0, 0.0, tr.P, stream)
+                    q_img, k_txt = d_text[1]
+                    sd.safedit_cross_attn_probs(q_img, k_txt, tr.valid, 0, 0.0, tr.P, stream)
                     sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream)
+                    ev = torch.cuda.Event()
+                    ev.record(stream)
+                    text_freed[0] = ev
                 if t == w.warmup - 1:
                     sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s, stream)
                 if t == 0:
                     sd.safedit_mask_is_row_constant(tr.mask, tr.verdict, None, stream)
                 if anchor:
-                    sd.safedit_attn_subset(cur["q"], k_st, v_st, None, 0, None, None, 0.0,
-                                           tr.o_state, 0, stream)
+                    eps_c, eps_u = a_c, a_u
+                    sd.safedit_attn_subset(aq, k_st, v_st, None, 0, None, None, 0.0, tr.o_state, 0, stream)
                 else:
-                    sd.safedit_scatter_state([cur["k_s"], cur["v_s"]], [k_st, v_st], tr.idx_s, tr.k, stream)
-                    sd.safedit_attn_subset(cur["q_s"], k_st, v_st, None, 0, None, None, 0.0, o_s, 0, stream)
+                    qs, ks, vs, eps_c, eps_u = sets[t % NSET][1]
+                    sd.safedit_scatter_state([ks, vs], [k_st, v_st], tr.idx_s, tr.k, stream)
+                    sd.safedit_attn_subset(qs, k_st, v_st, None, 0, None, None, 0.0, o_s, 0, stream)
                     sd.safedit_scatter_state([o_s], [tr.o_state], tr.idx_s, tr.k, stream)
                 g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx
-                sd.safedit_sw_cfg(cur["eps_c"], cur["eps_u"], tr.s, w.gamma_ctx, g_sens, tr.cfg_out, stream)
+                sd.safedit_sw_cfg(eps_c, eps_u, tr.s, w.gamma_ctx, g_sens, tr.cfg_out, stream)
                 out_h[t % NSET].copy_(tr.cfg_out, non_blocking=True)
                 if count:
                     counts["d2h"] += out_h[t % NSET].numel() * out_h[t % NSET].element_size()
                 ev = torch.cuda.Event()
                 ev.record(stream)
-                freed[t % NSET] = ev
+                if not anchor:
+                    freed[t % NSET] = ev
                 state_freed[cur_state[0]] = ev
 
     trajectory(False)
