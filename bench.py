@@ -143,7 +143,8 @@ class Trajectory:
         self.flop_dense = 4.0 * N * N * d * B * H
         self.bytes = {
             "cross_attn_probs": H * N * L * 4 + H * N * d * 2 + H * L * d * 2,
-            "partition_accumulate": H * N * L * 4 + N * 16 + L,
+            # the 16-byte groups of P that hold a content column (the kernel reads no others)
+            "partition_accumulate": H * N * 16 * int(self.content.view(-1, 4).any(dim=1).sum()) + N * 16 + L,
             "scatter_state": 2 * (2 * B * H * k * d * 2) + 4 * k,
             "sw_cfg": 3 * N * w.F * 4 + 4 * N,
         }

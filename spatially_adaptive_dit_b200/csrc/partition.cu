@@ -1,7 +1,8 @@
 // partition.cu -- PCSP (SAFE-DiT summary, 방법론 2; AccelAes summary B.1):
 //   * partition_accumulate: score[i] += sum_h sum_{content j} P[h,i,j], one
-//     warp per image token, 128-bit streaming loads of P, fp64 accumulation
-//     and a warp-shuffle reduction;
+//     warp per image token, 128-bit streaming loads of the 16-byte groups of
+//     P that hold a content column (padding is never read), fp64
+//     accumulation and a warp-shuffle reduction;
 //   * partition_finalize: the top-k split (ties to the lower index) by an
 //     8-pass radix select on order-preserving 64-bit keys, a stable
 //     block-scan compaction into ascending S / C index lists, and the
@@ -22,6 +23,7 @@ struct AccParams {
 };
 
 constexpr int kAccWarps = 8;
+constexpr int kAccHeads = 4;  // heads whose loads a lane keeps in flight at once (8 measured slower)
 
 // Vector path: L % 4 == 0, strides % 4 == 0, 16-byte aligned base,
 // L <= 128 * NCH (NCH passes of 128 columns per warp).
@@ -42,20 +44,22 @@ __global__ void __launch_bounds__(kAccWarps * 32) accumulate_vec_kernel(AccParam
     double acc = 0.0;
     const float* row0 = p.P + i * p.sN;
     int64_t h = 0;
-    for (; h + 4 <= p.H; h += 4) {
-      float4 v[4][NCH];
+    for (; h + kAccHeads <= p.H; h += kAccHeads) {
+      float4 v[kAccHeads][NCH];
 #pragma unroll
-      for (int hh = 0; hh < 4; ++hh)
+      for (int hh = 0; hh < kAccHeads; ++hh)
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
-          const int64_t j = int64_t(c) * 128 + lane * 4;
-          if (j < p.L)
-            v[hh][c] = __ldcs(reinterpret_cast<const float4*>(row0 + (h + hh) * p.sH + j));
+          // only 16-byte groups holding a content column are read (text
+          // padding and the non-content tokens never leave HBM)
+          if ((cmask >> (c * 4)) & 0xFu)
+            v[hh][c] = __ldcs(reinterpret_cast<const float4*>(row0 + (h + hh) * p.sH +
+                                                              int64_t(c) * 128 + lane * 4));
           else
             v[hh][c] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-      for (int hh = 0; hh < 4; ++hh)
+      for (int hh = 0; hh < kAccHeads; ++hh)
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
           const uint32_t m = cmask >> (c * 4);
@@ -69,7 +73,7 @@ __global__ void __launch_bounds__(kAccWarps * 32) accumulate_vec_kernel(AccParam
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
         const int64_t j = int64_t(c) * 128 + lane * 4;
-        if (j < p.L) {
+        if ((cmask >> (c * 4)) & 0xFu) {
           const float4 v = __ldcs(reinterpret_cast<const float4*>(row0 + h * p.sH + j));
           const uint32_t m = cmask >> (c * 4);
           if (m & 1u) acc += static_cast<double>(v.x);
