@@ -661,6 +661,72 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_stress(args):
+    """The mask-path stress workload (B=1, H=32, N=16384, d=128, |S|=4915 from
+    the clustered blob scores): SRSU attention with the mask elided (no mask
+    input), with a kept text-padding key mask (trailing 1/8 of the keys -inf),
+    and with a kept non-uniform bf16 bias [1,1,N,N]; the row-constant check on
+    an all-zero mask (elided: read fully) and on the padding mask (kept: the
+    check stops at the first kept row).  Best of `--reps` CUDA-event timings;
+    one JSON line per case (not a bench line)."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    from spatially_adaptive_dit_b200 import safedit as sd
+    w = wl.STRESS
+    _, bf16_burst, _, src = _peaks()
+    stream = torch.cuda.Stream(device=dev)
+    q, k, v = wl.qkv(w, device=dev)
+    o = torch.zeros_like(q)
+    score = wl.blob_scores(w, device=dev).contiguous()
+    idx = torch.empty(w.k, dtype=torch.int32, device=dev)
+    sd.safedit_partition_finalize(score, w.N, w.k, idx, None, None, stream)
+    pad = torch.zeros(1, w.N, device=dev)
+    pad[:, w.N - w.N // 8:] = float("-inf")
+    bias = wl.mask(w, "bias", device=dev)            # [1,1,N,N] bf16
+    zero = wl.mask(w, "zero", device=dev)
+    padmask = wl.mask(w, "textpad", device=dev)
+    verdict = torch.zeros(1, dtype=torch.int32, device=dev)
+    flop = 4.0 * w.k * w.N * w.d * w.B * w.H
+
+    def best(fn):
+        times = []
+        with torch.cuda.stream(stream):
+            for _ in range(args.reps + 1):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                times.append((a, b))
+        stream.synchronize()
+        return min(a.elapsed_time(b) for a, b in times[1:])
+
+    cases = {
+        "srsu_mask_elided": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, None, None, 0.0, o, 1, stream),
+        "srsu_kept_padding": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, pad, None, 0.0, o, 1, stream),
+        "srsu_kept_bias": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, None, bias, 0.0, o, 1, stream),
+    }
+    base = None
+    for name, fn in cases.items():
+        ms = best(fn)
+        base = base or ms
+        tf = flop / (ms * 1e-3) / 1e12
+        print(json.dumps({"stress": name, "ms": round(ms, 4), "tflops": round(tf, 1),
+                          "frac_of_burst": round(tf / bf16_burst, 3), "slowdown": round(ms / base, 3),
+                          "peak": f"bf16_tflops {bf16_burst} ({src})"}), flush=True)
+    hbm = _peaks()[0]
+    for name, m in (("mask_check_elided_zero", zero), ("mask_check_kept_padding", padmask)):
+        ms = best(lambda: sd.safedit_mask_is_row_constant(m, verdict, None, stream))
+        gbs = m.numel() * 2 / (ms * 1e-3) / 1e9
+        print(json.dumps({"stress": name, "ms": round(ms, 4), "verdict": int(verdict.item()),
+                          "gbs_if_read_fully": round(gbs, 1), "frac_hbm_if_read_fully": round(gbs / hbm, 3)}),
+              flush=True)
+    status = sd.safedit_get_device_status(stream)
+    if status != 0:
+        print(json.dumps({"stress": "status", "status": status}))
+        sys.exit(3)
+
+
 def run_sweep(args):
     """The 3072^2 sensitive-fraction sweep (B=2, H=24, N=36864, d=96): SRSU
     attention of |S| = rho N gathered rows over all N keys, scattered into the
@@ -812,13 +878,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,
                     choices=["srsu", "anchor", "xattn", "accumulate", "pcsp", "finalize", "scatter", "cfg",
-                             "stepcache", "mask", "ffn1", "ffn2", "ffn", "qkv", "sweep"],
+                             "stepcache", "mask", "ffn1", "ffn2", "ffn", "qkv", "sweep", "stress"],
                     help="run one kernel of the path in isolation (profiling target)")
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--cfg-f", type=int, default=W.F, help="prediction width for --only cfg")
     args = ap.parse_args()
     if args.only == "sweep":
         run_sweep(args)
+        return
+    if args.only == "stress":
+        run_stress(args)
         return
     if args.only:
         run_only(args)

@@ -83,7 +83,10 @@ __global__ void __launch_bounds__(kMaskWarps * 32) mask_rows_kernel(MaskParams p
   const int es = p.dtype == SAFEDIT_F32 ? 4 : (p.dtype == SAFEDIT_BOOL ? 1 : 2);
   for (int64_t row = blockIdx.x * int64_t(kMaskWarps) + (threadIdx.x >> 5); row < nrows;
        row += nwarps) {
-    if (!p.row_flags && *reinterpret_cast<volatile int*>(p.verdict) == 0) return;
+    // warp-uniform exit once another row has been found kept
+    if (!p.row_flags &&
+        __any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(p.verdict) == 0))
+      return;
     const int64_t q = row % p.Nq;
     const int64_t bh = row / p.Nq;
     const int64_t h = bh % p.Hm, b = bh / p.Hm;
@@ -110,7 +113,9 @@ __global__ void __launch_bounds__(kMaskWarps * 32) mask_rows_kernel(MaskParams p
     ok = __all_sync(0xffffffffu, ok);
     if (lane == 0) {
       if (p.row_flags) p.row_flags[row] = ok ? 1 : 0;
-      if (!ok) *p.verdict = 0;
+      // one store clears the verdict: thousands of warps storing to the same
+      // word would serialise in L2
+      if (!ok && *reinterpret_cast<volatile int*>(p.verdict) != 0) *p.verdict = 0;
     }
   }
 }
