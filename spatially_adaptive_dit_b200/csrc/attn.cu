@@ -31,6 +31,7 @@
 // Every mbarrier wait is bounded; an expired wait raises the CTA's abort
 // flag, drains in-flight TMA loads and MMAs, frees TMEM and returns.
 #include <cmath>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -52,6 +53,10 @@ struct AttnCfg {
   static constexpr int SMEM_TILES = 2 + 2 * NS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES * TILE_BYTES + BAR_BYTES;
+  static constexpr int PAD_BYTES = 8 * 2 * 128 * 4;    // per warp: 2 key tiles of pad
+  static constexpr int BIAS_BYTES = 8 * 32 * 128;      // per warp: 32 rows x 64 bf16 keys
+  static_assert(SMEM_BYTES + PAD_BYTES <= 232448, "shared memory");
+  static_assert(SMEM_BYTES + BIAS_BYTES <= 232448, "shared memory");
   static_assert(D == 64 || D == 96 || D == 128, "head dim");
   static_assert(256 + 2 * D <= 512, "TMEM columns");
 };
@@ -61,6 +66,7 @@ struct AttnParams {
   int64_t q_sb, q_sh, q_sr;  // element strides
   const int* idx;            // nullable
   int n_rows, Nq, Nk, H;
+  float scale;               // softmax scale
   float scale_log2;          // scale * log2(e)
   const float* pad;          // nullable, [B, Nk]
   int64_t pad_sb;
@@ -98,12 +104,61 @@ __device__ __forceinline__ uint32_t swizzle_off(uint32_t off, uint32_t layout) {
   return layout == 2u ? (off ^ (((off >> 7) & 7u) << 4)) : (off ^ (((off >> 7) & 3u) << 4));
 }
 
-template <int D, bool PAD, bool BIAS>
+// Kept-bias element type (template parameter of the kernel).
+constexpr int kBiasNone = 0, kBiasBf16 = 1, kBiasF32 = 2;
+
+// Four pad values starting at key `k0` (a multiple of 4); zero past Nk.
+__device__ __forceinline__ float4 load_pad4(const float* row, int k0, int Nk) {
+  if (k0 + 4 <= Nk) return __ldg(reinterpret_cast<const float4*>(row + k0));
+  float v[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) v[e] = (k0 + e < Nk) ? __ldg(row + k0 + e) : 0.f;
+  return make_float4(v[0], v[1], v[2], v[3]);
+}
+
+// Asynchronous 16-byte global -> shared copy (no register staging); bytes
+// past `src_bytes` are zero-filled and not read.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// Stages the bf16 bias of this warp's 32 query rows, keys [k0, k0 + 64),
+// into the warp's 4 KB buffer with coalesced copies (each instruction moves
+// four 128-byte row segments).  Row rr's 16-byte chunk ch lands in slot
+// ch ^ (rr & 7) of the row's 128 bytes, so that the row-per-thread reads
+// back are free of bank conflicts.  qrow[i] is the query index of row
+// 4 i + lane / 8 (negative: no row); keys past Nk are zero-filled or skipped.
+__device__ __forceinline__ void stage_bias_bf16(uint32_t buf, const __nv_bfloat16* base, int64_t sq,
+                                                const int (&qrow)[8], int k0, int Nk, int lane) {
+  const int ch = lane & 7;
+  const int left = Nk - (k0 + ch * 8);
+  if (left > 0) {
+    const uint32_t bytes = left >= 8 ? 16u : uint32_t(left) * 2u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int rr = 4 * i + (lane >> 3);
+      if (qrow[i] >= 0)
+        cp_async16(buf + uint32_t(rr * 128 + ((ch ^ (rr & 7)) << 4)),
+                   base + int64_t(qrow[i]) * sq + k0 + ch * 8, bytes);
+    }
+  }
+  cp_async_commit();
+}
+
+template <int D, bool PAD, int BIAS>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_subset_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = AttnCfg<D>;
-  constexpr bool MASKED = PAD || BIAS;
+  constexpr bool MASKED = PAD || BIAS != kBiasNone;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -201,170 +256,247 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (my_q < 0 || my_q >= p.Nq) my_q = -1;
     }
     const float sl2 = p.scale_log2;
+    // Kept masks.  Their operands for the next key columns are fetched ahead,
+    // so that the load latency overlaps the current columns instead of
+    // sitting between S and P.  The pad (alone): one tile ahead, one 16-byte
+    // load per lane into this warp's double-buffered 512-byte slice in shared
+    // memory, read back as broadcasts.  A bf16 bias: one 64-key pass ahead,
+    // copied asynchronously and coalesced into this warp's 4 KB buffer, read
+    // back row per thread.  An f32 bias, and the pad beside a bf16 bias (no
+    // shared memory left for both buffers), are read in place.
+    constexpr bool PAD_SMEM = PAD && BIAS != kBiasBf16;
+    uint8_t* const mask_smem = smem + C::SMEM_TILES * C::TILE_BYTES + C::BAR_BYTES;
+    float* const pad_smem = PAD_SMEM ? reinterpret_cast<float*>(mask_smem) + warp * 256 : nullptr;
+    const uint32_t bias_buf = smem_u32(mask_smem) + uint32_t(warp * 4096);
+    const float* const pad_row = PAD ? p.pad + b * p.pad_sb : nullptr;
+    float4 pad_next = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (PAD_SMEM) pad_next = load_pad4(pad_row, 4 * lane, p.Nk);
+    const __nv_bfloat16* const bias_bh =
+        BIAS == kBiasBf16
+            ? static_cast<const __nv_bfloat16*>(p.bias) + b * p.bias_sb + h * p.bias_sh
+            : nullptr;
+    int qrow[8];  // query index of row 4 i + lane / 8 of this warp (bf16 bias staging)
+    if constexpr (BIAS == kBiasBf16) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qrow[i] = __shfl_sync(0xffffffffu, my_q, 4 * i + (lane >> 3));
+      stage_bias_bf16(bias_buf, bias_bh, p.bias_sq, qrow, 0, p.Nk, lane);
+    }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
+      const int key0 = j * C::BN;
+      if constexpr (PAD_SMEM) {
+        *reinterpret_cast<float4*>(pad_smem + (j & 1) * 128 + 4 * lane) = pad_next;
+        __syncwarp();
+        if (j + 1 < nk) pad_next = load_pad4(pad_row, key0 + C::BN + 4 * lane, p.Nk);
+      }
       if (!wait_warp(BAR(S_FULL + t), uint32_t(j & 1), ctl)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // x = raw scores (mask-free path) or log2-domain logits (kept masks)
-      float x[128];
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(tS + 0u, r0);
-        tmem_ld32(tS + 32u, r1);
-        tmem_ld32(tS + 64u, r2);
-        tmem_ld32(tS + 96u, r3);
-        tmem_wait_ld();
+      // The mask-free path takes the tile's 128 columns in one pass.  With
+      // kept masks the tile goes in two passes of 64 columns, each with its
+      // own online-softmax max, which keeps the mask operands of a pass in
+      // registers beside its scores; if the second pass raises the running
+      // max, the first pass's P (already in TMEM) is rescaled with it.
+      constexpr int NH = MASKED ? 2 : 1, HW = 128 / NH;
+      float alpha_p0 = 1.f;  // factor owed by the first pass's P
+      bool owe_p0 = false;
+      // one pass over columns [hf * HW, hf * HW + HW); hf is a compile-time
+      // constant, so every register array below is indexed statically
+      auto pass = [&](auto hf_tag) {
+        constexpr int hf = decltype(hf_tag)::value;
+        constexpr int c0 = hf * HW;  // first column of the pass
+        // x = raw scores (mask-free) or natural-unit logits
+        // scale * s + pad + bias (kept masks)
+        float x[HW];
+        {
+          uint32_t r[HW / 32][32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          x[e] = __uint_as_float(r0[e]);
-          x[32 + e] = __uint_as_float(r1[e]);
-          x[64 + e] = __uint_as_float(r2[e]);
-          x[96 + e] = __uint_as_float(r3[e]);
+          for (int q4 = 0; q4 < HW / 32; ++q4) tmem_ld32(tS + uint32_t(c0 + q4 * 32), r[q4]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q4 = 0; q4 < HW / 32; ++q4)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[q4 * 32 + e] = __uint_as_float(r[q4][e]);
         }
-      }
-      const int key0 = j * C::BN;
-      if (MASKED) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] *= sl2;
-      }
-      if (PAD) {
-        const float* pr = p.pad + b * p.pad_sb + key0;
-        const int lim = p.Nk - key0;
-#pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-          if (c + 4 <= lim) {
-            const float4 pv = __ldg(reinterpret_cast<const float4*>(pr + c));
-            x[c] = fmaf(pv.x, kLog2e, x[c]);
-            x[c + 1] = fmaf(pv.y, kLog2e, x[c + 1]);
-            x[c + 2] = fmaf(pv.z, kLog2e, x[c + 2]);
-            x[c + 3] = fmaf(pv.w, kLog2e, x[c + 3]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (c + e < lim) x[c + e] = fmaf(__ldg(pr + c + e), kLog2e, x[c + e]);
+        if constexpr (MASKED) {
+          const uint64_t sc2 = f2_pack(p.scale, p.scale);
+          const int lim = p.Nk - key0 - c0;
+          if constexpr (BIAS == kBiasBf16) {  // this pass's bias has landed
+            cp_async_wait_all();
+            __syncwarp();
           }
-        }
-      }
-      if (BIAS && my_q >= 0) {
-        const int lim = p.Nk - key0;
-        if (p.bias_f32) {
-          const float* br = static_cast<const float*>(p.bias) + b * p.bias_sb + h * p.bias_sh +
-                            int64_t(my_q) * p.bias_sq + key0;
 #pragma unroll
-          for (int c = 0; c < 128; c += 4) {
-            if (c + 4 <= lim) {
-              const float4 bv = __ldg(reinterpret_cast<const float4*>(br + c));
-              x[c] = fmaf(bv.x, kLog2e, x[c]);
-              x[c + 1] = fmaf(bv.y, kLog2e, x[c + 1]);
-              x[c + 2] = fmaf(bv.z, kLog2e, x[c + 2]);
-              x[c + 3] = fmaf(bv.w, kLog2e, x[c + 3]);
-            } else {
+          for (int c = 0; c < HW; c += 8) {
+            float add[8];
+            if constexpr (PAD_SMEM) {
+              const float* const ps = pad_smem + (j & 1) * 128 + c0;
+              const float4 a0 = *reinterpret_cast<const float4*>(ps + c);
+              const float4 a1 = *reinterpret_cast<const float4*>(ps + c + 4);
+              add[0] = a0.x; add[1] = a0.y; add[2] = a0.z; add[3] = a0.w;
+              add[4] = a1.x; add[5] = a1.y; add[6] = a1.z; add[7] = a1.w;
+            } else if constexpr (PAD) {
+              const float* const pr = pad_row + key0 + c0 + c;
+              if (c + 8 <= lim) {
+                const float4 a0 = __ldg(reinterpret_cast<const float4*>(pr));
+                const float4 a1 = __ldg(reinterpret_cast<const float4*>(pr + 4));
+                add[0] = a0.x; add[1] = a0.y; add[2] = a0.z; add[3] = a0.w;
+                add[4] = a1.x; add[5] = a1.y; add[6] = a1.z; add[7] = a1.w;
+              } else {
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (c + e < lim) x[c + e] = fmaf(__ldg(br + c + e), kLog2e, x[c + e]);
-            }
-          }
-        } else {
-          const __nv_bfloat16* br = static_cast<const __nv_bfloat16*>(p.bias) + b * p.bias_sb +
-                                    h * p.bias_sh + int64_t(my_q) * p.bias_sq + key0;
-#pragma unroll
-          for (int c = 0; c < 128; c += 8) {
-            if (c + 8 <= lim) {
-              const uint4 w = __ldg(reinterpret_cast<const uint4*>(br + c));
-              const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                x[c + 2 * e] = fmaf(__uint_as_float(ws[e] << 16), kLog2e, x[c + 2 * e]);
-                x[c + 2 * e + 1] =
-                    fmaf(__uint_as_float(ws[e] & 0xFFFF0000u), kLog2e, x[c + 2 * e + 1]);
+                for (int e = 0; e < 8; ++e) add[e] = (c + e < lim) ? __ldg(pr + e) : 0.f;
               }
             } else {
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                if (c + e < lim) x[c + e] = fmaf(__bfloat162float(br[c + e]), kLog2e, x[c + e]);
+              for (int e = 0; e < 8; ++e) add[e] = 0.f;
+            }
+            if constexpr (BIAS == kBiasBf16) {
+              uint32_t ws[4];
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(ws[0]), "=r"(ws[1]), "=r"(ws[2]), "=r"(ws[3])
+                           : "r"(bias_buf + uint32_t(lane * 128 + (((c / 8) ^ (lane & 7)) << 4))));
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                add[2 * e] += __uint_as_float(ws[e] << 16);
+                add[2 * e + 1] += __uint_as_float(ws[e] & 0xFFFF0000u);
+              }
+            } else if constexpr (BIAS == kBiasF32) {
+              if (my_q >= 0) {
+                const float* br = static_cast<const float*>(p.bias) + b * p.bias_sb +
+                                  h * p.bias_sh + int64_t(my_q) * p.bias_sq + key0 + c0 + c;
+                if (c + 8 <= lim) {
+                  const float4 b0 = __ldg(reinterpret_cast<const float4*>(br));
+                  const float4 b1 = __ldg(reinterpret_cast<const float4*>(br + 4));
+                  add[0] += b0.x; add[1] += b0.y; add[2] += b0.z; add[3] += b0.w;
+                  add[4] += b1.x; add[5] += b1.y; add[6] += b1.z; add[7] += b1.w;
+                } else {
+#pragma unroll
+                  for (int e = 0; e < 8; ++e)
+                    if (c + e < lim) add[e] += __ldg(br + e);
+                }
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              float y0, y1;
+              f2_unpack(f2_fma(f2_pack(x[c + e], x[c + e + 1]), sc2, f2_pack(add[e], add[e + 1])),
+                        y0, y1);
+              x[c + e] = y0;
+              x[c + e + 1] = y1;
             }
           }
+          if constexpr (BIAS == kBiasBf16) {
+            // every lane has read the buffer: stage the next pass into it
+            __syncwarp();
+            const int k_next = key0 + c0 + HW;
+            if (k_next < nk * C::BN)
+              stage_bias_bf16(bias_buf, bias_bh, p.bias_sq, qrow, k_next, p.Nk, lane);
+          }
         }
-      }
-      if (key0 + C::BN > p.Nk) {  // ragged last key tile
-        const int lim = p.Nk - key0;
+        if (key0 + C::BN > p.Nk) {  // ragged last key tile
+          const int lim = p.Nk - key0 - c0;
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= lim) x[c] = -INFINITY;
-      }
-      // row max of the tile (in log2 units)
-      float mt;
-      {
-        // four independent max chains (latency), three-input max (issue)
-        float m0 = fmaxf(x[0], x[1]), m1 = fmaxf(x[2], x[3]), m2 = fmaxf(x[4], x[5]),
-              m3 = fmaxf(x[6], x[7]);
-#pragma unroll
-        for (int c = 8; c < 128; c += 8) {
-          m0 = max3(m0, x[c], x[c + 1]);
-          m1 = max3(m1, x[c + 2], x[c + 3]);
-          m2 = max3(m2, x[c + 4], x[c + 5]);
-          m3 = max3(m3, x[c + 6], x[c + 7]);
+          for (int c = 0; c < HW; ++c)
+            if (c >= lim) x[c] = -INFINITY;
         }
-        mt = fmaxf(max3(m0, m1, m2), m3);
-        if (!MASKED) mt *= sl2;  // sl2 > 0: the max commutes with the scale
-      }
-      // lazy rescale: the running max moves only when it grows by > 2^8
-      bool need_o = false;
-      float alpha = 1.f;
-      if (mt > m_run + kRescaleThreshold) {
-        alpha = ex2_approx(m_run - mt);  // 0 when m_run = -inf
-        l_run *= alpha;
-        m_run = mt;
-        need_o = (j > 0);
-      }
-      if (__any_sync(0xffffffffu, need_o)) {
+        // row max of the pass (in log2 units)
+        float mt;
+        {
+          // four independent max chains (latency), three-input max (issue)
+          float m0 = fmaxf(x[0], x[1]), m1 = fmaxf(x[2], x[3]), m2 = fmaxf(x[4], x[5]),
+                m3 = fmaxf(x[6], x[7]);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+          for (int c = 8; c < HW; c += 8) {
+            m0 = max3(m0, x[c], x[c + 1]);
+            m1 = max3(m1, x[c + 2], x[c + 3]);
+            m2 = max3(m2, x[c + 4], x[c + 5]);
+            m3 = max3(m3, x[c + 6], x[c + 7]);
+          }
+          mt = fmaxf(max3(m0, m1, m2), m3);
+          // the max commutes with the positive factor into log2 units
+          mt *= MASKED ? kLog2e : sl2;
+        }
+        // lazy rescale: the running max moves only when it grows by > 2^8
+        bool need_o = false;
+        float alpha = 1.f;
+        if (mt > m_run + kRescaleThreshold) {
+          alpha = ex2_approx(m_run - mt);  // 0 when m_run = -inf
+          l_run *= alpha;
+          m_run = mt;
+          need_o = (j > 0);
+          if (hf == 1) {
+            owe_p0 = true;
+            alpha_p0 = alpha;
+          }
+        }
+        if (__any_sync(0xffffffffu, need_o)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + uint32_t(c * 32), r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(tO + uint32_t(c * 32), r);
+          }
+        }
+        if (hf == 1 && __any_sync(0xffffffffu, owe_p0)) {
+          // the first pass's 64 probabilities (32 packed columns)
+          tmem_wait_st();
           uint32_t r[32];
-          tmem_ld32(tO + uint32_t(c * 32), r);
+          tmem_ld32(tS, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(tO + uint32_t(c * 32), r);
+          for (int e = 0; e < 32; ++e)
+            r[e] = pack_bf16x2(__uint_as_float(r[e] << 16) * alpha_p0,
+                               __uint_as_float(r[e] & 0xFFFF0000u) * alpha_p0);
+          tmem_st32(tS, r);
         }
-      }
-      const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-      const float mul = MASKED ? 1.f : sl2;
-      const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(neg_m, neg_m);
-      // four independent partial sums: the row sum is not one serial chain
-      uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+        const float mul = MASKED ? kLog2e : sl2;
+        const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(neg_m, neg_m);
+        // four independent partial sums: the row sum is not one serial chain
+        uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f),
+                            f2_pack(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < HW / 32; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const uint64_t a2 = f2_fma(f2_pack(x[c * 32 + 2 * e], x[c * 32 + 2 * e + 1]), mul2, negm2);
-          float a0, a1, p0, p1;
-          f2_unpack(a2, a0, a1);
-          if (!MASKED && ((kExp2FmaMask >> e) & 1u)) {
-            exp2_pair_fma(a0, a1, p0, p1);
-          } else {
-            p0 = ex2_approx(a0);
-            p1 = ex2_approx(a1);
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t a2 =
+                f2_fma(f2_pack(x[c * 32 + 2 * e], x[c * 32 + 2 * e + 1]), mul2, negm2);
+            float a0, a1, p0, p1;
+            f2_unpack(a2, a0, a1);
+            if ((kExp2FmaMask >> e) & 1u) {
+              exp2_pair_fma(a0, a1, p0, p1);
+              if (MASKED) {  // exact zero weight below the normal range (masked keys)
+                p0 = a0 < -126.f ? 0.f : p0;
+                p1 = a1 < -126.f ? 0.f : p1;
+              }
+            } else {
+              p0 = ex2_approx(a0);
+              p1 = ex2_approx(a1);
+            }
+            sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
+            pk[e] = pack_bf16x2(p0, p1);
           }
-          sum2[e & 3] = f2_add(sum2[e & 3], f2_pack(p0, p1));
-          pk[e] = pack_bf16x2(p0, p1);
+          tmem_st16(tS + uint32_t((c0 / 32 + c) * 16), pk);
         }
-        tmem_st16(tS + uint32_t(c * 16), pk);
-      }
-      {
-        float s0, s1;
-        f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
-        l_run += s0 + s1;
-      }
+        {
+          float s0, s1;
+          f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), s0, s1);
+          l_run += s0 + s1;
+        }
+      };
+      pass(std::integral_constant<int, 0>{});
+      if constexpr (NH == 2) pass(std::integral_constant<int, 1>{});
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(P_FULL + t));
     }
+    if constexpr (BIAS == kBiasBf16) cp_async_wait_all();  // none in flight at exit
     // ---- epilogue: O / l -> bf16 rows
     if (ok && wait_warp(BAR(O_FULL), 0u, ctl)) {
       tc_fence_after();
@@ -508,26 +640,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-template <int D, bool PAD, bool BIAS>
+template <int D, bool PAD, int BIAS>
 static safedit_status launch_attn(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                   const AttnParams& p, int B, cudaStream_t stream) {
   using C = AttnCfg<D>;
   auto kern = attn_subset_kernel<D, PAD, BIAS>;
-  safedit_status st = set_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES);
+  constexpr int smem_bytes =
+      C::SMEM_BYTES + (BIAS == kBiasBf16 ? C::BIAS_BYTES : (PAD ? C::PAD_BYTES : 0));
+  safedit_status st = set_smem(reinterpret_cast<const void*>(kern), smem_bytes);
   if (st != SAFEDIT_OK) return st;
   dim3 grid((p.n_rows + 255) / 256, B * p.H);
-  kern<<<grid, kAttnThreads, C::SMEM_BYTES, stream>>>(tmK, tmV, p);
+  kern<<<grid, kAttnThreads, smem_bytes, stream>>>(tmK, tmV, p);
   return after_launch(1);
 }
 
 template <int D>
 static safedit_status dispatch_attn(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                     const AttnParams& p, int B, cudaStream_t s) {
-  const bool pad = p.pad != nullptr, bias = p.bias != nullptr;
-  if (pad && bias) return launch_attn<D, true, true>(tmK, tmV, p, B, s);
-  if (pad) return launch_attn<D, true, false>(tmK, tmV, p, B, s);
-  if (bias) return launch_attn<D, false, true>(tmK, tmV, p, B, s);
-  return launch_attn<D, false, false>(tmK, tmV, p, B, s);
+  const bool pad = p.pad != nullptr;
+  const int bias = p.bias == nullptr ? kBiasNone : (p.bias_f32 ? kBiasF32 : kBiasBf16);
+  if (pad) {
+    if (bias == kBiasBf16) return launch_attn<D, true, kBiasBf16>(tmK, tmV, p, B, s);
+    if (bias == kBiasF32) return launch_attn<D, true, kBiasF32>(tmK, tmV, p, B, s);
+    return launch_attn<D, true, kBiasNone>(tmK, tmV, p, B, s);
+  }
+  if (bias == kBiasBf16) return launch_attn<D, false, kBiasBf16>(tmK, tmV, p, B, s);
+  if (bias == kBiasF32) return launch_attn<D, false, kBiasF32>(tmK, tmV, p, B, s);
+  return launch_attn<D, false, kBiasNone>(tmK, tmV, p, B, s);
 }
 
 static safedit_status check_bhnd(const safedit_tensor* t) {
@@ -616,6 +755,7 @@ extern "C" safedit_status safedit_attn_subset(const safedit_tensor* q, const saf
   p.Nk = static_cast<int>(Nk);
   p.H = static_cast<int>(H);
   const float sc = (scale > 0.f) ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale = sc;
   p.scale_log2 = sc * kLog2e;
   p.out = static_cast<__nv_bfloat16*>(out->data);
   p.o_sb = out->strides[0];

@@ -127,6 +127,44 @@ def test_kept_masks_key_padding_and_bias():
     assert torch.equal(o1[0], o2[0])
 
 
+@pytest.mark.parametrize("D", [64, 96, 128])
+@pytest.mark.parametrize("kind", ["pad", "bias_f32", "bias_bf16", "pad+bias_f32", "pad+bias_bf16"])
+def test_kept_mask_variants_ragged_tail_and_max_jumps(D, kind):
+    """Every kept-mask kernel variant.  The last key tile is ragged, ending
+    inside the first and inside the second 64-column pass; the additive terms
+    raise the running max by far more than the lazy-rescale threshold, once
+    inside the first pass of a tile and once inside the second (the first
+    pass's probabilities, already in TMEM, are then rescaled); padded keys
+    hold garbage values that must get exactly zero weight."""
+    B, H, kr = 1, 2, 150
+    for N in (696, 600):  # last tile: 56 keys, 88 keys
+        q, k, v = _qkv(B, H, N, N, D, seed=1000 + N + D)
+        idx = _rand_idx(N, kr, seed=1001 + N)
+        pad = bias = None
+        if kind.startswith("pad"):
+            pad = torch.zeros(B, N)
+            pad[:, 5::7] = float("-inf")
+            pad[:, 128 + 10:128 + 20] += 9.0        # tile 1, first pass
+            pad[:, 256 + 70:256 + 90] += 18.0       # tile 2, second pass
+        if "bias" in kind:
+            g = _gen(1002 + N)
+            bias = torch.randn(B, H if kind.endswith("f32") else 1, N, N, generator=g) * 0.5
+            bias[..., ::2, 384 + 64:384 + 80] += 12.0   # tile 3, second pass, even query rows
+            bias[..., 1::2, 512 + 3:512 + 9] += 10.0    # ragged tile 4, first pass, odd rows
+            if kind.endswith("bf16"):
+                bias = bias.to(BF)
+        dv = lambda t: None if t is None else t.to(DEV)
+        out = run(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), pad=dv(pad), bias=dv(bias))
+        for h in range(H):
+            ref = oracle_rows(q, k, v, idx.numpy(), 0, h, pad=pad, bias=bias)
+            check_attn(f64(out[0, h]), ref, f"{kind} D={D} N={N} h{h}")
+        if pad is not None:
+            vg = v.clone()
+            vg[:, :, 5::7] = 1e4
+            o2 = run(q.to(DEV), k.to(DEV), vg.to(DEV), idx.to(DEV), pad=dv(pad), bias=dv(bias))
+            assert torch.equal(out, o2)
+
+
 def test_row_constant_mask_elision_is_invisible():
     """A row-constant additive bias (removable by the criterion) changes the
     GPU result only by rounding."""
