@@ -90,8 +90,10 @@ constexpr uint32_t kControlRegs = 88;
 // Column pairs (bit e of the mask = pair e of each 16-pair group) whose
 // exponentials go to the FMA-pipe polynomial instead of the MUFU unit, on the
 // mask-free path.  Balances the two pipes (measured on B200 at the 2560^2
-// SRSU launch: 1/4 of the pairs is best, 1/2 is slower than none); exact
-// zero weights of kept masks stay on the MUFU path.
+// SRSU launch: 1/4 of the pairs is best, 1/2 is slower than none).  Kept
+// masks put every exponential on the MUFU unit (measured faster there: the
+// mask terms already load the FMA pipe), which also gives masked keys their
+// exact zero weight.
 #ifndef SAFEDIT_EXP2_FMA_MASK
 #define SAFEDIT_EXP2_FMA_MASK 0x8888u
 #endif
@@ -469,12 +471,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 f2_fma(f2_pack(x[c * 32 + 2 * e], x[c * 32 + 2 * e + 1]), mul2, negm2);
             float a0, a1, p0, p1;
             f2_unpack(a2, a0, a1);
-            if ((kExp2FmaMask >> e) & 1u) {
+            if (!MASKED && ((kExp2FmaMask >> e) & 1u)) {
               exp2_pair_fma(a0, a1, p0, p1);
-              if (MASKED) {  // exact zero weight below the normal range (masked keys)
-                p0 = a0 < -126.f ? 0.f : p0;
-                p1 = a1 < -126.f ? 0.f : p1;
-              }
             } else {
               p0 = ex2_approx(a0);
               p1 = ex2_approx(a1);
