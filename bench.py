@@ -665,7 +665,7 @@ def run_stress(args):
     """The mask-path stress workload (B=1, H=32, N=16384, d=128, |S|=4915 from
     the clustered blob scores): SRSU attention with the mask elided (no mask
     input), with a kept text-padding key mask (trailing 1/8 of the keys -inf),
-    with a kept non-uniform bf16 bias [1,1,N,N], and with both; the row-constant check on
+    with a kept non-uniform bf16 bias [1,1,N,N], with both, and with the bias in f32; the row-constant check on
     an all-zero mask (elided: read fully) and on the padding mask (kept: the
     check stops at the first kept row).  Best of `--reps` CUDA-event timings;
     one JSON line per case (not a bench line)."""
@@ -683,6 +683,7 @@ def run_stress(args):
     pad = torch.zeros(1, w.N, device=dev)
     pad[:, w.N - w.N // 8:] = float("-inf")
     bias = wl.mask(w, "bias", device=dev)            # [1,1,N,N] bf16
+    bias32 = bias.float()                            # the same bias in f32 (1.07 GB)
     zero = wl.mask(w, "zero", device=dev)
     padmask = wl.mask(w, "textpad", device=dev)
     verdict = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -707,6 +708,7 @@ def run_stress(args):
         "srsu_kept_bias": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, None, bias, 0.0, o, 1, stream),
         "srsu_kept_padding_and_bias": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, pad, bias, 0.0, o, 1,
                                                                      stream),
+        "srsu_kept_bias_f32": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, None, bias32, 0.0, o, 1, stream),
     }
     base = None
     for name, fn in cases.items():

@@ -54,7 +54,7 @@ struct AttnCfg {
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES * TILE_BYTES + BAR_BYTES;
   static constexpr int PAD_BYTES = 8 * 2 * 128 * 4;    // per warp: 2 key tiles of pad
-  static constexpr int BIAS_BYTES = 8 * 32 * 128;      // per warp: 32 rows x 64 bf16 keys
+  static constexpr int BIAS_BYTES = 8 * 32 * 128;      // per warp: 32 rows x 128 bytes
   static_assert(SMEM_BYTES + PAD_BYTES <= 232448, "shared memory");
   static_assert(SMEM_BYTES + BIAS_BYTES <= 232448, "shared memory");
   static_assert(D == 64 || D == 96 || D == 128, "head dim");
@@ -83,10 +83,16 @@ struct AttnParams {
 // 12 warps: two softmax warpgroups (warps 0-7), then TMA producer (8), MMA
 // issuer (9) and two spare warps (10, 11) completing the third warpgroup, so
 // that setmaxnreg can move registers from the control warpgroup (88 each) to
-// the softmax warpgroups (208 each): 256*208 + 128*88 = 384*168.
+// the softmax warpgroups (208 each): 256*208 + 128*88 = 384*168.  The
+// kept-mask kernels hold half a key tile of scores at a time and split
+// 192 / 120 (256*192 + 128*120 = 384*168) when their mask operands are
+// staged in shared memory, which leaves them (nearly) spill-free; kernels
+// that read a mask operand in place keep 208, for the loads in flight.
 constexpr int kAttnThreads = 384;
-constexpr uint32_t kSoftmaxRegs = 208;
-constexpr uint32_t kControlRegs = 88;
+constexpr uint32_t kSoftmaxRegs = 208, kControlRegs = 88;
+constexpr uint32_t kSoftmaxRegsMasked = 192, kControlRegsMasked = 120;
+static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= 384 * 168, "register split");
+static_assert(256 * kSoftmaxRegsMasked + 128 * kControlRegsMasked <= 384 * 168, "register split");
 // Column pairs (bit e of the mask = pair e of each 16-pair group) whose
 // exponentials go to the FMA-pipe polynomial instead of the MUFU unit, on the
 // mask-free path.  Balances the two pipes (measured on B200 at the 2560^2
@@ -132,24 +138,27 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-// Stages the bf16 bias of this warp's 32 query rows, keys [k0, k0 + 64),
-// into the warp's 4 KB buffer with coalesced copies (each instruction moves
-// four 128-byte row segments).  Row rr's 16-byte chunk ch lands in slot
-// ch ^ (rr & 7) of the row's 128 bytes, so that the row-per-thread reads
-// back are free of bank conflicts.  qrow[i] is the query index of row
-// 4 i + lane / 8 (negative: no row); keys past Nk are zero-filled or skipped.
-__device__ __forceinline__ void stage_bias_bf16(uint32_t buf, const __nv_bfloat16* base, int64_t sq,
-                                                const int (&qrow)[8], int k0, int Nk, int lane) {
+// Stages the bias of this warp's 32 query rows, one 128-byte row segment
+// each (64 bf16 or 32 f32 keys from key k0), into the warp's 4 KB buffer with
+// coalesced copies (each instruction moves four row segments).  Row rr's
+// 16-byte chunk ch lands in slot ch ^ (rr & 7) of the row's 128 bytes, so
+// that the row-per-thread reads back are free of bank conflicts.  qrow[i] is
+// the query index of row 4 i + lane / 8 (negative: no row); keys past Nk are
+// zero-filled or skipped.
+template <typename T>
+__device__ __forceinline__ void stage_bias(uint32_t buf, const T* base, int64_t sq, const int (&qrow)[8],
+                                           int k0, int Nk, int lane) {
+  constexpr int EPC = 16 / int(sizeof(T));  // elements per 16-byte chunk
   const int ch = lane & 7;
-  const int left = Nk - (k0 + ch * 8);
+  const int left = Nk - (k0 + ch * EPC);
   if (left > 0) {
-    const uint32_t bytes = left >= 8 ? 16u : uint32_t(left) * 2u;
+    const uint32_t bytes = left >= EPC ? 16u : uint32_t(left) * uint32_t(sizeof(T));
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int rr = 4 * i + (lane >> 3);
       if (qrow[i] >= 0)
         cp_async16(buf + uint32_t(rr * 128 + ((ch ^ (rr & 7)) << 4)),
-                   base + int64_t(qrow[i]) * sq + k0 + ch * 8, bytes);
+                   base + int64_t(qrow[i]) * sq + k0 + ch * EPC, bytes);
     }
   }
   cp_async_commit();
@@ -161,6 +170,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                        const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = AttnCfg<D>;
   constexpr bool MASKED = PAD || BIAS != kBiasNone;
+  // every mask operand staged in shared memory (none read in place)
+  constexpr bool STAGED = MASKED && !(PAD && BIAS != kBiasNone);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -216,7 +227,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp < 8) {
     // ================================================== softmax warpgroups
-    setmaxnreg_inc<kSoftmaxRegs>();
+    setmaxnreg_inc<STAGED ? kSoftmaxRegsMasked : kSoftmaxRegs>();
     const int t = warp >> 2;            // query tile
     const int wr = warp & 3;            // TMEM lane quarter
     const int tid = threadIdx.x & 127;  // thread within the warpgroup
@@ -262,33 +273,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // so that the load latency overlaps the current columns instead of
     // sitting between S and P.  The pad (alone): one tile ahead, one 16-byte
     // load per lane into this warp's double-buffered 512-byte slice in shared
-    // memory, read back as broadcasts.  A bf16 bias: one 64-key pass ahead,
-    // copied asynchronously and coalesced into this warp's 4 KB buffer, read
-    // back row per thread.  An f32 bias, and the pad beside a bf16 bias (no
-    // shared memory left for both buffers), are read in place.
-    constexpr bool PAD_SMEM = PAD && BIAS != kBiasBf16;
+    // memory, read back as broadcasts.  A bias: one pass (64 bf16 or 32 f32
+    // keys) ahead, copied asynchronously and coalesced into this warp's 4 KB
+    // buffer, read back row per thread.  The pad beside a bias is read in
+    // place (no shared memory left for both buffers).
+    constexpr bool PAD_SMEM = PAD && BIAS == kBiasNone;
+    using BiasT = typename std::conditional<BIAS == kBiasF32, float, __nv_bfloat16>::type;
     uint8_t* const mask_smem = smem + C::SMEM_TILES * C::TILE_BYTES + C::BAR_BYTES;
-    float* const pad_smem = PAD_SMEM ? reinterpret_cast<float*>(mask_smem) + warp * 256 : nullptr;
+    const uint32_t pad_buf = smem_u32(mask_smem) + uint32_t(warp * 1024);
     const uint32_t bias_buf = smem_u32(mask_smem) + uint32_t(warp * 4096);
     const float* const pad_row = PAD ? p.pad + b * p.pad_sb : nullptr;
     float4 pad_next = make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (PAD_SMEM) pad_next = load_pad4(pad_row, 4 * lane, p.Nk);
-    const __nv_bfloat16* const bias_bh =
-        BIAS == kBiasBf16
-            ? static_cast<const __nv_bfloat16*>(p.bias) + b * p.bias_sb + h * p.bias_sh
+    const BiasT* const bias_bh =
+        BIAS != kBiasNone
+            ? static_cast<const BiasT*>(p.bias) + b * p.bias_sb + h * p.bias_sh
             : nullptr;
-    int qrow[8];  // query index of row 4 i + lane / 8 of this warp (bf16 bias staging)
-    if constexpr (BIAS == kBiasBf16) {
+    int qrow[8];  // query index of row 4 i + lane / 8 of this warp (bias staging)
+    if constexpr (BIAS != kBiasNone) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) qrow[i] = __shfl_sync(0xffffffffu, my_q, 4 * i + (lane >> 3));
-      stage_bias_bf16(bias_buf, bias_bh, p.bias_sq, qrow, 0, p.Nk, lane);
+      stage_bias(bias_buf, bias_bh, p.bias_sq, qrow, 0, p.Nk, lane);
     }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       const int key0 = j * C::BN;
       if constexpr (PAD_SMEM) {
-        *reinterpret_cast<float4*>(pad_smem + (j & 1) * 128 + 4 * lane) = pad_next;
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                         pad_buf + uint32_t((j & 1) * 512 + lane * 16)),
+                     "f"(pad_next.x), "f"(pad_next.y), "f"(pad_next.z), "f"(pad_next.w)
+                     : "memory");
         __syncwarp();
         if (j + 1 < nk) pad_next = load_pad4(pad_row, key0 + C::BN + 4 * lane, p.Nk);
       }
@@ -298,13 +313,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tc_fence_after();
       // The mask-free path takes the tile's 128 columns in one pass.  With
-      // kept masks the tile goes in two passes of 64 columns, each with its
-      // own online-softmax max, which keeps the mask operands of a pass in
-      // registers beside its scores; if the second pass raises the running
-      // max, the first pass's P (already in TMEM) is rescaled with it.
-      constexpr int NH = MASKED ? 2 : 1, HW = 128 / NH;
-      float alpha_p0 = 1.f;  // factor owed by the first pass's P
-      bool owe_p0 = false;
+      // kept masks the tile goes in passes of 64 columns (32 with an f32
+      // bias: one 128-byte bias row segment per pass), each with its own
+      // online-softmax max, which keeps the mask operands of a pass in
+      // registers beside its scores; when a pass raises the running max, the
+      // earlier passes' P (already in TMEM) is rescaled with it.
+      constexpr int NH = !MASKED ? 1 : (BIAS == kBiasF32 ? 4 : 2), HW = 128 / NH;
       // one pass over columns [hf * HW, hf * HW + HW); hf is a compile-time
       // constant, so every register array below is indexed statically
       auto pass = [&](auto hf_tag) {
@@ -326,7 +340,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if constexpr (MASKED) {
           const uint64_t sc2 = f2_pack(p.scale, p.scale);
           const int lim = p.Nk - key0 - c0;
-          if constexpr (BIAS == kBiasBf16) {  // this pass's bias has landed
+          if constexpr (BIAS != kBiasNone) {  // this pass's bias has landed
             cp_async_wait_all();
             __syncwarp();
           }
@@ -334,11 +348,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < HW; c += 8) {
             float add[8];
             if constexpr (PAD_SMEM) {
-              const float* const ps = pad_smem + (j & 1) * 128 + c0;
-              const float4 a0 = *reinterpret_cast<const float4*>(ps + c);
-              const float4 a1 = *reinterpret_cast<const float4*>(ps + c + 4);
-              add[0] = a0.x; add[1] = a0.y; add[2] = a0.z; add[3] = a0.w;
-              add[4] = a1.x; add[5] = a1.y; add[6] = a1.z; add[7] = a1.w;
+              const uint32_t ps = pad_buf + uint32_t((j & 1) * 512 + (c0 + c) * 4);
+              asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                           : "=f"(add[0]), "=f"(add[1]), "=f"(add[2]), "=f"(add[3])
+                           : "r"(ps));
+              asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                           : "=f"(add[4]), "=f"(add[5]), "=f"(add[6]), "=f"(add[7])
+                           : "r"(ps + 16u));
             } else if constexpr (PAD) {
               const float* const pr = pad_row + key0 + c0 + c;
               if (c + 8 <= lim) {
@@ -365,19 +381,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 add[2 * e + 1] += __uint_as_float(ws[e] & 0xFFFF0000u);
               }
             } else if constexpr (BIAS == kBiasF32) {
-              if (my_q >= 0) {
-                const float* br = static_cast<const float*>(p.bias) + b * p.bias_sb +
-                                  h * p.bias_sh + int64_t(my_q) * p.bias_sq + key0 + c0 + c;
-                if (c + 8 <= lim) {
-                  const float4 b0 = __ldg(reinterpret_cast<const float4*>(br));
-                  const float4 b1 = __ldg(reinterpret_cast<const float4*>(br + 4));
-                  add[0] += b0.x; add[1] += b0.y; add[2] += b0.z; add[3] += b0.w;
-                  add[4] += b1.x; add[5] += b1.y; add[6] += b1.z; add[7] += b1.w;
-                } else {
 #pragma unroll
-                  for (int e = 0; e < 8; ++e)
-                    if (c + e < lim) add[e] += __ldg(br + e);
-                }
+              for (int hc = 0; hc < 2; ++hc) {
+                float w[4];
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(w[0]), "=f"(w[1]), "=f"(w[2]), "=f"(w[3])
+                             : "r"(bias_buf +
+                                   uint32_t(lane * 128 + (((c / 4 + hc) ^ (lane & 7)) << 4))));
+#pragma unroll
+                for (int e = 0; e < 4; ++e) add[4 * hc + e] += w[e];
               }
             }
 #pragma unroll
@@ -389,12 +401,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               x[c + e + 1] = y1;
             }
           }
-          if constexpr (BIAS == kBiasBf16) {
+          if constexpr (BIAS != kBiasNone) {
             // every lane has read the buffer: stage the next pass into it
             __syncwarp();
             const int k_next = key0 + c0 + HW;
-            if (k_next < nk * C::BN)
-              stage_bias_bf16(bias_buf, bias_bh, p.bias_sq, qrow, k_next, p.Nk, lane);
+            if (k_next < nk * C::BN) stage_bias(bias_buf, bias_bh, p.bias_sq, qrow, k_next, p.Nk, lane);
           }
         }
         if (key0 + C::BN > p.Nk) {  // ragged last key tile
@@ -421,17 +432,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mt *= MASKED ? kLog2e : sl2;
         }
         // lazy rescale: the running max moves only when it grows by > 2^8
-        bool need_o = false;
+        bool need_o = false, raised = false;
         float alpha = 1.f;
         if (mt > m_run + kRescaleThreshold) {
           alpha = ex2_approx(m_run - mt);  // 0 when m_run = -inf
           l_run *= alpha;
           m_run = mt;
           need_o = (j > 0);
-          if (hf == 1) {
-            owe_p0 = true;
-            alpha_p0 = alpha;
-          }
+          raised = true;
         }
         if (__any_sync(0xffffffffu, need_o)) {
 #pragma unroll
@@ -444,17 +452,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st32(tO + uint32_t(c * 32), r);
           }
         }
-        if (hf == 1 && __any_sync(0xffffffffu, owe_p0)) {
-          // the first pass's 64 probabilities (32 packed columns)
-          tmem_wait_st();
-          uint32_t r[32];
-          tmem_ld32(tS, r);
-          tmem_wait_ld();
+        if constexpr (hf > 0) {
+          // the earlier passes' probabilities (hf * HW / 2 packed columns)
+          constexpr int PCOLS = hf * HW / 2;
+          if (__any_sync(0xffffffffu, raised)) {
+            tmem_wait_st();
+            if constexpr (PCOLS % 32 == 0) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            r[e] = pack_bf16x2(__uint_as_float(r[e] << 16) * alpha_p0,
-                               __uint_as_float(r[e] & 0xFFFF0000u) * alpha_p0);
-          tmem_st32(tS, r);
+              for (int q = 0; q < PCOLS / 32; ++q) {
+                uint32_t r[32];
+                tmem_ld32(tS + uint32_t(q * 32), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  r[e] = pack_bf16x2(__uint_as_float(r[e] << 16) * alpha,
+                                     __uint_as_float(r[e] & 0xFFFF0000u) * alpha);
+                tmem_st32(tS + uint32_t(q * 32), r);
+              }
+            } else {
+#pragma unroll
+              for (int q = 0; q < PCOLS / 16; ++q) {
+                uint32_t r[16];
+                tmem_ld16(tS + uint32_t(q * 16), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                  r[e] = pack_bf16x2(__uint_as_float(r[e] << 16) * alpha,
+                                     __uint_as_float(r[e] & 0xFFFF0000u) * alpha);
+                tmem_st16(tS + uint32_t(q * 16), r);
+              }
+            }
+          }
         }
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
         const float mul = MASKED ? kLog2e : sl2;
@@ -489,12 +517,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       };
       pass(std::integral_constant<int, 0>{});
-      if constexpr (NH == 2) pass(std::integral_constant<int, 1>{});
+      if constexpr (NH > 1) pass(std::integral_constant<int, 1>{});
+      if constexpr (NH > 2) {
+        pass(std::integral_constant<int, 2>{});
+        pass(std::integral_constant<int, 3>{});
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(P_FULL + t));
     }
-    if constexpr (BIAS == kBiasBf16) cp_async_wait_all();  // none in flight at exit
+    if constexpr (BIAS != kBiasNone) cp_async_wait_all();  // none in flight at exit
     // ---- epilogue: O / l -> bf16 rows
     if (ok && wait_warp(BAR(O_FULL), 0u, ctl)) {
       tc_fence_after();
@@ -524,7 +556,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
   } else {
-    setmaxnreg_dec<kControlRegs>();
+    setmaxnreg_dec<STAGED ? kControlRegsMasked : kControlRegs>();
     if (warp == 8) {
       // ================================================ TMA producer (K, V)
       if (lane == 0) {
@@ -644,7 +676,7 @@ static safedit_status launch_attn(const CUtensorMap& tmK, const CUtensorMap& tmV
   using C = AttnCfg<D>;
   auto kern = attn_subset_kernel<D, PAD, BIAS>;
   constexpr int smem_bytes =
-      C::SMEM_BYTES + (BIAS == kBiasBf16 ? C::BIAS_BYTES : (PAD ? C::PAD_BYTES : 0));
+      C::SMEM_BYTES + (BIAS != kBiasNone ? C::BIAS_BYTES : (PAD ? C::PAD_BYTES : 0));
   safedit_status st = set_smem(reinterpret_cast<const void*>(kern), smem_bytes);
   if (st != SAFEDIT_OK) return st;
   dim3 grid((p.n_rows + 255) / 256, B * p.H);

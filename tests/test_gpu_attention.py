@@ -132,10 +132,10 @@ def test_kept_masks_key_padding_and_bias():
 def test_kept_mask_variants_ragged_tail_and_max_jumps(D, kind):
     """Every kept-mask kernel variant.  The last key tile is ragged, ending
     inside the first and inside the second 64-column pass; the additive terms
-    raise the running max by far more than the lazy-rescale threshold, once
-    inside the first pass of a tile and once inside the second (the first
-    pass's probabilities, already in TMEM, are then rescaled); padded keys
-    hold garbage values that must get exactly zero weight."""
+    raise the running max by far more than the lazy-rescale threshold inside
+    every pass position of a tile (the earlier passes' probabilities, already
+    in TMEM, are then rescaled); padded keys hold garbage values that must get
+    exactly zero weight."""
     B, H, kr = 1, 2, 150
     for N in (696, 600):  # last tile: 56 keys, 88 keys
         q, k, v = _qkv(B, H, N, N, D, seed=1000 + N + D)
@@ -151,6 +151,10 @@ def test_kept_mask_variants_ragged_tail_and_max_jumps(D, kind):
             bias = torch.randn(B, H if kind.endswith("f32") else 1, N, N, generator=g) * 0.5
             bias[..., ::2, 384 + 64:384 + 80] += 12.0   # tile 3, second pass, even query rows
             bias[..., 1::2, 512 + 3:512 + 9] += 10.0    # ragged tile 4, first pass, odd rows
+            # with an f32 bias the passes are 32 keys wide: jumps in the second
+            # and in the fourth pass of tile 2 as well
+            bias[..., 1::3, 256 + 40:256 + 44] += 14.0
+            bias[..., 2::3, 256 + 100:256 + 110] += 16.0
             if kind.endswith("bf16"):
                 bias = bias.to(BF)
         dv = lambda t: None if t is None else t.to(DEV)
