@@ -53,10 +53,9 @@ struct AttnCfg {
   static constexpr int SMEM_TILES = 2 + 2 * NS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES * TILE_BYTES + BAR_BYTES;
-  static constexpr int PAD_BYTES = 8 * 2 * 128 * 4;    // per warp: 2 key tiles of pad
+  static constexpr int PAD_BYTES = 3 * 128 * 4;        // pad of 3 key tiles (all warps)
   static constexpr int BIAS_BYTES = 8 * 32 * 128;      // per warp: 32 rows x 128 bytes
-  static_assert(SMEM_BYTES + PAD_BYTES <= 232448, "shared memory");
-  static_assert(SMEM_BYTES + BIAS_BYTES <= 232448, "shared memory");
+  static_assert(SMEM_BYTES + BIAS_BYTES + PAD_BYTES <= 232448, "shared memory");
   static_assert(D == 64 || D == 96 || D == 128, "head dim");
   static_assert(256 + 2 * D <= 512, "TMEM columns");
 };
@@ -85,9 +84,8 @@ struct AttnParams {
 // that setmaxnreg can move registers from the control warpgroup (88 each) to
 // the softmax warpgroups (208 each): 256*208 + 128*88 = 384*168.  The
 // kept-mask kernels hold half a key tile of scores at a time and split
-// 192 / 120 (256*192 + 128*120 = 384*168) when their mask operands are
-// staged in shared memory, which leaves them (nearly) spill-free; kernels
-// that read a mask operand in place keep 208, for the loads in flight.
+// 192 / 120 (256*192 + 128*120 = 384*168), which leaves them (nearly)
+// spill-free.
 constexpr int kAttnThreads = 384;
 constexpr uint32_t kSoftmaxRegs = 208, kControlRegs = 88;
 constexpr uint32_t kSoftmaxRegsMasked = 192, kControlRegsMasked = 120;
@@ -170,8 +168,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                        const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = AttnCfg<D>;
   constexpr bool MASKED = PAD || BIAS != kBiasNone;
-  // every mask operand staged in shared memory (none read in place)
-  constexpr bool STAGED = MASKED && !(PAD && BIAS != kBiasNone);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -227,7 +223,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp < 8) {
     // ================================================== softmax warpgroups
-    setmaxnreg_inc<STAGED ? kSoftmaxRegsMasked : kSoftmaxRegs>();
+    setmaxnreg_inc<MASKED ? kSoftmaxRegsMasked : kSoftmaxRegs>();
     const int t = warp >> 2;            // query tile
     const int wr = warp & 3;            // TMEM lane quarter
     const int tid = threadIdx.x & 127;  // thread within the warpgroup
@@ -271,20 +267,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float sl2 = p.scale_log2;
     // Kept masks.  Their operands for the next key columns are fetched ahead,
     // so that the load latency overlaps the current columns instead of
-    // sitting between S and P.  The pad (alone): one tile ahead, one 16-byte
-    // load per lane into this warp's double-buffered 512-byte slice in shared
-    // memory, read back as broadcasts.  A bias: one pass (64 bf16 or 32 f32
-    // keys) ahead, copied asynchronously and coalesced into this warp's 4 KB
-    // buffer, read back row per thread.  The pad beside a bias is read in
-    // place (no shared memory left for both buffers).
-    constexpr bool PAD_SMEM = PAD && BIAS == kBiasNone;
-    using BiasT = typename std::conditional<BIAS == kBiasF32, float, __nv_bfloat16>::type;
+    // sitting between S and P.  The pad: one tile ahead, one 16-byte load per
+    // lane into a three-slot ring (slot = tile mod 3, 1.5 KB) shared by all
+    // eight softmax warps, read back as broadcasts.  Every warp writes the
+    // same values there (before waiting for the tile's S) and reads them after
+    // its own __syncwarp.  A warp that writes tile j + 1 has finished tile j,
+    // whose S needed P(j - 1) of its own query tile and P(j - 2) of the other
+    // (the MMA issue order), so every other warp is reading tile j - 1 or
+    // later: slots j - 1, j and j + 1 are distinct.
+    // A bias: one pass (64 bf16 or 32 f32 keys) ahead, copied asynchronously
+    // and coalesced into this warp's 4 KB buffer, read back row per thread.
     uint8_t* const mask_smem = smem + C::SMEM_TILES * C::TILE_BYTES + C::BAR_BYTES;
-    const uint32_t pad_buf = smem_u32(mask_smem) + uint32_t(warp * 1024);
     const uint32_t bias_buf = smem_u32(mask_smem) + uint32_t(warp * 4096);
+    const uint32_t pad_buf = smem_u32(mask_smem) + uint32_t(BIAS != kBiasNone ? C::BIAS_BYTES : 0);
     const float* const pad_row = PAD ? p.pad + b * p.pad_sb : nullptr;
     float4 pad_next = make_float4(0.f, 0.f, 0.f, 0.f);
-    if constexpr (PAD_SMEM) pad_next = load_pad4(pad_row, 4 * lane, p.Nk);
+    if constexpr (PAD) pad_next = load_pad4(pad_row, 4 * lane, p.Nk);
+    using BiasT = typename std::conditional<BIAS == kBiasF32, float, __nv_bfloat16>::type;
     const BiasT* const bias_bh =
         BIAS != kBiasNone
             ? static_cast<const BiasT*>(p.bias) + b * p.bias_sb + h * p.bias_sh
@@ -297,11 +296,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < nk; ++j) {
+    int pad_slot = 0;  // j mod 3
+    for (int j = 0; j < nk; ++j, pad_slot = (pad_slot == 2) ? 0 : pad_slot + 1) {
       const int key0 = j * C::BN;
-      if constexpr (PAD_SMEM) {
+      if constexpr (PAD) {
         asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
-                         pad_buf + uint32_t((j & 1) * 512 + lane * 16)),
+                         pad_buf + uint32_t(pad_slot * 512 + lane * 16)),
                      "f"(pad_next.x), "f"(pad_next.y), "f"(pad_next.z), "f"(pad_next.w)
                      : "memory");
         __syncwarp();
@@ -347,25 +347,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int c = 0; c < HW; c += 8) {
             float add[8];
-            if constexpr (PAD_SMEM) {
-              const uint32_t ps = pad_buf + uint32_t((j & 1) * 512 + (c0 + c) * 4);
+            if constexpr (PAD) {
+              const uint32_t ps = pad_buf + uint32_t(pad_slot * 512 + (c0 + c) * 4);
               asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                            : "=f"(add[0]), "=f"(add[1]), "=f"(add[2]), "=f"(add[3])
                            : "r"(ps));
               asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                            : "=f"(add[4]), "=f"(add[5]), "=f"(add[6]), "=f"(add[7])
                            : "r"(ps + 16u));
-            } else if constexpr (PAD) {
-              const float* const pr = pad_row + key0 + c0 + c;
-              if (c + 8 <= lim) {
-                const float4 a0 = __ldg(reinterpret_cast<const float4*>(pr));
-                const float4 a1 = __ldg(reinterpret_cast<const float4*>(pr + 4));
-                add[0] = a0.x; add[1] = a0.y; add[2] = a0.z; add[3] = a0.w;
-                add[4] = a1.x; add[5] = a1.y; add[6] = a1.z; add[7] = a1.w;
-              } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) add[e] = (c + e < lim) ? __ldg(pr + e) : 0.f;
-              }
             } else {
 #pragma unroll
               for (int e = 0; e < 8; ++e) add[e] = 0.f;
@@ -556,7 +545,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
   } else {
-    setmaxnreg_dec<STAGED ? kControlRegsMasked : kControlRegs>();
+    setmaxnreg_dec<MASKED ? kControlRegsMasked : kControlRegs>();
     if (warp == 8) {
       // ================================================ TMA producer (K, V)
       if (lane == 0) {
@@ -676,7 +665,7 @@ static safedit_status launch_attn(const CUtensorMap& tmK, const CUtensorMap& tmV
   using C = AttnCfg<D>;
   auto kern = attn_subset_kernel<D, PAD, BIAS>;
   constexpr int smem_bytes =
-      C::SMEM_BYTES + (BIAS != kBiasNone ? C::BIAS_BYTES : (PAD ? C::PAD_BYTES : 0));
+      C::SMEM_BYTES + (BIAS != kBiasNone ? C::BIAS_BYTES : 0) + (PAD ? C::PAD_BYTES : 0);
   safedit_status st = set_smem(reinterpret_cast<const void*>(kern), smem_bytes);
   if (st != SAFEDIT_OK) return st;
   dim3 grid((p.n_rows + 255) / 256, B * p.H);
