@@ -53,7 +53,7 @@ struct AttnCfg {
   static constexpr int SMEM_TILES = 2 + 2 * NS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES * TILE_BYTES + BAR_BYTES;
-  static constexpr int PAD_BYTES = 3 * 128 * 4;        // pad of 3 key tiles (all warps)
+  static constexpr int PAD_BYTES = 3 * 128 * 4 + 128;  // pad of 3 key tiles (all warps) + live-tile bits
   static constexpr int BIAS_BYTES = 8 * 32 * 128;      // per warp: 32 rows x 128 bytes
   static_assert(SMEM_BYTES + BIAS_BYTES + PAD_BYTES <= 232448, "shared memory");
   static_assert(D == 64 || D == 96 || D == 128, "head dim");
@@ -105,6 +105,9 @@ constexpr uint32_t kExp2FmaMask = SAFEDIT_EXP2_FMA_MASK;
 constexpr uint64_t kDrainNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Key tiles whose pad is -inf throughout carry exactly zero weight and are
+// skipped (a bitmask of live tiles in shared memory; up to 1024 tiles).
+constexpr int kLiveWords = 32;
 
 __device__ __forceinline__ uint32_t swizzle_off(uint32_t off, uint32_t layout) {
   return layout == 2u ? (off ^ (((off >> 7) & 7u) << 4)) : (off ^ (((off >> 7) & 3u) << 4));
@@ -189,6 +192,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int b = bh / p.H, h = bh - b * p.H;
   const int row0 = blockIdx.x * 256;
   const int nk = (p.Nk + C::BN - 1) / C::BN;
+  // live key tiles (kept key padding): a tile whose pad entries are all -inf
+  // adds nothing to any row (its weights are exactly zero) and is skipped by
+  // every role; every role walks the same bitmask, so they agree on the
+  // sequence of tiles
+  uint32_t* const live_bits = reinterpret_cast<uint32_t*>(
+      smem + C::SMEM_TILES * C::TILE_BYTES + C::BAR_BYTES + (BIAS != kBiasNone ? C::BIAS_BYTES : 0) +
+      3 * 128 * 4);
+  const bool skip_tiles = PAD && nk <= kLiveWords * 32;
+  if constexpr (PAD) {
+    if (threadIdx.x < kLiveWords) live_bits[threadIdx.x] = 0u;
+    __syncthreads();
+    if (skip_tiles) {
+      const float* pr = p.pad + b * p.pad_sb;
+      for (int j = threadIdx.x >> 5; j < nk; j += kAttnThreads / 32) {
+        bool live = false;
+        for (int c = lane; c < C::BN && j * C::BN + c < p.Nk; c += 32)
+          live |= !(__ldg(pr + j * C::BN + c) == -INFINITY);
+        if (__any_sync(0xffffffffu, live) && lane == 0) atomicOr(live_bits + (j >> 5), 1u << (j & 31));
+      }
+    }
+  }
+  const uint32_t live_s = smem_u32(live_bits);
+  auto live_word = [&](int w) -> uint32_t {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(live_s + uint32_t(w) * 4u));
+    return v;
+  };
+  // first live tile at or after j (nk if none)
+  auto next_live = [&](int j) -> int {
+    if (!skip_tiles) return j;
+    while (j < nk) {
+      const uint32_t w = live_word(j >> 5) >> (j & 31);
+      if (w) return j + __ffs(w) - 1;
+      j = (j | 31) + 1;
+    }
+    return nk;
+  };
+  auto live_count = [&]() -> int {
+    if (!skip_tiles) return nk;
+    int n = 0;
+    for (int w = 0; w < (nk + 31) / 32; ++w) n += __popc(live_word(w));
+    return n;
+  };
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -282,7 +328,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t pad_buf = smem_u32(mask_smem) + uint32_t(BIAS != kBiasNone ? C::BIAS_BYTES : 0);
     const float* const pad_row = PAD ? p.pad + b * p.pad_sb : nullptr;
     float4 pad_next = make_float4(0.f, 0.f, 0.f, 0.f);
-    if constexpr (PAD) pad_next = load_pad4(pad_row, 4 * lane, p.Nk);
+    const int n_live = live_count();
+    int j_first = next_live(0);
+    if constexpr (PAD) pad_next = load_pad4(pad_row, j_first * C::BN + 4 * lane, p.Nk);
     using BiasT = typename std::conditional<BIAS == kBiasF32, float, __nv_bfloat16>::type;
     const BiasT* const bias_bh =
         BIAS != kBiasNone
@@ -292,22 +340,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if constexpr (BIAS != kBiasNone) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) qrow[i] = __shfl_sync(0xffffffffu, my_q, 4 * i + (lane >> 3));
-      stage_bias(bias_buf, bias_bh, p.bias_sq, qrow, 0, p.Nk, lane);
+      stage_bias(bias_buf, bias_bh, p.bias_sq, qrow, j_first * C::BN, p.Nk, lane);
     }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int pad_slot = 0;  // j mod 3
-    for (int j = 0; j < nk; ++j, pad_slot = (pad_slot == 2) ? 0 : pad_slot + 1) {
+    int pad_slot = 0;  // it mod 3
+    // it counts the live key tiles processed (it drives the barrier phases),
+    // j is the key tile itself
+    int j = j_first;
+    for (int it = 0; it < n_live; ++it) {
       const int key0 = j * C::BN;
+      const int j_next = next_live(j + 1);
       if constexpr (PAD) {
         asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
                          pad_buf + uint32_t(pad_slot * 512 + lane * 16)),
                      "f"(pad_next.x), "f"(pad_next.y), "f"(pad_next.z), "f"(pad_next.w)
                      : "memory");
         __syncwarp();
-        if (j + 1 < nk) pad_next = load_pad4(pad_row, key0 + C::BN + 4 * lane, p.Nk);
+        if (j_next < nk) pad_next = load_pad4(pad_row, j_next * C::BN + 4 * lane, p.Nk);
       }
-      if (!wait_warp(BAR(S_FULL + t), uint32_t(j & 1), ctl)) {
+      if (!wait_warp(BAR(S_FULL + t), uint32_t(it & 1), ctl)) {
         ok = false;
         break;
       }
@@ -393,7 +445,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if constexpr (BIAS != kBiasNone) {
             // every lane has read the buffer: stage the next pass into it
             __syncwarp();
-            const int k_next = key0 + c0 + HW;
+            const int k_next = (hf + 1 < NH) ? key0 + c0 + HW : j_next * C::BN;
             if (k_next < nk * C::BN) stage_bias(bias_buf, bias_bh, p.bias_sq, qrow, k_next, p.Nk, lane);
           }
         }
@@ -427,7 +479,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           alpha = ex2_approx(m_run - mt);  // 0 when m_run = -inf
           l_run *= alpha;
           m_run = mt;
-          need_o = (j > 0);
+          need_o = (it > 0);
           raised = true;
         }
         if (__any_sync(0xffffffffu, need_o)) {
@@ -514,6 +566,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(P_FULL + t));
+      j = j_next;
+      pad_slot = (pad_slot == 2) ? 0 : pad_slot + 1;
     }
     if constexpr (BIAS != kBiasNone) cp_async_wait_all();  // none in flight at exit
     // ---- epilogue: O / l -> bf16 rows
@@ -522,6 +576,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool live = my_q >= 0;
       if (live && !(l_run > 0.f)) set_status(p.status, SAFEDIT_ERR_MASKED_ROW);
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      // with skipped key tiles O may never have been written: a row with no
+      // weight (fully masked: an error, reported above) is written as zeros
+      const bool zero_row = PAD && !(l_run > 0.f);
       __nv_bfloat16* orow = nullptr;
       if (live) {
         const int64_t orow_idx = p.out_scattered ? int64_t(my_q) : int64_t(my_row);
@@ -536,7 +593,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
+            w[e] = zero_row ? 0u
+                            : pack_bf16x2(__uint_as_float(r[2 * e]) * inv,
+                                          __uint_as_float(r[2 * e + 1]) * inv);
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
@@ -550,23 +609,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // ================================================ TMA producer (K, V)
       if (lane == 0) {
         int issued_k = 0, issued_v = 0;
-        for (int j = 0; j < nk; ++j) {
-          const int s = j % C::NS;
-          const uint32_t ph = uint32_t((j / C::NS) & 1);
+        const int n_live = live_count();
+        for (int it = 0, kt = next_live(0); it < n_live; ++it, kt = next_live(kt + 1)) {
+          const int s = it % C::NS;
+          const uint32_t ph = uint32_t((it / C::NS) & 1);
           if (!wait_bounded(BAR(K_EMPTY + s), ph ^ 1u, ctl)) break;
           mbar_arrive_expect_tx(BAR(K_FULL + s), C::TILE_BYTES);
 #pragma unroll
           for (int c = 0; c < C::NCH; ++c)
             tma_load_4d(sK + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmK, BAR(K_FULL + s),
-                        c * C::CH, j * C::BN, h, b);
-          issued_k = j + 1;
+                        c * C::CH, kt * C::BN, h, b);
+          issued_k = it + 1;
           if (!wait_bounded(BAR(V_EMPTY + s), ph ^ 1u, ctl)) break;
           mbar_arrive_expect_tx(BAR(V_FULL + s), C::TILE_BYTES);
 #pragma unroll
           for (int c = 0; c < C::NCH; ++c)
             tma_load_4d(sV + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &tmV, BAR(V_FULL + s),
-                        c * C::CH, j * C::BN, h, b);
-          issued_v = j + 1;
+                        c * C::CH, kt * C::BN, h, b);
+          issued_v = it + 1;
         }
         // every copy has landed before the CTA leaves (already true unless a
         // role aborted before consuming it)
@@ -606,9 +666,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mma_ts(d_tmem, p_tmem + uint32_t(kk * 8), adv(vd, uint32_t(kk * 16 * C::ROWB)), idesc_pv,
                    (acc || kk > 0) ? 1u : 0u);
         };
-        bool ok = wait_bounded(BAR(Q_FULL + 0), 0u, ctl) &&
-                  wait_bounded(BAR(Q_FULL + 1), 0u, ctl) && wait_bounded(BAR(K_FULL + 0), 0u, ctl);
-        if (ok) {
+        // n_live counts key tiles in issue order (all of them unless tiles of
+        // -inf padding are skipped); no live tile: no MMA, O_FULL at once
+        const int n_live = live_count();
+        bool ok = wait_bounded(BAR(Q_FULL + 0), 0u, ctl) && wait_bounded(BAR(Q_FULL + 1), 0u, ctl) &&
+                  (n_live == 0 || wait_bounded(BAR(K_FULL + 0), 0u, ctl));
+        if (ok && n_live > 0) {
           tc_fence_after();
           issue_qk(tS0, qd0, kd0);
           tc_commit(BAR(S_FULL + 0));
@@ -616,10 +679,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tc_commit(BAR(S_FULL + 1));
           tc_commit(BAR(K_EMPTY + 0));
         }
-        for (int j = 0; ok && j < nk; ++j) {
+        for (int j = 0; ok && j < n_live; ++j) {
           const int s = j % C::NS;
           const uint32_t ph = uint32_t((j / C::NS) & 1);
-          const bool more = (j + 1 < nk);
+          const bool more = (j + 1 < n_live);
           const int s1 = (j + 1) % C::NS;
           const uint32_t ph1 = uint32_t(((j + 1) / C::NS) & 1);
           if (!(ok = wait_bounded(BAR(V_FULL + s), ph, ctl))) break;

@@ -169,6 +169,39 @@ def test_kept_mask_variants_ragged_tail_and_max_jumps(D, kind):
             assert torch.equal(out, o2)
 
 
+@pytest.mark.parametrize("D", [96, 128])
+@pytest.mark.parametrize("bias_kind", [None, "bf16", "f32"])
+def test_key_tiles_of_padding_are_skipped_exactly(D, bias_kind):
+    """Key tiles whose pad is -inf throughout carry exactly zero weight and are
+    skipped: dead tiles first, in the middle and last (the ragged one), with
+    live tiles between them; garbage in the dead tiles' values must not leak,
+    and the result must match the oracle."""
+    B, H, N, kr = 1, 2, 1000, 140          # 8 key tiles, the last one ragged (104 keys)
+    q, k, v = _qkv(B, H, N, N, D, seed=2000 + D)
+    idx = _rand_idx(N, kr, seed=2001)
+    pad = torch.zeros(B, N)
+    for t0 in (0, 2, 3):
+        pad[:, t0 * 128:(t0 + 1) * 128] = float("-inf")
+    pad[:, 896:] = float("-inf")           # the ragged last tile, all of it
+    pad[:, 5 * 128 + 7:5 * 128 + 40] = float("-inf")   # a partly padded live tile
+    bias = None
+    if bias_kind is not None:
+        g = _gen(2002)
+        bias = torch.randn(B, 1, N, N, generator=g)
+        if bias_kind == "bf16":
+            bias = bias.to(BF)
+    dv = lambda t: None if t is None else t.to(DEV)
+    out = run(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), pad=dv(pad), bias=dv(bias))
+    for h in range(H):
+        ref = oracle_rows(q, k, v, idx.numpy(), 0, h, pad=pad, bias=bias)
+        check_attn(f64(out[0, h]), ref, f"D={D} bias={bias_kind} h{h}")
+    vg = v.clone()
+    dead = torch.isinf(pad[0])
+    vg[:, :, dead] = 1e4
+    o2 = run(q.to(DEV), k.to(DEV), vg.to(DEV), idx.to(DEV), pad=dv(pad), bias=dv(bias))
+    assert torch.equal(out, o2)
+
+
 def test_row_constant_mask_elision_is_invisible():
     """A row-constant additive bias (removable by the criterion) changes the
     GPU result only by rounding."""
