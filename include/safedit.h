@@ -183,9 +183,13 @@ safedit_status safedit_mask_is_row_constant(const safedit_tensor *mask,
  * d_idx [n_idx] i32 in [0, Nq) and unique, or NULL (then n_rows = Nq and
  *   n_idx is ignored).  Out-of-range indices set SAFEDIT_ERR_INDEX and the
  *   row is skipped.
- * key_pad (nullable) [B, Nk] f32, additive (0 or -inf for kept text padding).
+ * key_pad (nullable) [B, Nk] f32, additive (0 or -inf for kept text padding);
+ *   inner stride 1, batch stride a multiple of 4 elements, data 16-byte
+ *   aligned.  Key tiles of 128 keys whose pad is -inf throughout carry exactly
+ *   zero weight and are not computed (an exact shortcut).
  * bias (nullable) [B, 1|H, Nq, Nk] f32 or bf16, additive, a kept non-uniform
- *   bias; inner stride 1, row stride a multiple of 8 elements.
+ *   bias; inner stride 1, every other stride a multiple of 16 bytes (4 f32 or
+ *   8 bf16 elements), data 16-byte aligned.
  * scale: 0 selects 1/sqrt(d).
  * out: out_scattered == 0 -> [B,H,n_rows,d] compact (row r at r);
  *      out_scattered == 1 -> [B,H,Nq,d] state, row r written at index i
