@@ -371,6 +371,18 @@ def measure_extensions(tr, stream, dev, unfused_pcsp_ms, reps=5):
                                                                                       stream)), 4),
                           "note": f"[1,1,{wl.STRESS.N},{wl.STRESS.N}] bf16 all-zero mask (removable: read fully)"}
     del mask
+    # SRSU with kept masks at the stress shape: time per call and slowdown
+    # against the same launch with the mask elided
+    cases, flop = stress_srsu_cases(sd, dev, stream)
+    ms = {name: best_ms(fn) for name, fn in cases.items()}
+    base = ms["srsu_mask_elided"]
+    out["kept_mask_stress"] = {
+        name: {"ms": round(t, 4), "tflops": round(flop / (t * 1e-3) / 1e12, 1), "vs_elided": round(t / base, 3)}
+        for name, t in ms.items()}
+    out["kept_mask_stress"]["workload"] = (
+        f"B=1, H=32, N={wl.STRESS.N}, d=128, |S|={wl.STRESS.k} (blob scores); padding = trailing 1/8 of the keys "
+        "at -inf; bias = [1,1,N,N] N(0,1) in bf16 or f32")
+    del cases
     out["workload"] = (f"B={B}, |S|={k} focus rows per batch, D={D}, F={F}; "
                        "synthetic weights N(0,1)/sqrt(fan_in)")
     if sd.safedit_get_device_status(stream) != 0:
@@ -661,6 +673,33 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def stress_srsu_cases(sd, dev, stream):
+    """The SRSU launches of the mask-stress workload (B=1, H=32, N=16384,
+    d=128, |S|=4915 from the clustered blob scores): mask elided (no mask
+    input), kept text-padding key mask (trailing 1/8 of the keys -inf), kept
+    non-uniform bias [1,1,N,N] in bf16, both, and the bias in f32.  Returns
+    the launch closures (name -> fn) and the flop of one call."""
+    w = wl.STRESS
+    q, k, v = wl.qkv(w, device=dev)
+    o = torch.zeros_like(q)
+    score = wl.blob_scores(w, device=dev).contiguous()
+    idx = torch.empty(w.k, dtype=torch.int32, device=dev)
+    sd.safedit_partition_finalize(score, w.N, w.k, idx, None, None, stream)
+    pad = torch.zeros(1, w.N, device=dev)
+    pad[:, w.N - w.N // 8:] = float("-inf")
+    bias = wl.mask(w, "bias", device=dev)            # [1,1,N,N] bf16
+    bias32 = bias.float()                            # the same bias in f32 (1.07 GB)
+    att = lambda kp, bb: (lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, kp, bb, 0.0, o, 1, stream))
+    cases = {
+        "srsu_mask_elided": att(None, None),
+        "srsu_kept_padding": att(pad, None),
+        "srsu_kept_bias": att(None, bias),
+        "srsu_kept_padding_and_bias": att(pad, bias),
+        "srsu_kept_bias_f32": att(None, bias32),
+    }
+    return cases, 4.0 * w.k * w.N * w.d * w.B * w.H
+
+
 def run_stress(args):
     """The mask-path stress workload (B=1, H=32, N=16384, d=128, |S|=4915 from
     the clustered blob scores): SRSU attention with the mask elided (no mask
@@ -675,19 +714,10 @@ def run_stress(args):
     w = wl.STRESS
     _, bf16_burst, _, src = _peaks()
     stream = torch.cuda.Stream(device=dev)
-    q, k, v = wl.qkv(w, device=dev)
-    o = torch.zeros_like(q)
-    score = wl.blob_scores(w, device=dev).contiguous()
-    idx = torch.empty(w.k, dtype=torch.int32, device=dev)
-    sd.safedit_partition_finalize(score, w.N, w.k, idx, None, None, stream)
-    pad = torch.zeros(1, w.N, device=dev)
-    pad[:, w.N - w.N // 8:] = float("-inf")
-    bias = wl.mask(w, "bias", device=dev)            # [1,1,N,N] bf16
-    bias32 = bias.float()                            # the same bias in f32 (1.07 GB)
+    cases, flop = stress_srsu_cases(sd, dev, stream)
     zero = wl.mask(w, "zero", device=dev)
     padmask = wl.mask(w, "textpad", device=dev)
     verdict = torch.zeros(1, dtype=torch.int32, device=dev)
-    flop = 4.0 * w.k * w.N * w.d * w.B * w.H
 
     def best(fn):
         times = []
@@ -702,14 +732,6 @@ def run_stress(args):
         stream.synchronize()
         return min(a.elapsed_time(b) for a, b in times[1:])
 
-    cases = {
-        "srsu_mask_elided": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, None, None, 0.0, o, 1, stream),
-        "srsu_kept_padding": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, pad, None, 0.0, o, 1, stream),
-        "srsu_kept_bias": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, None, bias, 0.0, o, 1, stream),
-        "srsu_kept_padding_and_bias": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, pad, bias, 0.0, o, 1,
-                                                                     stream),
-        "srsu_kept_bias_f32": lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, None, bias32, 0.0, o, 1, stream),
-    }
     base = None
     for name, fn in cases.items():
         ms = best(fn)
