@@ -18,6 +18,7 @@ Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|referenc
 """
 import argparse
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -406,19 +407,27 @@ def whole_job_tflops(flop_per_rank, n_ranks, max_ms):
     return flop_per_rank * n_ranks / (max_ms * 1e-3) / 1e12
 
 
+def _code_sha(path):
+    """sha256 prefix of a C/CUDA source with its comments and whitespace
+    removed: equal for two versions that differ only in comments."""
+    import hashlib
+    with open(path) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return hashlib.sha256(" ".join(src.split()).encode()).hexdigest()[:16]
+
+
 def _ncu_traffic():
     """DRAM bytes per SRSU launch (dram__bytes_read.sum + dram__bytes_write.sum)
-    from the committed ncu summary, or None when the kernel source changed
-    since those counters were taken."""
-    import hashlib
+    from the committed ncu summary, or None when the kernel's code changed
+    since those counters were taken (comment-only edits do not count)."""
     p = os.path.join(ROOT, "profiles", "attn_subset_srsu_2560.traffic.json")
     src = os.path.join(ROOT, "spatially_adaptive_dit_b200", "csrc", "attn.cu")
     try:
         with open(p) as f:
             d = json.load(f)
-        with open(src, "rb") as f:
-            cur = hashlib.sha256(f.read()).hexdigest()[:16]
-        return d.get("bytes_per_launch") if d.get("attn_cu_sha256_16") == cur else None
+        return d.get("bytes_per_launch") if d.get("attn_cu_code_sha256_16") == _code_sha(src) else None
     except Exception:
         return None
 

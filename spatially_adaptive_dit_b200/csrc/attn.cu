@@ -28,6 +28,11 @@
 //     2^8, which is exact after the final division by the row sum); packed
 //     f32x2 FMAs and adds, three-input max; a quarter of the exponentials on
 //     the FMA pipe (degree-3 polynomial), the rest on the MUFU unit.
+//   * kept masks (template PAD / BIAS): logits scale s + pad + bias in one
+//     packed FMA per pair; the pad one key tile ahead in a shared three-slot
+//     ring, the bias one pass ahead through per-warp cp.async staging; each
+//     key tile in passes of 64 (f32 bias: 32) columns; key tiles whose pad is
+//     -inf throughout are skipped by every role; every exponential on MUFU.
 // Every mbarrier wait is bounded; an expired wait raises the CTA's abort
 // flag, drains in-flight TMA loads and MMAs, frees TMEM and returns.
 #include <cmath>
