@@ -202,6 +202,24 @@ def test_key_tiles_of_padding_are_skipped_exactly(D, bias_kind):
     assert torch.equal(out, o2)
 
 
+@pytest.mark.parametrize("N", [1024 * 128, 1026 * 128 - 56])
+def test_key_tile_skipping_at_its_capacity(N):
+    """The live-tile bitmask covers up to 1024 key tiles: at exactly 1024
+    tiles the skipping runs with every bitmask word in use (dead tiles first,
+    in the middle and last); past that every tile is processed, and the result
+    must be the same."""
+    B, H, D, kr = 1, 1, 64, 64
+    q, k, v = _qkv(B, H, 512, N, D, seed=3000)
+    idx = _rand_idx(512, kr, seed=3001)
+    nk = (N + 127) // 128
+    pad = torch.zeros(B, N)
+    for t0 in (0, 500, nk - 1):
+        pad[:, t0 * 128:min(N, (t0 + 1) * 128)] = float("-inf")
+    out = run(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), pad=pad.to(DEV))
+    ref = oracle_rows(q, k, v, idx.numpy(), 0, 0, pad=pad)
+    check_attn(f64(out[0, 0]), ref, f"N={N}")
+
+
 def test_row_constant_mask_elision_is_invisible():
     """A row-constant additive bias (removable by the criterion) changes the
     GPU result only by rounding."""
