@@ -91,6 +91,18 @@ def test_attn_host_validation(sd):
     assert call(R(q), R(k), R(v), None, 0, R(pad), None, 0.0, R(o), 0, None) == sd.ERR_SHAPE
     bias = _desc(sd, (1, 1, 256, 256), (65536, 65536, 256, 1), sd.F16)
     assert call(R(q), R(k), R(v), None, 0, None, R(bias), 0.0, R(o), 0, None) == sd.ERR_DTYPE
+    # key pad: batch stride not a 16-byte multiple, inner stride not 1, misaligned data
+    for strides, ptr in (((258, 1), 0x1000), ((512, 2), 0x1000), ((256, 1), 0x1008)):
+        padb = _desc(sd, (1, 256), strides, sd.F32, ptr=ptr)
+        assert call(R(q), R(k), R(v), None, 0, R(padb), None, 0.0, R(o), 0, None) == sd.ERR_ALIGNMENT
+    # bias: a bf16 row stride that is not a multiple of 8 elements (an f32 one
+    # of 4 would pass), a head dim that is neither 1 nor H, a row count not Nq
+    bias_s = _desc(sd, (1, 1, 256, 256), (260 * 256, 260 * 256, 260, 1), sd.BF16)
+    assert call(R(q), R(k), R(v), None, 0, None, R(bias_s), 0.0, R(o), 0, None) == sd.ERR_ALIGNMENT
+    bias_h = _desc(sd, (1, 3, 256, 256), (3 * 65536, 65536, 256, 1), sd.BF16)
+    assert call(R(q), R(k), R(v), None, 0, None, R(bias_h), 0.0, R(o), 0, None) == sd.ERR_SHAPE
+    bias_r = _desc(sd, (1, 1, 200, 256), (51200, 51200, 256, 1), sd.F32)
+    assert call(R(q), R(k), R(v), None, 0, None, R(bias_r), 0.0, R(o), 0, None) == sd.ERR_SHAPE
 
 
 def test_bandwidth_kernels_host_validation(sd):
