@@ -1,8 +1,10 @@
 /* A plain C client of libsafedit.so (include/safedit.h), with no Python in
  * the loop: device memory from the CUDA runtime, seeded inputs from a small
  * LCG, one SRSU subset-attention call (gathered rows over all keys, output
- * scattered into a state), one row-constant mask check and one SW-CFG call,
- * each compared with the fp64 oracle (test infrastructure, liboracle.so).
+ * scattered into a state), the same rows with kept masks (key padding and an
+ * f32 bias, compact output), one row-constant mask check and one SW-CFG
+ * call, each compared with the fp64 oracle (test infrastructure,
+ * liboracle.so).
  *
  *   abi_client          run the checks on the current CUDA device (exit 0 = pass)
  *   abi_client --abi    only the host-side argument checks (no GPU needed)
@@ -163,6 +165,53 @@ int main(int argc, char **argv) {
   printf("attn_subset: relFro %.3e  max|err| %.3e  untouched rows %s\n", rel, mx,
          kept ? "ok" : "CHANGED");
   if (!(rel <= 5e-3 && mx <= 2e-2 && kept)) return 6;
+
+  /* the same rows with kept masks, compact output: a key-padding vector (key
+   * tile 2 -inf throughout, so it is skipped, plus scattered -inf keys) and a
+   * dense f32 bias [1,1,N,N] */
+  float *hpad = malloc((size_t)N * 4), *hbias = malloc((size_t)(N * N) * 4);
+  double *pad64 = malloc((size_t)N * 8), *brows = malloc((size_t)(n_idx * N) * 8);
+  double *ref2 = malloc((size_t)(n_idx * d) * 8);
+  uint16_t *ho2 = malloc((size_t)(n_idx * d) * 2);
+  if (!hpad || !hbias || !pad64 || !brows || !ref2 || !ho2) return 2;
+  for (int64_t j = 0; j < N; ++j) {
+    hpad[j] = ((j >= 256 && j < 384) || j % 11 == 5) ? -INFINITY : 0.f;
+    pad64[j] = hpad[j];
+  }
+  for (int64_t i = 0; i < N * N; ++i) hbias[i] = (float)(0.5 * normal01());
+  for (int64_t r = 0; r < n_idx; ++r)
+    for (int64_t j = 0; j < N; ++j) brows[r * N + j] = hbias[(int64_t)idx[r] * N + j];
+  void *dpad, *dbias, *dout2;
+  CHECK_CUDA(cudaMalloc(&dpad, (size_t)N * 4));
+  CHECK_CUDA(cudaMalloc(&dbias, (size_t)(N * N) * 4));
+  CHECK_CUDA(cudaMalloc(&dout2, (size_t)(n_idx * d) * 2));
+  CHECK_CUDA(cudaMemcpy(dpad, hpad, (size_t)N * 4, cudaMemcpyHostToDevice));
+  CHECK_CUDA(cudaMemcpy(dbias, hbias, (size_t)(N * N) * 4, cudaMemcpyHostToDevice));
+  safedit_tensor tpad;
+  memset(&tpad, 0, sizeof tpad);
+  tpad.data = dpad, tpad.dtype = SAFEDIT_F32, tpad.ndim = 2;
+  tpad.dims[0] = 1, tpad.dims[1] = N, tpad.strides[0] = N, tpad.strides[1] = 1;
+  safedit_tensor tbias = tensor4(dbias, SAFEDIT_F32, 1, 1, N, N);
+  safedit_tensor to2 = tensor4(dout2, SAFEDIT_BF16, 1, 1, n_idx, d);
+  CHECK_SD(safedit_attn_subset(&tq, &tk, &tv, (const int32_t *)didx, (int32_t)n_idx, &tpad, &tbias,
+                               0.f, &to2, 0, NULL));
+  CHECK_SD(safedit_get_device_status(&status, NULL));
+  if (status != SAFEDIT_OK) {
+    fprintf(stderr, "device status %s\n", safedit_status_string((safedit_status)status));
+    return 4;
+  }
+  CHECK_CUDA(cudaMemcpy(ho2, dout2, (size_t)(n_idx * d) * 2, cudaMemcpyDeviceToHost));
+  if (oracle_attn_subset(N, N, d, q, k, v, idx, n_idx, pad64, brows, 1.0 / sqrt((double)d), ref2) != 0)
+    return 5;
+  num = 0.0, den = 0.0, mx = 0.0;
+  for (int64_t i = 0; i < n_idx * d; ++i) {
+    const double g = from_bf16(ho2[i]), e = ref2[i];
+    num += (g - e) * (g - e), den += e * e;
+    if (fabs(g - e) > mx) mx = fabs(g - e);
+  }
+  const double rel2 = sqrt(num / den);
+  printf("attn_subset with kept masks: relFro %.3e  max|err| %.3e\n", rel2, mx);
+  if (!(rel2 <= 5e-3 && mx <= 2e-2)) return 10;
 
   /* mask check: a per-row constant additive mask [1,1,64,256] f32 is removable */
   const int64_t mq = 64, mk = 256;

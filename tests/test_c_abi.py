@@ -1,8 +1,9 @@
 """The C ABI used from plain C, without Python in the loop: tests/c_abi/abi_client.c
 is compiled with gcc against include/safedit.h and linked with libsafedit.so,
 the CUDA runtime and the oracle library (test infrastructure).  On the CPU it
-runs the host-side argument checks; on a GPU it also runs one SRSU attention,
-one mask check and one SW-CFG call against the oracle."""
+runs the host-side argument checks; on a GPU it also runs one SRSU attention
+(without and with kept masks), one mask check and one SW-CFG call against the
+oracle."""
 import os
 import subprocess
 
