@@ -280,21 +280,32 @@ def test_config_2560_srsu_launch_as_benchmarked():
         check_attn(f64(got), ref, f"b{b}h{h}")
 
 
-def test_config_stress_kept_masks_sampled():
+@pytest.mark.parametrize("kind", ["pad", "bias_bf16", "pad+bias_bf16", "bias_f32"])
+def test_config_stress_kept_masks_sampled(kind):
+    """The mask-stress shape in the launch configuration the benchmark times
+    (blob-score rows scattered into the state), for every kept-mask variant;
+    sampled rows of two heads against the oracle."""
     w = wl.STRESS
     q, k, v = wl.qkv(w, device=DEV)
     score = wl.blob_scores(w).to(DEV)
     idx = torch.empty(w.k, dtype=torch.int32, device=DEV)
     sd().safedit_partition_finalize(score, w.N, w.k, idx, None, None)
-    pad = torch.zeros(1, w.N, device=DEV)
-    pad[:, w.N - w.N // 8:] = float("-inf")   # text-padding style key mask (kept)
-    bias = wl.mask(w, "bias", device=DEV)     # non-uniform bias (kept), [1,1,N,N] bf16
-    out = run(q, k, v, idx, pad=pad, bias=bias)
+    pad = bias = None
+    if kind.startswith("pad"):
+        pad = torch.zeros(1, w.N, device=DEV)
+        pad[:, w.N - w.N // 8:] = float("-inf")   # text-padding style key mask (kept)
+    if "bias" in kind:
+        bias = wl.mask(w, "bias", device=DEV)     # non-uniform bias (kept), [1,1,N,N] bf16
+        if kind.endswith("f32"):
+            bias = bias.float()
+    state = torch.zeros(w.B, w.H, w.N, w.d, dtype=BF, device=DEV)
+    run(q, k, v, idx, pad=pad, bias=bias, out=state, scattered=True)
     rows = np.linspace(0, w.k - 1, 24).astype(np.int64)
     ic = idx.cpu().numpy()
     for h in (0, 31):
         ref = oracle_rows(q, k, v, ic, 0, h, rows=rows, pad=pad, bias=bias)
-        check_attn(f64(out[0, h, torch.as_tensor(rows, device=DEV)]), ref, f"h{h}")
+        got = state[0, h, torch.as_tensor(ic[rows].astype(np.int64), device=DEV)]
+        check_attn(f64(got), ref, f"{kind} h{h}")
 
 
 def test_3072_sweep_sampled():
