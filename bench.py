@@ -113,22 +113,46 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-class Trajectory:
-    """Device-resident buffers and the launch sequence of one trajectory."""
+def head_range(H, world, rank):
+    """Heads [h0, h1) of rank `rank` when one generation's H heads are split
+    evenly over `world` GPUs."""
+    if H % world != 0:
+        raise ValueError(f"{H} heads do not split evenly over {world} GPUs")
+    n = H // world
+    return rank * n, (rank + 1) * n
 
-    def __init__(self, w, dev, seed_step=0):
+
+def score_all_reduce(score):
+    """The one exchange of a head-sharded generation: the fp64 PCSP score
+    vector (each rank's sum over its own heads) summed over all ranks, so
+    that every rank makes the identical S/C split."""
+    torch.distributed.all_reduce(score, op=torch.distributed.ReduceOp.SUM)
+
+
+class Trajectory:
+    """Device-resident buffers and the launch sequence of one trajectory.
+    heads=(h0, h1) keeps only those heads of the (same, globally seeded)
+    generation on this device; reduce_score then completes the PCSP score
+    over the other devices' heads before the split."""
+
+    def __init__(self, w, dev, seed_step=0, heads=None, reduce_score=None):
         from spatially_adaptive_dit_b200 import safedit as sd
         self.sd, self.w, self.dev = sd, w, dev
-        B, H, N, d, L, k = w.B, w.H, w.N, w.d, w.L, w.k
+        B, N, d, L, k = w.B, w.N, w.d, w.L, w.k
+        h0, h1 = (0, w.H) if heads is None else heads
+        H = h1 - h0
+        sl = (lambda t: t) if heads is None else (lambda t: t[:, h0:h1].contiguous())
+        self.reduce_score = reduce_score
         self.k = k
-        self.q, self.k_full, self.v_full = wl.qkv(w, step=seed_step, device=dev)
-        self.k_s, self.v_s = wl.fresh_sensitive_kv(w, k, step=seed_step, device=dev)
+        self.q, self.k_full, self.v_full = (sl(t) for t in wl.qkv(w, step=seed_step, device=dev))
+        self.k_s, self.v_s = (sl(t) for t in wl.fresh_sensitive_kv(w, k, step=seed_step, device=dev))
         self.k_state = torch.empty_like(self.k_full)
         self.v_state = torch.empty_like(self.v_full)
         self.k_state.copy_(self.k_full)
         self.v_state.copy_(self.v_full)
         self.o_state = torch.zeros_like(self.q)
         self.q_img, self.k_txt, self.valid, self.content = wl.text(w, step=seed_step, device=dev)
+        self.q_img, self.k_txt = sl(self.q_img), sl(self.k_txt)
         self.P = torch.empty(H, N, L, device=dev)
         self.score = torch.zeros(N, dtype=torch.float64, device=dev)
         self.idx_s = torch.empty(k, dtype=torch.int32, device=dev)
@@ -174,6 +198,8 @@ class Trajectory:
                     self.q_img, self.k_txt, self.valid, 0, 0.0, self.P, stream))
                 timed("partition_accumulate", lambda: sd.safedit_partition_accumulate(
                     self.P, self.content, self.score, stream))
+            if t == w.warmup - 1 and self.reduce_score is not None:
+                timed("score_all_reduce", lambda: self.reduce_score(self.score))
             if t == w.warmup - 1:
                 timed("partition_finalize", lambda: sd.safedit_partition_finalize(
                     self.score, w.N, self.k, self.idx_s, self.idx_c, self.s, stream))
@@ -207,7 +233,11 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     from spatially_adaptive_dit_b200 import safedit as sd
-    tr = Trajectory(W, dev, seed_step=1000 * rank)
+    sharded = args.shard == "heads" and ws > 1
+    if sharded:  # one generation, H / ws heads per GPU, one score all-reduce
+        tr = Trajectory(W, dev, seed_step=0, heads=head_range(W.H, ws, rank), reduce_score=score_all_reduce)
+    else:  # independent replicas
+        tr = Trajectory(W, dev, seed_step=1000 * rank)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
@@ -272,10 +302,12 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": WORKLOAD, "global_batch": W.B * ws, "seq_len": W.N,
-                       "parallelism": f"replicas x{ws} (independent trajectories, no collective)",
+            "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": W.B if sharded else W.B * ws, "seq_len": W.N,
+                       "parallelism": (f"heads x{ws} (one generation, {W.H // ws} heads per GPU; one all-reduce "
+                                       "of the fp64 score vector after the warm-up)") if sharded else
+                                      f"replicas x{ws} (independent trajectories, no collective)",
                        "l2": "inputs larger than L2 (Q/K/V/state 236 MB each), no flush needed",
                        "srsu_calls_per_step": n_srsu // args.steps,
                        "srsu_ms_per_call": round(srsu_call_ms, 4)},
@@ -524,6 +556,8 @@ def run_e2e(tr, stream, args):
                     ev = torch.cuda.Event()
                     ev.record(stream)
                     text_freed[0] = ev
+                if t == w.warmup - 1 and tr.reduce_score is not None:
+                    tr.reduce_score(tr.score)
                 if t == w.warmup - 1:
                     sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s, stream)
                 if t == 0:
@@ -909,6 +943,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: independent replicas (default, weak scaling) or one generation split by heads "
+                         "(strong scaling; the PCSP score is all-reduced once)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,

@@ -55,3 +55,55 @@ def test_two_gloo_ranks_reduce_max_and_independent_replicas():
     import bench
     # 2 replicas of 1 TFLOP each in a slowest-rank time of 1 s -> 2 TFLOP/s
     assert abs(bench.whole_job_tflops(1e12, 2, 1000.0) - 2.0) < 1e-12
+
+
+def _heads_rank(rank, world, port, out):
+    """One rank of a head-sharded generation: its share of the PCSP score,
+    the benchmark's all-reduce, then the split."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    import numpy as np
+    import bench
+    import oracle
+    H, N, L, k = 8, 96, 16, 29
+    g = torch.Generator()
+    g.manual_seed(7)
+    P = torch.rand(H, N, L, generator=g)       # the same probabilities on every rank
+    content = torch.zeros(L, dtype=torch.uint8)
+    content[1:L - 1] = 1
+    h0, h1 = bench.head_range(H, world, rank)
+    score = torch.from_numpy(np.ascontiguousarray(oracle.partition_accumulate(P[h0:h1], content)))
+    bench.score_all_reduce(score)
+    full = oracle.partition_accumulate(P, content)
+    err = float(np.abs(score.numpy() - full).max() / np.abs(full).max())
+    idx_rank = oracle.partition_select(score.numpy(), k)[0].tolist()
+    idx_full = oracle.partition_select(full, k)[0].tolist()
+    dist.barrier()
+    out[rank] = (err, idx_rank, idx_full, (h0, h1))
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_two_gloo_ranks_head_sharded_split_matches_one_process():
+    """Head sharding of one generation: each rank sums the score over its own
+    heads, one all-reduce completes it, and every rank then makes the same
+    S/C split as a single process over all heads."""
+    import bench
+    assert [bench.head_range(24, 8, r) for r in (0, 7)] == [(0, 3), (21, 24)]
+    with pytest.raises(ValueError):
+        bench.head_range(24, 16, 0)
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_heads_rank, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+        res = dict(out)
+    assert res[0][3] == (0, 4) and res[1][3] == (4, 8)
+    for r in range(world):
+        err, idx_rank, idx_full, _ = res[r]
+        assert err <= 1e-14
+        assert idx_rank == idx_full
+    assert res[0][1] == res[1][1]
