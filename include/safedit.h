@@ -182,7 +182,10 @@ safedit_status safedit_mask_is_row_constant(const safedit_tensor *mask,
  * q [B,H,Nq,d] bf16; k, v [B,H,Nk,d] bf16; d in {64, 96, 128}.
  * d_idx [n_idx] i32 in [0, Nq) and unique, or NULL (then n_rows = Nq and
  *   n_idx is ignored).  Out-of-range indices set SAFEDIT_ERR_INDEX and the
- *   row is skipped.
+ *   row is skipped.  Uniqueness is the caller's contract (the split of
+ *   safedit_partition_finalize is unique by construction); with
+ *   out_scattered == 1 and the debug index check on, a duplicate sets
+ *   SAFEDIT_ERR_INDEX (see safedit_debug_set_index_check).
  * key_pad (nullable) [B, Nk] f32, additive (0 or -inf for kept text padding);
  *   inner stride 1, batch stride a multiple of 4 elements, data 16-byte
  *   aligned.  Key tiles of 128 keys whose pad is -inf throughout carry exactly
@@ -212,8 +215,10 @@ safedit_status safedit_attn_subset(const safedit_tensor *q,
  * For t < n_tensors: dst[t][b,h,d_idx[r],:] = src[t][b,h,r,:], r < n_idx.
  * src[t] [B,H,n_idx,d], dst[t] [B,H,N,d], same dtype (any 2- or 4-byte
  * type), same B, H, d per pair; d*elt % 16 == 0.  1 <= n_tensors <= 4, one
- * launch for all.  d_idx must be unique (not checked); out-of-range entries
- * set SAFEDIT_ERR_INDEX and are skipped.  Other rows are untouched.
+ * launch for all.  d_idx must be unique: two equal entries would race for
+ * one row (checked only in the debug index-check mode, where a duplicate
+ * sets SAFEDIT_ERR_INDEX); out-of-range entries set SAFEDIT_ERR_INDEX and
+ * are skipped.  Other rows are untouched.
  */
 safedit_status safedit_scatter_state(const safedit_tensor *src,
                                      const safedit_tensor *dst,
@@ -231,8 +236,10 @@ safedit_status safedit_gather_rows(const safedit_tensor *src,
  *   gamma_i = gamma_ctx + (gamma_sens - gamma_ctx) * s_i,
  * applied to the prediction after the forward pass; [P3 B.2] spatial CFG.
  *   out[i,f] = eps_u[i,f] + gamma_i * (eps_c[i,f] - eps_u[i,f])   (f32 FMA)
- * eps_c, eps_u, out [N, F] f32 with inner stride 1 (out may alias either
- * input).  d_s [N] f32.  gamma_ctx == gamma_sens gives plain CFG (SAFE-Core).
+ * eps_c, eps_u [N, F] f32, or both bf16 (widened exactly to f32), with
+ * inner stride 1; out [N, F] f32, inner stride 1 (with f32 inputs out may
+ * alias either input; with bf16 inputs it must not overlap them).  d_s [N]
+ * f32.  gamma_ctx == gamma_sens gives plain CFG (SAFE-Core).
  */
 safedit_status safedit_sw_cfg(const safedit_tensor *eps_c,
                               const safedit_tensor *eps_u, const float *d_s,
@@ -275,7 +282,8 @@ safedit_status safedit_stepcache_sw_cfg(const safedit_tensor *eps_c_a,
  * d_idx_out M_out must equal M.  N must be a multiple of 8.  d_bias: NULL or
  * N f32 on the device.  act: 0 identity, 1 GELU (tanh form, fp32).
  * Accumulation is fp32 over all of K (tensor cores), rounded to bf16 once.
- * d_idx_out: NULL or M int32 on the device, unique (not checked); an entry
+ * d_idx_out: NULL or M int32 on the device, unique (checked only in the
+ * debug index-check mode, where a duplicate sets SAFEDIT_ERR_INDEX); an entry
  * outside [0, M_out) sets SAFEDIT_ERR_INDEX on the device status word and
  * that row is skipped.  Rows of out that no r maps to are untouched.
  * M == 0 or N == 0 is a no-op; K == 0 is SAFEDIT_ERR_SHAPE.
@@ -287,9 +295,12 @@ safedit_status safedit_gemm_bias_act(const safedit_tensor *a,
                                      const safedit_tensor *out, void *stream);
 
 /* ------------------------------------------------------------------------
- * Device status word: waits for `stream`, copies the word of the current
- * device into *host_status (a safedit_status value, SAFEDIT_OK if nothing
- * was flagged since the last read) and clears it.
+ * Device status word: on `stream`, takes the word of the current device out
+ * and clears it in one atomic step (a one-thread kernel), then waits for the
+ * stream and stores it in *host_status (a safedit_status value, SAFEDIT_OK if
+ * nothing was flagged since the last read).  An error that a kernel on
+ * another stream records meanwhile is either returned by this call or kept
+ * for the next one.
  */
 safedit_status safedit_get_device_status(int32_t *host_status, void *stream);
 
@@ -304,6 +315,16 @@ uint64_t safedit_kernel_launch_count(void);
  * already satisfied give up, which exercises the SAFEDIT_ERR_TIMEOUT path
  * without a real hang.  Returns the previous value. */
 uint64_t safedit_debug_set_wait_limit_ns(uint64_t ns);
+
+/* Debug knob: with `on` non-zero, every call that writes rows through an
+ * index vector (safedit_scatter_state, safedit_attn_subset with
+ * out_scattered == 1, safedit_gemm_bias_act with d_idx_out) first launches a
+ * check of that vector on the same stream: an entry out of range or equal to
+ * an earlier one sets SAFEDIT_ERR_INDEX in the device status word (the
+ * scattering kernel still runs; its output is then unspecified).  The check
+ * is one CTA with a bitmap of the row range in shared memory and allocates
+ * nothing.  Off by default.  Returns the previous setting. */
+int32_t safedit_debug_set_index_check(int32_t on);
 
 #ifdef __cplusplus
 }

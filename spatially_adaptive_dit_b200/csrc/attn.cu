@@ -11,9 +11,9 @@
 //
 // Design (one CTA per SM, 384 threads = 3 warpgroups):
 //   * 2 query tiles of 128 rows (256 rows per CTA).  The softmax warpgroup of
-//     tile t (warps 4t..4t+3) gathers its rows q[idx[r]] with 16-byte loads
-//     straight into the swizzled K-major shared-memory layout the tensor core
-//     reads (the indexed gather replaces a copy of Q_S).
+//     tile t (warps 4t..4t+3) gathers its rows q[idx[r]] with 16-byte
+//     cp.async copies straight into the swizzled K-major shared-memory layout
+//     the tensor core reads (the indexed gather replaces a copy of Q_S).
 //   * the third warpgroup: warp 8 streams K and V tiles (128 keys) through an
 //     NS-stage TMA ring, warp 9 issues tcgen05.mma, warps 10-11 only lend
 //     their registers (setmaxnreg: 208 per softmax thread, 88 per control
@@ -279,29 +279,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int wr = warp & 3;            // TMEM lane quarter
     const int tid = threadIdx.x & 127;  // thread within the warpgroup
     const int tile_row0 = row0 + t * 128;
-    // ---- indexed gather of the tile's query rows into swizzled smem
+    // ---- indexed gather of the tile's query rows: 16-byte cp.async copies
+    // (no register staging) straight into the swizzled K-major layout
     {
       const uint32_t qs = sQ + t * C::TILE_BYTES;
       const __nv_bfloat16* qbh = p.q + b * p.q_sb + h * p.q_sh;
+      constexpr int UPC = C::ROWB / 16;  // units per chunk row
       for (int u = tid; u < 128 * C::UNITS; u += 128) {
         const int rr = u / C::UNITS, cu = u - rr * C::UNITS;
         const int gr = tile_row0 + rr;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        const __nv_bfloat16* src = qbh;  // not read when nothing is copied (zero fill)
+        uint32_t bytes = 0u;
         if (gr < p.n_rows) {
           const int qi = p.idx ? __ldg(p.idx + gr) : gr;
-          if (qi >= 0 && qi < p.Nq)
-            val = __ldg(reinterpret_cast<const uint4*>(qbh + int64_t(qi) * p.q_sr) + cu);
-          else if (cu == 0)
+          if (qi >= 0 && qi < p.Nq) {
+            src = qbh + int64_t(qi) * p.q_sr + cu * 8;
+            bytes = 16u;
+          } else if (cu == 0) {
             set_status(p.status, SAFEDIT_ERR_INDEX);
+          }
         }
-        constexpr int UPC = C::ROWB / 16;  // units per chunk row
         const int chunk = cu / UPC, cin = cu - chunk * UPC;
         const uint32_t off = uint32_t(chunk * C::CHUNK_BYTES) +
                              swizzle_off(uint32_t(rr * C::ROWB + cin * 16), C::LAYOUT);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(qs + off), "r"(val.x),
-                     "r"(val.y), "r"(val.z), "r"(val.w)
-                     : "memory");
+        cp_async16(qs + off, src, bytes);
       }
+      cp_async_commit();
+      cp_async_wait_all();
       fence_proxy_async_smem();
       mbar_arrive(BAR(Q_FULL + t));
     }
@@ -856,6 +860,9 @@ extern "C" safedit_status safedit_attn_subset(const safedit_tensor* q, const saf
   p.status = status_ptr();
   if (!p.status) return SAFEDIT_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d_idx && out_scattered && index_check_enabled() &&
+      (st = launch_index_check(d_idx, static_cast<int32_t>(n_rows), Nq, p.status, s)) != SAFEDIT_OK)
+    return st;
   switch (D) {
     case 64: return dispatch_attn<64>(tmK, tmV, p, static_cast<int>(B), s);
     case 96: return dispatch_attn<96>(tmK, tmV, p, static_cast<int>(B), s);

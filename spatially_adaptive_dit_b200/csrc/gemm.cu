@@ -546,6 +546,9 @@ extern "C" safedit_status safedit_gemm_bias_act(const safedit_tensor* a, const s
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d_idx_out && index_check_enabled() &&
+      (st = launch_index_check(d_idx_out, static_cast<int32_t>(M), M_out, p.status, s)) != SAFEDIT_OK)
+    return st;
   if (pair) {
     if ((st = set_smem(reinterpret_cast<const void*>(gemm_bias_act_pair_kernel), kG2Smem)) !=
         SAFEDIT_OK)

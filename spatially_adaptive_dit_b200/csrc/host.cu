@@ -10,13 +10,21 @@
 #include "internal.h"
 
 // One status word per device: the first device-detected error since the last
-// safedit_get_device_status().  Static storage: the library allocates nothing.
+// safedit_get_device_status(), and the word that call takes out of it.
+// Static storage: the library allocates nothing.
 static __device__ int g_device_status;
+static __device__ int g_status_taken;
+
+// Reads and clears the status word in one atomic step, so that an error a
+// kernel on another stream records at the same moment is either returned
+// now or kept for the next read, never lost.
+__global__ void status_take_kernel() { g_status_taken = atomicExch(&g_device_status, 0); }
 
 namespace sd {
 
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<uint64_t> g_wait_limit{1000000000ull};
+static std::atomic<int32_t> g_index_check{0};
 
 constexpr int kMaxDevices = 64;
 static int* g_status_addr[kMaxDevices] = {nullptr};
@@ -40,6 +48,8 @@ safedit_status after_launch(int n) {
 }
 
 uint64_t wait_limit_ns() { return g_wait_limit.load(std::memory_order_relaxed); }
+
+bool index_check_enabled() { return g_index_check.load(std::memory_order_relaxed) != 0; }
 
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -88,14 +98,14 @@ extern "C" {
 
 safedit_status safedit_get_device_status(int32_t* host_status, void* stream) {
   if (!host_status) return SAFEDIT_ERR_INVALID_ARG;
-  int* p = sd::status_ptr();
-  if (!p) return SAFEDIT_ERR_CUDA;
+  if (!sd::status_ptr()) return SAFEDIT_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  status_take_kernel<<<1, 1, 0, s>>>();
+  if (sd::after_launch(1) != SAFEDIT_OK) return SAFEDIT_ERR_CUDA;
   int v = 0;
-  if (cudaMemcpyAsync(&v, p, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+  if (cudaMemcpyFromSymbolAsync(&v, g_status_taken, sizeof(int), 0, cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
     return SAFEDIT_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return SAFEDIT_ERR_CUDA;
-  if (cudaMemsetAsync(p, 0, sizeof(int), s) != cudaSuccess) return SAFEDIT_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return SAFEDIT_ERR_CUDA;
   *host_status = v;
   return SAFEDIT_OK;
@@ -120,5 +130,7 @@ const char* safedit_status_string(safedit_status st) {
 uint64_t safedit_kernel_launch_count(void) { return sd::g_launches.load(); }
 
 uint64_t safedit_debug_set_wait_limit_ns(uint64_t ns) { return sd::g_wait_limit.exchange(ns); }
+
+int32_t safedit_debug_set_index_check(int32_t on) { return sd::g_index_check.exchange(on ? 1 : 0); }
 
 }  // extern "C"

@@ -53,6 +53,17 @@ safedit_status after_launch(int n);
 
 uint64_t wait_limit_ns();
 
+// Debug mode (safedit_debug_set_index_check): index vectors that scatter
+// rows are checked for duplicates before the scattering kernel runs.
+bool index_check_enabled();
+
+// Launches the duplicate / range check of d_idx[0, n_idx) against
+// [0, n_rows): one CTA with a bitmap of the row range in shared memory
+// (windows of 1.8 M rows), a duplicate or out-of-range entry sets
+// SAFEDIT_ERR_INDEX in the status word.  Needs no memory beyond the CTA's.
+safedit_status launch_index_check(const int32_t* d_idx, int32_t n_idx, int64_t n_rows, int* status,
+                                  cudaStream_t stream);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda).  dims/box are innermost first; strides_bytes has rank-1
 // entries (dims 1..rank-1).

@@ -4,6 +4,9 @@
 //     [B,H,rows,d] tensors in one launch (SAFE-DiT summary, 방법론 3: cached
 //     context states, refreshed sensitive rows), 16-byte vector accesses,
 //     every row a contiguous run so that a warp touches whole lines;
+//   * the debug-mode index check: every entry of a scattering index vector
+//     in range and no two equal (a duplicate would make two writers race
+//     for one row);
 //   * sw_cfg: gamma_i = gamma_ctx + (gamma_sens - gamma_ctx) s_i and
 //     out = u + gamma_i (c - u) (SAFE-DiT summary, 방법론 4), one fp32 FMA
 //     chain per element on 128-bit loads.
@@ -88,6 +91,51 @@ __global__ void __launch_bounds__(kRowThreads) row_copy_kernel(RowCopyParams p) 
   }
 }
 
+// ------------------------------------------------------------ index check
+constexpr int kIdxThreads = 1024;
+constexpr int kIdxWords = 58112;  // 227 KB of bitmap: 1,859,584 rows per window
+
+// One CTA.  For each window of the row range: clear the bitmap, mark every
+// index in the window with an atomic OR (a bit already set is a duplicate),
+// repeat.  Out-of-range entries are flagged on the first window.
+__global__ void __launch_bounds__(kIdxThreads) index_check_kernel(const int32_t* idx, int32_t n_idx,
+                                                                   int64_t n_rows, int words,
+                                                                   int* status) {
+  extern __shared__ uint32_t bm[];
+  const int64_t span = int64_t(words) * 32;
+  for (int64_t base = 0; base < n_rows; base += span) {
+    for (int w = threadIdx.x; w < words; w += kIdxThreads) bm[w] = 0u;
+    __syncthreads();
+    bool bad = false;
+    for (int r = threadIdx.x; r < n_idx; r += kIdxThreads) {
+      const int64_t i = __ldg(idx + r);
+      if (i < 0 || i >= n_rows) {
+        bad |= (base == 0);
+        continue;
+      }
+      const int64_t off = i - base;
+      if (off < 0 || off >= span) continue;
+      const uint32_t bit = 1u << (off & 31);
+      bad |= (atomicOr(&bm[off >> 5], bit) & bit) != 0u;
+    }
+    if (bad) set_status(status, SAFEDIT_ERR_INDEX);
+    __syncthreads();
+  }
+}
+
+safedit_status launch_index_check(const int32_t* d_idx, int32_t n_idx, int64_t n_rows, int* status,
+                                  cudaStream_t stream) {
+  if (n_idx <= 0 || n_rows <= 0) return SAFEDIT_OK;
+  const int64_t need = (n_rows + 31) / 32;
+  const int words = static_cast<int>(need < kIdxWords ? need : kIdxWords);
+  const int bytes = words * 4;
+  static_assert(kIdxWords * 4 <= 232448, "bitmap");
+  safedit_status st = set_smem(reinterpret_cast<const void*>(index_check_kernel), kIdxWords * 4);
+  if (st != SAFEDIT_OK) return st;
+  index_check_kernel<<<1, kIdxThreads, bytes, stream>>>(d_idx, n_idx, n_rows, words, status);
+  return after_launch(1);
+}
+
 static safedit_status row_copy(const safedit_tensor* src, const safedit_tensor* dst, int n_tensors,
                                const int32_t* d_idx, int32_t n_idx, void* stream, int scatter) {
   if (!src || !dst || n_tensors < 1 || n_tensors > kMaxRowTensors || n_idx < 0)
@@ -149,6 +197,11 @@ static safedit_status row_copy(const safedit_tensor* src, const safedit_tensor* 
   p.scatter = scatter;
   p.status = status_ptr();
   if (!p.status) return SAFEDIT_ERR_CUDA;
+  if (scatter && index_check_enabled()) {
+    const safedit_status st = launch_index_check(d_idx, n_idx, n_rows_x, p.status,
+                                                 static_cast<cudaStream_t>(stream));
+    if (st != SAFEDIT_OK) return st;
+  }
   dim3 grid(max_blocks, max_bh, n_tensors);
   row_copy_kernel<<<grid, kRowThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
   return after_launch(1);
@@ -156,8 +209,8 @@ static safedit_status row_copy(const safedit_tensor* src, const safedit_tensor* 
 
 // --------------------------------------------------------------- sw_cfg ---
 struct CfgParams {
-  const float* c;
-  const float* u;
+  const void* c;    // f32 or bf16 (the template parameter of the kernel)
+  const void* u;
   const float* s;
   float* out;
   int64_t N, F;
@@ -165,7 +218,22 @@ struct CfgParams {
   float g_ctx, g_diff;
 };
 
+// Four consecutive predictions as floats (bf16 widened exactly), streamed.
+__device__ __forceinline__ float4 load4_cs(const float* p) {
+  return __ldcs(reinterpret_cast<const float4*>(p));
+}
+__device__ __forceinline__ float4 load4_cs(const __nv_bfloat16* p) {
+  const uint2 v = __ldcs(reinterpret_cast<const uint2*>(p));
+  return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                     __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+}
+__device__ __forceinline__ float load1(const float* p) { return *p; }
+__device__ __forceinline__ float load1(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+template <typename T>
 __global__ void __launch_bounds__(256) sw_cfg_vec4_kernel(CfgParams p) {
+  const T* pc = static_cast<const T*>(p.c);
+  const T* pu = static_cast<const T*>(p.u);
   const int64_t F4 = p.F >> 2;
   const int64_t total = p.N * F4;
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
@@ -173,8 +241,8 @@ __global__ void __launch_bounds__(256) sw_cfg_vec4_kernel(CfgParams p) {
     const int64_t i = e / F4;
     const int64_t f = (e - i * F4) << 2;
     const float g = fmaf(p.g_diff, __ldg(p.s + i), p.g_ctx);
-    const float4 c = __ldcs(reinterpret_cast<const float4*>(p.c + i * p.sc + f));
-    const float4 u = __ldcs(reinterpret_cast<const float4*>(p.u + i * p.su + f));
+    const float4 c = load4_cs(pc + i * p.sc + f);
+    const float4 u = load4_cs(pu + i * p.su + f);
     float4 o;
     o.x = fmaf(g, c.x - u.x, u.x);
     o.y = fmaf(g, c.y - u.y, u.y);
@@ -184,14 +252,17 @@ __global__ void __launch_bounds__(256) sw_cfg_vec4_kernel(CfgParams p) {
   }
 }
 
+template <typename T>
 __global__ void __launch_bounds__(256) sw_cfg_scalar_kernel(CfgParams p) {
+  const T* pc = static_cast<const T*>(p.c);
+  const T* pu = static_cast<const T*>(p.u);
   const int64_t total = p.N * p.F;
   for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < total;
        e += int64_t(gridDim.x) * blockDim.x) {
     const int64_t i = e / p.F;
     const int64_t f = e - i * p.F;
     const float g = fmaf(p.g_diff, p.s[i], p.g_ctx);
-    const float c = p.c[i * p.sc + f], u = p.u[i * p.su + f];
+    const float c = load1(pc + i * p.sc + f), u = load1(pu + i * p.su + f);
     p.out[i * p.so + f] = fmaf(g, c - u, u);
   }
 }
@@ -277,7 +348,8 @@ safedit_status safedit_sw_cfg(const safedit_tensor* eps_c, const safedit_tensor*
   if ((st = check_tensor(eps_c, 2)) != SAFEDIT_OK) return st;
   if ((st = check_tensor(eps_u, 2)) != SAFEDIT_OK) return st;
   if ((st = check_tensor(out, 2)) != SAFEDIT_OK) return st;
-  if (eps_c->dtype != SAFEDIT_F32 || eps_u->dtype != SAFEDIT_F32 || out->dtype != SAFEDIT_F32)
+  const bool bf16 = eps_c->dtype == SAFEDIT_BF16;
+  if ((eps_c->dtype != SAFEDIT_F32 && !bf16) || eps_u->dtype != eps_c->dtype || out->dtype != SAFEDIT_F32)
     return SAFEDIT_ERR_DTYPE;
   const int64_t N = eps_c->dims[0], F = eps_c->dims[1];
   if (eps_u->dims[0] != N || eps_u->dims[1] != F || out->dims[0] != N || out->dims[1] != F)
@@ -287,8 +359,8 @@ safedit_status safedit_sw_cfg(const safedit_tensor* eps_c, const safedit_tensor*
   if (N == 0 || F == 0) return SAFEDIT_OK;
   if (!d_s) return SAFEDIT_ERR_INVALID_ARG;
   CfgParams p;
-  p.c = static_cast<const float*>(eps_c->data);
-  p.u = static_cast<const float*>(eps_u->data);
+  p.c = eps_c->data;
+  p.u = eps_u->data;
   p.s = d_s;
   p.out = static_cast<float*>(out->data);
   p.N = N;
@@ -298,8 +370,11 @@ safedit_status safedit_sw_cfg(const safedit_tensor* eps_c, const safedit_tensor*
   p.so = out->strides[0];
   p.g_ctx = gamma_ctx;
   p.g_diff = gamma_sens - gamma_ctx;
+  // 4 predictions per thread: 16-byte (f32) or 8-byte (bf16) aligned groups
+  const uintptr_t in_align = bf16 ? 7u : 15u;
   const bool vec = (F % 4 == 0) && (p.sc % 4 == 0) && (p.su % 4 == 0) && (p.so % 4 == 0) &&
-                   aligned16(p.c) && aligned16(p.u) && aligned16(p.out);
+                   (reinterpret_cast<uintptr_t>(p.c) & in_align) == 0 &&
+                   (reinterpret_cast<uintptr_t>(p.u) & in_align) == 0 && aligned16(p.out);
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -308,10 +383,15 @@ safedit_status safedit_sw_cfg(const safedit_tensor* eps_c, const safedit_tensor*
   const int64_t cap = int64_t(sms) * 8;
   if (blocks > cap) blocks = cap;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (vec)
-    sw_cfg_vec4_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+  const unsigned grid = static_cast<unsigned>(blocks);
+  if (vec && bf16)
+    sw_cfg_vec4_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
+  else if (vec)
+    sw_cfg_vec4_kernel<float><<<grid, 256, 0, s>>>(p);
+  else if (bf16)
+    sw_cfg_scalar_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
   else
-    sw_cfg_scalar_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+    sw_cfg_scalar_kernel<float><<<grid, 256, 0, s>>>(p);
   return after_launch(1);
 }
 

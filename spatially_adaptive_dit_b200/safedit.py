@@ -33,7 +33,7 @@ EXPORTED = ("safedit_cross_attn_probs", "safedit_partition_accumulate", "safedit
             "safedit_partition_finalize", "safedit_mask_is_row_constant", "safedit_attn_subset",
             "safedit_scatter_state", "safedit_gather_rows", "safedit_sw_cfg", "safedit_stepcache_sw_cfg",
             "safedit_gemm_bias_act", "safedit_get_device_status", "safedit_status_string", "safedit_kernel_launch_count",
-            "safedit_debug_set_wait_limit_ns")
+            "safedit_debug_set_wait_limit_ns", "safedit_debug_set_index_check")
 
 
 class SafeditTensor(ctypes.Structure):
@@ -69,9 +69,11 @@ _lib.safedit_status_string.restype = ctypes.c_char_p
 _lib.safedit_kernel_launch_count.restype = ctypes.c_uint64
 _lib.safedit_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.safedit_debug_set_wait_limit_ns.restype = ctypes.c_uint64
+_lib.safedit_debug_set_index_check.argtypes = [ctypes.c_int32]
+_lib.safedit_debug_set_index_check.restype = ctypes.c_int32
 for _n in EXPORTED:
     if _n not in ("safedit_status_string", "safedit_kernel_launch_count",
-                  "safedit_debug_set_wait_limit_ns"):
+                  "safedit_debug_set_wait_limit_ns", "safedit_debug_set_index_check"):
         getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -215,6 +217,10 @@ def safedit_kernel_launch_count() -> int:
 
 def safedit_debug_set_wait_limit_ns(ns: int) -> int:
     return int(_lib.safedit_debug_set_wait_limit_ns(int(ns)))
+
+
+def safedit_debug_set_index_check(on: bool) -> bool:
+    return bool(_lib.safedit_debug_set_index_check(1 if on else 0))
 
 
 def raw_call(name, *args):

@@ -334,3 +334,19 @@ def test_compact_query_rows_over_all_keys():
         for h in range(H):
             ref = oracle.attn_subset(f64(q[b, h]), f64(k[b, h]), f64(v[b, h]))
             check_attn(f64(out[b, h]), ref, f"b{b}h{h}")
+
+
+def test_config_2560_dense_anchor_as_benchmarked():
+    """The CAR anchor of the headline workload in the launch configuration the
+    benchmark times (idx = NULL: all 25600 rows of all 48 slices, output
+    [B,H,N,d]); sampled rows of two slices against the oracle's dense
+    (matrix-form) attention on those query rows."""
+    w = wl.W2560
+    q, k, v = wl.qkv(w, device=DEV)
+    out = torch.zeros(w.B, w.H, w.N, w.d, dtype=BF, device=DEV)
+    run(q, k, v, out=out)
+    rows = np.linspace(0, w.N - 1, 64).astype(np.int64)
+    rt = torch.as_tensor(rows, device=DEV)
+    for (b, h) in [(0, 3), (1, 20)]:
+        ref = oracle.attn_dense(f64(q[b, h, rt]), f64(k[b, h]), f64(v[b, h]))
+        check_attn(f64(out[b, h, rt]), ref, f"anchor b{b}h{h}")

@@ -95,6 +95,33 @@ def test_sw_cfg(N, F):
     assert np.abs(cd.cpu().double().numpy() - ref2).max() <= 1e-5 * (1 + np.abs(ref2).max())
 
 
+@pytest.mark.parametrize("N,F,vec", [(4096, 16, True), (300, 6, False), (257, 16, False)])
+def test_sw_cfg_bf16_predictions(N, F, vec):
+    """bf16 eps_c / eps_u (widened exactly), f32 output; vector path (F % 4
+    == 0, 8-byte aligned rows) and the scalar path (odd widths, and a view
+    whose rows start off the 8-byte boundary)."""
+    g = _gen(N + 13 * F)
+    c = torch.randn(N, F, generator=g).to(torch.bfloat16)
+    u = torch.randn(N, F, generator=g).to(torch.bfloat16)
+    s = torch.rand(N, generator=g)
+    cd, ud = c.to(DEV), u.to(DEV)
+    if not vec and F % 4 == 0:  # same values at an address 2 bytes past an 8-byte boundary
+        cb = torch.empty(N * F + 1, dtype=torch.bfloat16, device=DEV)
+        cb[1:].copy_(cd.flatten())
+        cd = cb[1:].view(N, F)
+    out = torch.empty(N, F, device=DEV)
+    sd().safedit_sw_cfg(cd, ud, s.to(DEV), 3.0, 5.0, out)
+    expect_status(0)
+    ref = oracle.sw_cfg(c.double(), u.double(), s, 3.0, 5.0)
+    gam = 3.0 + 2.0 * s.double().numpy()[:, None]
+    scale = np.abs(u.double().numpy()) + np.abs(gam) * np.abs((c.double() - u.double()).numpy())
+    err = np.abs(out.cpu().double().numpy() - ref)
+    assert np.all(err <= CFG_REL * scale + 1e-30)
+    with pytest.raises(sd().SafeditError) as e:  # mixed input types
+        sd().safedit_sw_cfg(cd, u.float().to(DEV), s.to(DEV), 3.0, 5.0, out)
+    assert e.value.code == sd().ERR_DTYPE
+
+
 # ------------------------------------------------------------- partition PCSP
 @pytest.mark.parametrize("H,N,L,nvalid", [(24, 4096, 256, 128), (2, 256, 32, 20), (3, 1000, 30, 25),
                                           (4, 300, 512, 400)])

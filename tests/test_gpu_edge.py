@@ -74,3 +74,54 @@ def test_projection_without_rows_or_columns():
     w0 = torch.empty(0, 64, dtype=BF, device=DEV)
     out0 = torch.empty(5, 0, dtype=BF, device=DEV)
     _no_launch(lambda: sd().safedit_gemm_bias_act(a1, w0, None, 0, None, out0))
+
+
+@pytest.fixture
+def index_check():
+    prev = sd().safedit_debug_set_index_check(True)
+    yield
+    sd().safedit_debug_set_index_check(prev)
+
+
+def test_debug_index_check_flags_duplicates(index_check):
+    """Debug mode: every scattering index vector is checked before the
+    scatter.  A duplicate (two writers for one row) or an out-of-range entry
+    sets SAFEDIT_ERR_INDEX; a unique vector passes and the results are the
+    ones the unchecked calls give.  Index ranges wider than one shared-memory
+    bitmap window (1.8 M rows) are checked window by window."""
+    B, H, N, D, kr = 1, 2, 300, 64, 40
+    g = torch.Generator().manual_seed(3)
+    uniq = torch.randperm(N, generator=g)[:kr].to(torch.int32).to(DEV)
+    dup = uniq.clone()
+    dup[17] = dup[3]
+    src = torch.randn(B, H, kr, D, generator=g).to(BF).to(DEV)
+    dst = torch.zeros(B, H, N, D, dtype=BF, device=DEV)
+    q = torch.randn(B, H, N, D, generator=g).to(BF).to(DEV)
+    a = torch.randn(kr, 64, generator=g).to(BF).to(DEV)
+    w = torch.randn(64, 64, generator=g).to(BF).to(DEV)
+    y = torch.zeros(N, 64, dtype=BF, device=DEV)
+    calls = [
+        lambda ix: sd().safedit_scatter_state([src], [dst], ix, kr),
+        lambda ix: sd().safedit_attn_subset(q, q, q, ix, kr, None, None, 0.0, dst, 1),
+        lambda ix: sd().safedit_gemm_bias_act(a, w, None, 0, ix, y),
+    ]
+    for call in calls:
+        call(uniq)
+        expect_status(0)
+        call(dup)
+        expect_status(sd().ERR_INDEX)
+    # without the check a duplicate goes unnoticed (the caller's contract)
+    sd().safedit_debug_set_index_check(False)
+    sd().safedit_scatter_state([src], [dst], dup, kr)
+    expect_status(0)
+    sd().safedit_debug_set_index_check(True)
+    # more rows than one bitmap window: a duplicate in the second window
+    big = 1_859_584 + 1000
+    src2 = torch.randn(1, 1, 3, 8, generator=g).to(BF).to(DEV)
+    dst2 = torch.zeros(1, 1, big, 8, dtype=BF, device=DEV)
+    ix2 = torch.tensor([5, big - 1, big - 1], dtype=torch.int32, device=DEV)
+    sd().safedit_scatter_state([src2], [dst2], ix2, 3)
+    expect_status(sd().ERR_INDEX)
+    ix2[2] = big - 2
+    sd().safedit_scatter_state([src2], [dst2], ix2, 3)
+    expect_status(0)

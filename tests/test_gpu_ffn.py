@@ -243,3 +243,34 @@ def test_gathered_qkv_projection_feeds_srsu():
             ref = oracle.attn_subset(proj[:, 0, h], kst, vst)
             rf = rel_fro(f64(out[bb, h]), ref)
             assert rf <= 1e-2, f"b{bb}h{h}: relFro={rf:.3e}"
+
+
+def test_w2_projection_at_bench_shape_scattered_into_cache():
+    """The FFN W2 projection of the 2560^2 workload exactly as the benchmark
+    launches it: the bf16 hidden layer of every focus row (B = 2 batches of
+    |S| = 7680 rows, K = 4D = 9216, N = D = 2304, so 144 k-blocks per tile)
+    times W2 plus b2, each row written to its token's row of the FFN cache
+    (CTA-pair kernel).  Sampled rows of both batches against the oracle with
+    the per-element bound of a projection; the rows no focus token maps to
+    keep their bytes."""
+    w = wl.W2560
+    B, k, D, F = w.B, w.k, w.D_model, w.D_ff
+    w1, b1, w2, b2 = wl.ffn_weights(w)
+    score = wl.blob_scores(wl.Workload("2560b", 2, B=1, H=1, N=w.N, d=w.d, L=1, n_valid=1,
+                                       rho=w.rho, grid=w.grid)).to(DEV)
+    idx = torch.empty(k, dtype=torch.int32, device=DEV)
+    sd().safedit_partition_finalize(score, w.N, k, idx, None, None)
+    hid = wl.normal((B, k, F), w, 777, device=DEV)      # a bf16 hidden layer of unit scale
+    y0 = wl.ffn_states(w)[1]                            # the FFN cache [B, N, D] bf16
+    y = y0.to(DEV)
+    sd().safedit_gemm_bias_act(hid, w2.to(DEV), b2.to(DEV), 0, idx, y)
+    expect_status(0)
+    ic = idx.cpu().long()
+    rows = np.linspace(0, k - 1, 40).astype(np.int64)
+    for bb in range(B):
+        got = y[bb, ic[rows].to(DEV)].cpu()
+        _check_plain(got, hid[bb, torch.as_tensor(rows, device=DEV)].cpu(), w2, b2)
+    hit = torch.zeros(w.N, dtype=torch.bool)
+    hit[ic] = True
+    keep = torch.nonzero(~hit).flatten()[::97]
+    assert torch.equal(y[:, keep.to(DEV)].cpu().view(torch.int16), y0[:, keep].view(torch.int16))
