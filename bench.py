@@ -55,6 +55,77 @@ def _dist():
     return ws, rank, local
 
 
+def percentiles(ms):
+    """p10 / p50 / p90 (nearest rank) of a list of timings."""
+    v = sorted(ms)
+    pick = lambda q: v[int(round(q * (len(v) - 1)))]
+    return {"p10": round(pick(0.1), 4), "p50": round(pick(0.5), 4), "p90": round(pick(0.9), 4)}
+
+
+class L2Flush:
+    """Writes a buffer of four times the L2 size, so that the next launch finds
+    none of its inputs in L2, then reads it back, so that the lines left in L2
+    are clean and the timed launch does not pay for writing them back (run
+    between timed repetitions, outside the events)."""
+
+    def __init__(self, dev):
+        self.bytes = 4 * torch.cuda.get_device_properties(dev).L2_cache_size
+        self.buf = torch.empty(self.bytes // 4, dtype=torch.int32, device=dev)
+        self.sink = torch.empty((), dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1)
+        torch.amax(self.buf, dim=0, out=self.sink)
+
+
+def time_reps_interleaved(fns, stream, reps=20, warmup=3):
+    """Like time_reps for several launches at once, taken in turn within every
+    repetition (so that clock and power drift over the run affects them
+    alike).  Returns name -> p10 / p50 / p90."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            for fn in fns.values():
+                fn()
+        evs = {n: [] for n in fns}
+        for _ in range(reps):
+            for n, fn in fns.items():
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                evs[n].append((a, b))
+    stream.synchronize()
+    out = {}
+    for n, lst in evs.items():
+        out[n] = percentiles([a.elapsed_time(b) for a, b in lst])
+        out[n]["n"] = reps
+    return out
+
+
+def time_reps(fn, stream, reps=20, warmup=3, flush=None):
+    """CUDA-event timings (ms) of `reps` launches of fn() on `stream` after
+    `warmup` untimed ones; `flush` (optional) runs before every launch,
+    outside the events.  Returns p10 / p50 / p90 and the sample count."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            fn()
+        evs = []
+        for _ in range(reps):
+            if flush is not None:
+                flush()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            evs.append((a, b))
+    stream.synchronize()
+    out = percentiles([a.elapsed_time(b) for a, b in evs])
+    out["n"] = reps
+    return out
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -135,9 +206,10 @@ class Trajectory:
     generation on this device; reduce_score then completes the PCSP score
     over the other devices' heads before the split."""
 
-    def __init__(self, w, dev, seed_step=0, heads=None, reduce_score=None):
+    def __init__(self, w, dev, seed_step=0, heads=None, reduce_score=None, pcsp="fused"):
         from spatially_adaptive_dit_b200 import safedit as sd
         self.sd, self.w, self.dev = sd, w, dev
+        self.pcsp = pcsp  # "fused": one pcsp_score launch; "unfused": probabilities, then aggregation
         B, N, d, L, k = w.B, w.N, w.d, w.L, w.k
         h0, h1 = (0, w.H) if heads is None else heads
         H = h1 - h0
@@ -164,22 +236,29 @@ class Trajectory:
         self.verdict = torch.zeros(1, dtype=torch.int32, device=dev)
         self.eps_c, self.eps_u = wl.cfg_preds(w, step=seed_step, device=dev)
         self.cfg_out = torch.empty_like(self.eps_c)
+        self.H = H
         self.flop_srsu = 4.0 * k * N * d * B * H
         self.flop_dense = 4.0 * N * N * d * B * H
         self.bytes = {
             "cross_attn_probs": H * N * L * 4 + H * N * d * 2 + H * L * d * 2,
+            # Q_img and K_txt of the cond branch read once, the fp64 score read and written
+            "pcsp_score": H * N * d * 2 + H * L * d * 2 + 2 * N * 8,
             # the 16-byte groups of P that hold a content column (the kernel reads no others)
             "partition_accumulate": H * N * 16 * int(self.content.view(-1, 4).any(dim=1).sum()) + N * 16 + L,
             "scatter_state": 2 * (2 * B * H * k * d * 2) + 4 * k,
             "sw_cfg": 3 * N * w.F * 4 + 4 * N,
         }
 
-    def run(self, stream, ev=None):
+    def run(self, stream, ev=None, flush=None):
         """Enqueue one trajectory on `stream`.  ev: dict name -> list to which
-        (start, end) CUDA events of each launch are appended."""
+        (start, end) CUDA events of each launch are appended.  flush: called
+        before every attention and scatter launch, outside its events (an L2
+        flush where the per-device state would otherwise stay in L2)."""
         sd, w = self.sd, self.w
 
         def timed(name, fn):
+            if flush is not None and name in ("attn_dense_anchor", "attn_subset_srsu", "scatter_state"):
+                flush()
             if ev is None:
                 fn()
                 return
@@ -193,7 +272,10 @@ class Trajectory:
         self.score.zero_()
         for t in range(w.steps):
             anchor = (t % w.period == 0)
-            if t < w.warmup:  # PCSP warm-up on the cond branch
+            if t < w.warmup and self.pcsp == "fused":  # PCSP warm-up on the cond branch
+                timed("pcsp_score", lambda: sd.safedit_pcsp_score(
+                    self.q_img, self.k_txt, self.valid, self.content, 0, 0.0, self.score, stream))
+            elif t < w.warmup:
                 timed("cross_attn_probs", lambda: sd.safedit_cross_attn_probs(
                     self.q_img, self.k_txt, self.valid, 0, 0.0, self.P, stream))
                 timed("partition_accumulate", lambda: sd.safedit_partition_accumulate(
@@ -235,14 +317,26 @@ def run_ours(args):
     from spatially_adaptive_dit_b200 import safedit as sd
     sharded = args.shard == "heads" and ws > 1
     if sharded:  # one generation, H / ws heads per GPU, one score all-reduce
-        tr = Trajectory(W, dev, seed_step=0, heads=head_range(W.H, ws, rank), reduce_score=score_all_reduce)
+        tr = Trajectory(W, dev, seed_step=0, heads=head_range(W.H, ws, rank), reduce_score=score_all_reduce,
+                        pcsp=args.pcsp)
     else:  # independent replicas
-        tr = Trajectory(W, dev, seed_step=1000 * rank)
-    stream = torch.cuda.Stream(device=dev)
+        tr = Trajectory(W, dev, seed_step=1000 * rank, pcsp=args.pcsp)
     torch.cuda.synchronize()
+    # the peak below counts the trajectory's own buffers, not the temporaries of their construction
+    torch.cuda.reset_peak_memory_stats(dev)
+    # L2: this device's K/V state must not be served from L2 between launches
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    state_bytes = tr.k_state.numel() * tr.k_state.element_size()
+    flush = L2Flush(dev) if 2 * state_bytes < 2 * l2 else None
+    l2_note = (f"per-device K/V state {2 * state_bytes / 1e6:.0f} MB fits in L2 ({l2 / 1e6:.0f} MB): L2 flushed "
+               f"({4 * l2 / 1e6:.0f} MB write) before every attention and scatter launch, outside their events"
+               if flush is not None else
+               f"inputs larger than L2 (Q/K/V/state {state_bytes / 1e6:.0f} MB each per device, L2 "
+               f"{l2 / 1e6:.0f} MB), no flush needed")
+    stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            tr.run(stream)
+            tr.run(stream, flush=flush)
     stream.synchronize()
     assert sd.safedit_get_device_status(stream) == 0
 
@@ -259,7 +353,7 @@ def run_ours(args):
     t0.record(stream)
     with torch.cuda.stream(stream):
         for _ in range(args.steps):
-            tr.run(stream, ev)
+            tr.run(stream, ev, flush=flush)
     t1.record(stream)
     t1.synchronize()
     torch.cuda.synchronize()
@@ -278,7 +372,16 @@ def run_ours(args):
     # ---- end to end through the public API with host buffers (pinned)
     e2e = run_e2e(tr, stream, args)
     e2e["ms"] = max_over_ranks([e2e["ms"]], dev)[0]
-    unfused = statistics.mean(per["cross_attn_probs"]) + statistics.mean(per["partition_accumulate"])
+    # the unfused PCSP rows (probabilities, then aggregation), each launched alone
+    rows_flush = L2Flush(dev)
+    alone = {
+        "cross_attn_probs": time_reps(lambda: sd.safedit_cross_attn_probs(
+            tr.q_img, tr.k_txt, tr.valid, 0, 0.0, tr.P, stream), stream, flush=rows_flush),
+        "partition_accumulate": time_reps(lambda: sd.safedit_partition_accumulate(
+            tr.P, tr.content, tr.score, stream), stream, flush=rows_flush),
+    }
+    del rows_flush
+    unfused = alone["cross_attn_probs"]["p50"] + alone["partition_accumulate"]["p50"]
     ext = measure_extensions(tr, stream, dev, unfused)
 
     if rank == 0:
@@ -287,18 +390,28 @@ def run_ours(args):
         srsu_call_ms = srsu_ms / n_srsu
         achieved = tr.flop_srsu / (srsu_call_ms * 1e-3) / 1e12
         kern = {}
+
+        def bw(entry, name, ms):
+            if name in tr.bytes:
+                gbs = tr.bytes[name] / (ms * 1e-3) / 1e9
+                entry.update({"gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)})
+
         for n, v in per.items():
             m = statistics.mean(v)
-            entry = {"ms_mean": round(m, 4), "calls_per_step": len(v) // args.steps}
-            if n in tr.bytes:
-                gbs = tr.bytes[n] / (m * 1e-3) / 1e9
-                entry.update({"gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)})
+            entry = {"ms_mean": round(m, 4), "calls_per_step": len(v) // args.steps, **percentiles(v),
+                     "n": len(v), "timed": "inside the trajectory"}
+            bw(entry, n, entry["p50"])
             if n == "attn_dense_anchor":
                 entry["tflops"] = round(tr.flop_dense / (m * 1e-3) / 1e12, 1)
             if n == "attn_subset_srsu":
                 entry["tflops"] = round(tr.flop_srsu / (m * 1e-3) / 1e12, 1)
             kern[n] = entry
+        for n, t in alone.items():
+            entry = {**t, "timed": "launched alone, 3 warm-ups + 20 reps, L2 flushed before each"}
+            bw(entry, n, t["p50"])
+            kern[n] = entry
         traffic = _ncu_traffic()
+        algo_bytes = _srsu_algorithmic_bytes(tr)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3),
@@ -308,18 +421,24 @@ def run_ours(args):
                        "parallelism": (f"heads x{ws} (one generation, {W.H // ws} heads per GPU; one all-reduce "
                                        "of the fp64 score vector after the warm-up)") if sharded else
                                       f"replicas x{ws} (independent trajectories, no collective)",
-                       "l2": "inputs larger than L2 (Q/K/V/state 236 MB each), no flush needed",
+                       "l2": l2_note,
+                       "pcsp": ("fused pcsp_score on the warm-up step" if tr.pcsp == "fused" else
+                                "cross_attn_probs + partition_accumulate on the warm-up step"),
                        "srsu_calls_per_step": n_srsu // args.steps,
                        "srsu_ms_per_call": round(srsu_call_ms, 4)},
             "kernels": kern,
             "roofline": {"kernel": "attn_subset (SRSU)", "bound": "tensor", "achieved": round(achieved, 1),
                          "peak": bf16_sust, "peak_kind": f"bf16_tflops_sustained ({src})",
-                         "unit": "TFLOP/s", "frac": round(achieved / bf16_sust, 4), "traffic": traffic},
+                         "unit": "TFLOP/s", "frac": round(achieved / bf16_sust, 4),
+                         "frac_of_burst": round(achieved / bf16_burst, 4), "traffic": traffic,
+                         "algorithmic_bytes": algo_bytes,
+                         "traffic_over_algorithmic": None if traffic is None else round(traffic / algo_bytes, 3)},
             "gpu_launches": launches,
             "memory": {"peak_allocated_gb": round(peak_gb, 2),
-                       "note": "all buffers of the attention path incl. the 0.63 GB probability tensor; "
-                               "a dense masked path that materialises bf16 scores [B,H,N,N] would need "
-                               f"{W.B * W.H * W.N * W.N * 2 / 1e9:.1f} GB for them alone"},
+                       "note": f"this device's buffers of the attention path ({tr.H} heads) incl. the "
+                               f"{tr.P.numel() * 4 / 1e9:.2f} GB probability tensor; a dense masked path that "
+                               "materialises bf16 scores [B,H,N,N] would need "
+                               f"{W.B * tr.H * W.N * W.N * 2 / 1e9:.1f} GB for them alone"},
             "device_status": status,
             "extensions": ext,
             "e2e": {"value": round(whole_job_tflops(tr.flop_srsu * n_srsu / args.steps, ws, e2e["ms"]), 3),
@@ -329,10 +448,10 @@ def run_ours(args):
         }
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
-            gms = {n: e["ms_mean"] for n, e in kern.items()}
-            gms.update({"ffn_block": ext["ffn_block_ms"], "mask_is_row_constant": ext["mask_stress"]["ms"],
-                        "qkv_projection_gathered": ext["qkv_projection_gathered"]["ms"],
-                        "stepcache_sw_cfg": ext["stepcache_sw_cfg"]["ms"]})
+            gms = {n: e.get("p50", e.get("ms_mean")) for n, e in kern.items()}
+            gms.update({"ffn_block": ext["ffn_block"]["p50"], "mask_is_row_constant": ext["mask_stress"]["p50"],
+                        "qkv_projection_gathered": ext["qkv_projection_gathered"]["p50"],
+                        "stepcache_sw_cfg": ext["stepcache_sw_cfg"]["p50"]})
             line["oracle_rows"] = oracle_rows(gms)
         print(json.dumps(line), flush=True)
     if ws > 1:
@@ -340,15 +459,26 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
-def measure_extensions(tr, stream, dev, unfused_pcsp_ms, reps=5):
-    """The steps around the per-step path, each launched alone on the same
-    workload (best of `reps` CUDA-event timings after 2 warm-ups): the fused
+def _srsu_algorithmic_bytes(tr):
+    """Bytes one SRSU launch must move at least: K and V of every slice read
+    once, the gathered Q rows read and the output rows written."""
+    w = tr.w
+    return (2 * w.N + 2 * tr.k) * w.d * 2 * w.B * tr.H + 4 * tr.k
+
+
+def measure_extensions(tr, stream, dev, unfused_pcsp_ms):
+    """The steps around the per-step path and the other configurations, each
+    launched alone (3 warm-ups + 20 CUDA-event reps, p50 with p10 / p90; L2
+    flushed before every rep wherever the inputs could stay in L2): the fused
     PCSP score, SkipSparse's projections on the focus rows (gathered Q|K|V;
     FFN W1 with bias and GELU; FFN W2 with bias, rows scattered into the FFN
-    cache) and the StepCache guidance combine."""
+    cache), the StepCache guidance combine, the mask check and the kept-mask
+    SRSU calls of the stress shape, the 1024^2 configuration, the 3072^2
+    sensitive-fraction sweep and the guidance combines at F = 4096."""
     sd, w = tr.sd, tr.w
     hbm, bf16_burst, _, src = _peaks()
     k, D, F, B = tr.k, w.D_model, w.D_ff, w.B
+    flush = L2Flush(dev)
     w1, b1, w2, b2 = (t.to(dev) for t in wl.ffn_weights(w))
     wqkv, bqkv = (t.to(dev) for t in wl.qkv_proj_weights(w))
     x, y = (t.to(dev) for t in wl.ffn_states(w))
@@ -358,25 +488,17 @@ def measure_extensions(tr, stream, dev, unfused_pcsp_ms, reps=5):
     qkv = torch.empty(B, k, 3 * D, dtype=torch.bfloat16, device=dev)
     prev_c, prev_u = wl.cfg_preds(w, step=1, device=dev)
 
-    def best_ms(fn):
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                fn()
-            evs = []
-            for _ in range(reps):
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                fn()
-                b.record(stream)
-                evs.append((a, b))
-        stream.synchronize()
-        return min(a.elapsed_time(b) for a, b in evs)
-
-    def gemm_entry(ms, flop):
-        tf = flop / (ms * 1e-3) / 1e12
-        return {"ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / bf16_burst, 3),
+    def gemm_entry(t, flop):
+        tf = flop / (t["p50"] * 1e-3) / 1e12
+        return {**t, "tflops": round(tf, 1), "frac": round(tf / bf16_burst, 3),
                 "peak": bf16_burst, "peak_kind": f"bf16_tflops burst ({src})"}
+
+    def bw_entry(t, nbytes, note=None):
+        gbs = nbytes / (t["p50"] * 1e-3) / 1e9
+        e = {**t, "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
+        if note:
+            e["note"] = note
+        return e
 
     gather = lambda: sd.safedit_gather_rows([x.view(B, 1, w.N, D)], [xs], tr.idx_s, k, stream)
     ffn1 = lambda: sd.safedit_gemm_bias_act(xs3, w1, b1, 1, None, h, stream)
@@ -384,43 +506,157 @@ def measure_extensions(tr, stream, dev, unfused_pcsp_ms, reps=5):
     proj = lambda: sd.safedit_gemm_bias_act(xs3, wqkv, bqkv, 0, None, qkv, stream)
     gather()
     ffn_flop = 2.0 * B * k * D * F
+    pcsp = time_reps(lambda: sd.safedit_pcsp_score(tr.q_img, tr.k_txt, tr.valid, tr.content, 0, 0.0, tr.score,
+                                                   stream), stream, flush=flush)
     out = {
-        "pcsp_fused": {"ms": round(best_ms(lambda: sd.safedit_pcsp_score(
-            tr.q_img, tr.k_txt, tr.valid, tr.content, 0, 0.0, tr.score, stream)), 4),
-            "unfused_ms": round(unfused_pcsp_ms, 4)},
-        "qkv_projection_gathered": gemm_entry(best_ms(proj), 2.0 * B * k * D * 3 * D),
-        "ffn_w1_bias_gelu": gemm_entry(best_ms(ffn1), ffn_flop),
-        "ffn_w2_bias_scatter": gemm_entry(best_ms(ffn2), ffn_flop),
-        "ffn_block_ms": round(best_ms(lambda: (gather(), ffn1(), ffn2())), 4),
+        "pcsp_fused": {**pcsp, "unfused_ms": round(unfused_pcsp_ms, 4)},
+        "qkv_projection_gathered": gemm_entry(time_reps(proj, stream), 2.0 * B * k * D * 3 * D),
+        "ffn_w1_bias_gelu": gemm_entry(time_reps(ffn1, stream), ffn_flop),
+        "ffn_w2_bias_scatter": gemm_entry(time_reps(ffn2, stream), ffn_flop),
+        "ffn_block": time_reps(lambda: (gather(), ffn1(), ffn2()), stream),
     }
-    sc_ms = best_ms(lambda: sd.safedit_stepcache_sw_cfg(prev_c, tr.eps_c, prev_u, tr.eps_u, tr.s, 0.5,
-                                                        w.gamma_ctx, w.gamma_sens, tr.cfg_out, stream))
     sc_bytes = 5 * tr.eps_c.numel() * 4 + 4 * w.N
-    out["stepcache_sw_cfg"] = {"ms": round(sc_ms, 4), "gbs": round(sc_bytes / (sc_ms * 1e-3) / 1e9, 1),
-                               "note": f"F={tr.eps_c.shape[1]}: {sc_bytes / 1e6:.1f} MB, launch-bound"}
+    out["stepcache_sw_cfg"] = bw_entry(
+        time_reps(lambda: sd.safedit_stepcache_sw_cfg(prev_c, tr.eps_c, prev_u, tr.eps_u, tr.s, 0.5, w.gamma_ctx,
+                                                      w.gamma_sens, tr.cfg_out, stream), stream, flush=flush),
+        sc_bytes, f"F={tr.eps_c.shape[1]}: {sc_bytes / 1e6:.1f} MB, launch-bound")
     del x, y, xs, h, qkv, w1, w2
     mask = torch.zeros(1, 1, wl.STRESS.N, wl.STRESS.N, dtype=torch.bfloat16, device=dev)
-    out["mask_stress"] = {"ms": round(best_ms(lambda: sd.safedit_mask_is_row_constant(mask, tr.verdict, None,
-                                                                                      stream)), 4),
-                          "note": f"[1,1,{wl.STRESS.N},{wl.STRESS.N}] bf16 all-zero mask (removable: read fully)"}
+    out["mask_stress"] = bw_entry(
+        time_reps(lambda: sd.safedit_mask_is_row_constant(mask, tr.verdict, None, stream), stream, flush=flush),
+        mask.numel() * 2, f"[1,1,{wl.STRESS.N},{wl.STRESS.N}] bf16 all-zero mask (removable: read fully)")
     del mask
     # SRSU with kept masks at the stress shape: time per call and slowdown
     # against the same launch with the mask elided
     cases, flop = stress_srsu_cases(sd, dev, stream)
-    ms = {name: best_ms(fn) for name, fn in cases.items()}
-    base = ms["srsu_mask_elided"]
+    ms = time_reps_interleaved(cases, stream)
+    base = ms["srsu_mask_elided"]["p50"]
     out["kept_mask_stress"] = {
-        name: {"ms": round(t, 4), "tflops": round(flop / (t * 1e-3) / 1e12, 1), "vs_elided": round(t / base, 3)}
+        name: {**t, "tflops": round(flop / (t["p50"] * 1e-3) / 1e12, 1), "vs_elided": round(t["p50"] / base, 3)}
         for name, t in ms.items()}
     out["kept_mask_stress"]["workload"] = (
         f"B=1, H=32, N={wl.STRESS.N}, d=128, |S|={wl.STRESS.k} (blob scores); padding = trailing 1/8 of the keys "
-        "at -inf; bias = [1,1,N,N] N(0,1) in bf16 or f32")
+        "at -inf; bias = [1,1,N,N] N(0,1) in bf16 or f32; the five launches taken in turn within every rep")
     del cases
+    torch.cuda.empty_cache()
+    out["config_1024"] = measure_1024(sd, dev, stream, flush)
+    torch.cuda.empty_cache()
+    out["sweep_3072"] = measure_sweep_3072(sd, dev, stream)
+    torch.cuda.empty_cache()
+    out["guidance_f4096"] = measure_cfg_wide(sd, dev, stream, flush)
     out["workload"] = (f"B={B}, |S|={k} focus rows per batch, D={D}, F={F}; "
                        "synthetic weights N(0,1)/sqrt(fan_in)")
+    out["timing"] = "3 warm-ups + 20 CUDA-event reps per entry; p50 (p10 / p90 beside it)"
     if sd.safedit_get_device_status(stream) != 0:
         raise RuntimeError("device status set during the extension measurements")
     return out
+
+
+def measure_1024(sd, dev, stream, flush):
+    """The 1024^2-equivalent configuration (B=2, H=24, N=4096, d=96, L=256
+    with 128 valid, |S|=0.3N=1229): every row of the path launched alone on
+    its buffers.  Its K/V state (38 MB per tensor) fits in L2, so L2 is
+    flushed before every rep."""
+    w = wl.W1024
+    hbm, bf16_burst, _, src = _peaks()
+    tr = Trajectory(w, dev)
+    with torch.cuda.stream(stream):
+        tr.run(stream)  # fills the split, the state and the scores
+    stream.synchronize()
+    t = {
+        "attn_subset_srsu": time_reps(lambda: sd.safedit_attn_subset(
+            tr.q, tr.k_state, tr.v_state, tr.idx_s, tr.k, None, None, 0.0, tr.o_state, 1, stream), stream,
+            flush=flush),
+        "attn_dense_anchor": time_reps(lambda: sd.safedit_attn_subset(
+            tr.q, tr.k_state, tr.v_state, None, 0, None, None, 0.0, tr.o_state, 0, stream), stream, flush=flush),
+        "pcsp_score": time_reps(lambda: sd.safedit_pcsp_score(
+            tr.q_img, tr.k_txt, tr.valid, tr.content, 0, 0.0, tr.score, stream), stream, flush=flush),
+        "cross_attn_probs": time_reps(lambda: sd.safedit_cross_attn_probs(
+            tr.q_img, tr.k_txt, tr.valid, 0, 0.0, tr.P, stream), stream, flush=flush),
+        "partition_accumulate": time_reps(lambda: sd.safedit_partition_accumulate(
+            tr.P, tr.content, tr.score, stream), stream, flush=flush),
+        "partition_finalize": time_reps(lambda: sd.safedit_partition_finalize(
+            tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s, stream), stream, flush=flush),
+        "scatter_state": time_reps(lambda: sd.safedit_scatter_state(
+            [tr.k_s, tr.v_s], [tr.k_state, tr.v_state], tr.idx_s, tr.k, stream), stream, flush=flush),
+        "sw_cfg": time_reps(lambda: sd.safedit_sw_cfg(
+            tr.eps_c, tr.eps_u, tr.s, w.gamma_ctx, w.gamma_sens, tr.cfg_out, stream), stream, flush=flush),
+    }
+    for name, flop in (("attn_subset_srsu", tr.flop_srsu), ("attn_dense_anchor", tr.flop_dense)):
+        tf = flop / (t[name]["p50"] * 1e-3) / 1e12
+        t[name].update({"tflops": round(tf, 1), "frac_of_burst": round(tf / bf16_burst, 3)})
+    for name, nbytes in tr.bytes.items():
+        if name in t:
+            gbs = nbytes / (t[name]["p50"] * 1e-3) / 1e9
+            t[name].update({"gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)})
+    t["workload"] = ("1024^2-equivalent: B=2, H=24, N=4096 (64x64), d=96, L=256 (128 valid), |S|=0.3N=1229; "
+                     "L2 flushed before every rep (the 38 MB K/V state would stay in L2)")
+    status = sd.safedit_get_device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} in the 1024^2 measurements")
+    del tr
+    return t
+
+
+def measure_sweep_3072(sd, dev, stream):
+    """The 3072^2 sensitive-fraction sweep (B=2, H=24, N=36864, d=96): SRSU
+    attention of |S| = rho N rows (the top rho N of the clustered blob scores)
+    over all N keys, scattered into the output state, and the dense anchor at
+    rho = 1.  Inputs far larger than L2."""
+    w = wl.W3072
+    _, bf16_burst, bf16_sust, src = _peaks()
+    q, k, v = wl.qkv(w, device=dev)
+    o = torch.zeros_like(q)
+    score = wl.blob_scores(w, device=dev).contiguous()
+    out = {}
+    for rho in w.rho_sweep:
+        kk = wl.k_of(rho, w.N)
+        dense = kk == w.N
+        idx = None
+        if not dense:
+            idx = torch.empty(kk, dtype=torch.int32, device=dev)
+            sd.safedit_partition_finalize(score, w.N, kk, idx, None, None, stream)
+        t = time_reps(lambda: sd.safedit_attn_subset(q, k, v, idx, 0 if dense else kk, None, None, 0.0, o,
+                                                     0 if dense else 1, stream), stream, reps=10)
+        flop = 4.0 * kk * w.N * w.d * w.B * w.H
+        tf = flop / (t["p50"] * 1e-3) / 1e12
+        out[f"rho_{float(rho):.1f}"] = {**t, "rows": kk, "dense": dense, "tflop_per_call": round(flop / 1e12, 3),
+                                        "tflops": round(tf, 1), "frac_of_burst": round(tf / bf16_burst, 3),
+                                        "frac_of_sustained": round(tf / bf16_sust, 3)}
+    out["workload"] = "3072^2-equivalent: B=2, H=24, N=36864 (192x192), d=96; 3 warm-ups + 10 reps per point"
+    out["peak"] = (f"bf16_tflops burst {bf16_burst}, sustained {bf16_sust} ({src}); the points run right after "
+                   "the long trajectory run, under the power cap")
+    status = sd.safedit_get_device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} in the 3072^2 sweep")
+    del q, k, v, o
+    return out
+
+
+def measure_cfg_wide(sd, dev, stream, flush):
+    """The guidance combines at a synthetic prediction width F = 4096 over
+    N = 25600 tokens (the bandwidth sweep of the launch-bound F = 16 kernels):
+    SW-CFG 1.26 GB, StepCache + SW-CFG 2.1 GB per call."""
+    w = W
+    hbm = _peaks()[0]
+    F = 4096
+    c, u = wl.cfg_preds(w, device=dev, F=F)
+    pc, pu = wl.cfg_preds(w, step=1, device=dev, F=F)
+    sv = torch.rand(w.N, device=dev)
+    o = torch.empty_like(c)
+    res = {}
+    for name, fn, nbytes in (
+            ("sw_cfg", lambda: sd.safedit_sw_cfg(c, u, sv, w.gamma_ctx, w.gamma_sens, o, stream),
+             3 * w.N * F * 4 + 4 * w.N),
+            ("stepcache_sw_cfg", lambda: sd.safedit_stepcache_sw_cfg(pc, c, pu, u, sv, 0.5, w.gamma_ctx,
+                                                                     w.gamma_sens, o, stream),
+             5 * w.N * F * 4 + 4 * w.N)):
+        t = time_reps(fn, stream, flush=flush)
+        gbs = nbytes / (t["p50"] * 1e-3) / 1e9
+        res[name] = {**t, "bytes": nbytes, "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
+    res["workload"] = f"N={w.N}, F={F} fp32 (synthetic width; the real F=16 is launch-bound)"
+    del c, u, pc, pu, o
+    return res
 
 
 def max_over_ranks(values, device):
@@ -551,8 +787,11 @@ def run_e2e(tr, stream, args):
             with torch.cuda.stream(stream):
                 if t < w.warmup:
                     q_img, k_txt = d_text[1]
-                    sd.safedit_cross_attn_probs(q_img, k_txt, tr.valid, 0, 0.0, tr.P, stream)
-                    sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream)
+                    if tr.pcsp == "fused":
+                        sd.safedit_pcsp_score(q_img, k_txt, tr.valid, tr.content, 0, 0.0, tr.score, stream)
+                    else:
+                        sd.safedit_cross_attn_probs(q_img, k_txt, tr.valid, 0, 0.0, tr.P, stream)
+                        sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream)
                     ev = torch.cuda.Event()
                     ev.record(stream)
                     text_freed[0] = ev
@@ -806,7 +1045,7 @@ def run_sweep(args):
     torch.cuda.set_device(dev)
     from spatially_adaptive_dit_b200 import safedit as sd
     w = wl.W3072
-    _, bf16_burst, _, src = _peaks()
+    _, bf16_burst, bf16_sust, src = _peaks()
     q, k, v = wl.qkv(w, device=dev)
     o = torch.zeros_like(q)
     stream = torch.cuda.Stream(device=dev)
@@ -946,6 +1185,9 @@ def main():
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="N > 1: independent replicas (default, weak scaling) or one generation split by heads "
                          "(strong scaling; the PCSP score is all-reduced once)")
+    ap.add_argument("--pcsp", default="fused", choices=["fused", "unfused"],
+                    help="PCSP warm-up in the timed trajectory: the fused score kernel (default) or the "
+                         "probabilities kernel followed by the aggregation")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,
