@@ -86,3 +86,41 @@ def test_tiny_trajectory_matches_oracle_schedule(w):
         c, u = steps[t]["eps_c"].double().numpy(), steps[t]["eps_u"].double().numpy()
         g = np.abs(c - u) * max(w.gamma_ctx, w.gamma_sens) + np.abs(u)
         assert np.all(np.abs(gpu["cfg"][t].double().numpy() - ref["cfg"][t]) <= CFG_REL * g + 1e-30)
+
+
+@pytest.mark.parametrize("pcsp", ["fused", "unfused"])
+def test_head_sharded_trajectory_split_matches_unsharded(pcsp):
+    """The benchmark's head-sharded path on one GPU: two trajectories of the
+    1024^2 workload keep heads [0, 12) and [12, 24) of the same seeded
+    generation; the second one's PCSP score (its heads only) is added to the
+    first one's through the reduce hook, standing in for the all-reduce,
+    before the split.  The summed score and the S/C split must equal those of
+    the unsharded trajectory (the two sums differ only in the order of fp64
+    additions), and each shard's attention output must equal the unsharded
+    output on its heads."""
+    import bench
+    w = wl.W1024
+    dev = torch.device(DEV)
+    stream = torch.cuda.Stream()
+    full = bench.Trajectory(w, dev, pcsp=pcsp)
+    with torch.cuda.stream(stream):
+        full.run(stream)
+    stream.synchronize()
+    taken = {}
+    hi = bench.Trajectory(w, dev, heads=(12, 24), reduce_score=lambda s: taken.setdefault("hi", s.clone()), pcsp=pcsp)
+    with torch.cuda.stream(stream):
+        hi.run(stream)
+    stream.synchronize()
+    lo = bench.Trajectory(w, dev, heads=(0, 12), reduce_score=lambda s: s.add_(taken["hi"]), pcsp=pcsp)
+    with torch.cuda.stream(stream):
+        lo.run(stream)
+    stream.synchronize()
+    expect_status(0)
+    sf, sl = full.score.cpu().numpy(), lo.score.cpu().numpy()
+    assert np.abs(sl - sf).max() <= 1e-12 * np.abs(sf).max()
+    tau = np.sort(sf)[::-1][w.k - 1]
+    near = set(np.nonzero(np.abs(sf - tau) <= 1e-6 * abs(tau))[0].tolist())
+    assert set(lo.idx_s.cpu().tolist()) - near == set(full.idx_s.cpu().tolist()) - near
+    if not near:
+        assert torch.equal(lo.idx_s, full.idx_s)
+        assert torch.equal(lo.o_state, full.o_state[:, :12])
