@@ -1152,8 +1152,11 @@ def run_only(args):
     }
     fn, flop, nbytes = fns[args.only]
     times = []
+    flush = L2Flush(dev) if args.flush else None
     with torch.cuda.stream(stream):
         for i in range(args.reps):
+            if flush is not None:
+                flush()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -1163,7 +1166,8 @@ def run_only(args):
     stream.synchronize()
     ms = [a.elapsed_time(b) for a, b in times]
     status = sd.safedit_get_device_status(stream)
-    out = {"only": args.only, "reps": args.reps, "ms": [round(x, 4) for x in ms], "status": status}
+    out = {"only": args.only, "reps": args.reps, "ms": [round(x, 4) for x in ms], "status": status,
+           "l2_flushed": bool(args.flush)}
     if args.only in ("cfg", "stepcache"):
         out["F"] = args.cfg_f
     best = min(ms[1:] if len(ms) > 1 else ms)
@@ -1195,6 +1199,7 @@ def main():
                              "stepcache", "mask", "ffn1", "ffn2", "ffn", "qkv", "sweep", "stress"],
                     help="run one kernel of the path in isolation (profiling target)")
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--flush", action="store_true", help="--only: flush L2 before every rep (outside the events)")
     ap.add_argument("--cfg-f", type=int, default=W.F, help="prediction width for --only cfg")
     args = ap.parse_args()
     if args.only == "sweep":

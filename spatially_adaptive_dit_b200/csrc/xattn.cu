@@ -201,14 +201,18 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_before();
         mbar_arrive(BAR(6 + w));
       }
-#pragma unroll 1
-      for (int c = 0; c < nc; ++c) {
-        if (!((vmask >> c) & 1u)) {
-          // an all-padding chunk: stored from the zero box, no staging
-          if (c * 32 < p.L4 && r == 0) {
+      // all-padding chunks first: stored from the zero box, no staging, so
+      // that those writes overlap the normalise pass below
+      if (r == 0) {
+        for (int c = 0; c < nc; ++c)
+          if (!((vmask >> c) & 1u) && c * 32 < p.L4) {
             tma_store_3d(&tmP, sZero, c * 32, row0, h);
             bulk_commit();
           }
+      }
+#pragma unroll 1
+      for (int c = 0; c < nc; ++c) {
+        if (!((vmask >> c) & 1u)) {
           if (p.L4 < p.L && row0 + r < p.N) {
             for (int j = max(c * 32, p.L4); j < min(c * 32 + 32, p.L); ++j)
               p.P[h * p.p_sh + int64_t(row0 + r) * p.p_sn + j] = 0.f;
