@@ -42,6 +42,24 @@ def test_status_strings_and_counters(sd):
     assert sd.safedit_kernel_launch_count() >= 0
     old = sd.safedit_debug_set_wait_limit_ns(12345)
     assert sd.safedit_debug_set_wait_limit_ns(old) == 12345
+    prev = sd.safedit_debug_set_index_check(True)
+    assert sd.safedit_debug_set_index_check(prev) is True
+
+
+def test_sw_cfg_argument_checks(sd):
+    """Prediction dtypes: both f32 or both bf16; the output is f32."""
+    n, f = 64, 16
+    c32 = _desc(sd, (n, f), (f, 1), sd.F32)
+    c16 = _desc(sd, (n, f), (f, 1), sd.BF16)
+    out = _desc(sd, (n, f), (f, 1), sd.F32)
+    out16 = _desc(sd, (n, f), (f, 1), sd.BF16)
+    call = lambda c, u, o: sd.raw_call("safedit_sw_cfg", ctypes.byref(c), ctypes.byref(u), ctypes.c_void_p(0x20000),
+                                       ctypes.c_float(3.0), ctypes.c_float(5.0), ctypes.byref(o), None)
+    assert call(c32, c16, out) == sd.ERR_DTYPE
+    assert call(c16, c32, out) == sd.ERR_DTYPE
+    assert call(c16, c16, out16) == sd.ERR_DTYPE
+    wide = _desc(sd, (n, f), (f, 2), sd.BF16)
+    assert call(wide, c16, out) == sd.ERR_ALIGNMENT
 
 
 def _desc(sd, dims, strides, dtype, ptr=0x10000):
