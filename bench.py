@@ -237,6 +237,13 @@ class Trajectory:
         self.eps_c, self.eps_u = wl.cfg_preds(w, step=seed_step, device=dev)
         self.cfg_out = torch.empty_like(self.eps_c)
         self.H = H
+        # tail-balanced attention: one workspace per launch shape (S rows,
+        # all rows), as large as the launch plan asks (none where it keeps
+        # whole units, as at 2560^2)
+        self.attn_ws = {}
+        for rows in (k, N):
+            nb = sd.safedit_attn_subset_workspace_size(B, H, rows, N, d)
+            self.attn_ws[rows] = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
         self.flop_srsu = 4.0 * k * N * d * B * H
         self.flop_dense = 4.0 * N * N * d * B * H
         self.bytes = {
@@ -248,6 +255,12 @@ class Trajectory:
             "scatter_state": 2 * (2 * B * H * k * d * 2) + 4 * k,
             "sw_cfg": 3 * N * w.F * 4 + 4 * N,
         }
+
+    def attn(self, q, k_state, v_state, idx, n_idx, out, scattered, stream):
+        """One attention launch through the tail-balanced entry point."""
+        rows = n_idx if idx is not None else q.shape[2]
+        self.sd.safedit_attn_subset_ws(q, k_state, v_state, idx, n_idx, None, None, 0.0, out, scattered,
+                                       self.attn_ws[rows], stream)
 
     def run(self, stream, ev=None, flush=None):
         """Enqueue one trajectory on `stream`.  ev: dict name -> list to which
@@ -292,15 +305,13 @@ class Trajectory:
                 # CAR: fresh K/V become the cached state (buffer swap), dense refresh of all rows
                 self.k_state, self.k_full = self.k_full, self.k_state
                 self.v_state, self.v_full = self.v_full, self.v_state
-                timed("attn_dense_anchor", lambda: sd.safedit_attn_subset(
-                    self.q, self.k_state, self.v_state, None, 0, None, None, 0.0, self.o_state, 0,
-                    stream))
+                timed("attn_dense_anchor", lambda: self.attn(
+                    self.q, self.k_state, self.v_state, None, 0, self.o_state, 0, stream))
             else:
                 timed("scatter_state", lambda: sd.safedit_scatter_state(
                     [self.k_s, self.v_s], [self.k_state, self.v_state], self.idx_s, self.k, stream))
-                timed("attn_subset_srsu", lambda: sd.safedit_attn_subset(
-                    self.q, self.k_state, self.v_state, self.idx_s, self.k, None, None, 0.0,
-                    self.o_state, 1, stream))
+                timed("attn_subset_srsu", lambda: self.attn(
+                    self.q, self.k_state, self.v_state, self.idx_s, self.k, self.o_state, 1, stream))
             g_ctx = w.gamma_ctx
             g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx  # global CFG before the split
             timed("sw_cfg", lambda: sd.safedit_sw_cfg(self.eps_c, self.eps_u, self.s, g_ctx, g_sens,
@@ -536,7 +547,7 @@ def measure_extensions(tr, stream, dev, unfused_pcsp_ms):
         for name, t in ms.items()}
     out["kept_mask_stress"]["workload"] = (
         f"B=1, H=32, N={wl.STRESS.N}, d=128, |S|={wl.STRESS.k} (blob scores); padding = trailing 1/8 of the keys "
-        "at -inf; bias = [1,1,N,N] N(0,1) in bf16 or f32; the five launches taken in turn within every rep")
+        "at -inf; bias = [1,1,N,N] N(0,1) in bf16 or f32; the six launches taken in turn within every rep")
     del cases
     torch.cuda.empty_cache()
     out["config_1024"] = measure_1024(sd, dev, stream, flush)
@@ -564,10 +575,11 @@ def measure_1024(sd, dev, stream, flush):
         tr.run(stream)  # fills the split, the state and the scores
     stream.synchronize()
     t = {
-        "attn_subset_srsu": time_reps(lambda: sd.safedit_attn_subset(
-            tr.q, tr.k_state, tr.v_state, tr.idx_s, tr.k, None, None, 0.0, tr.o_state, 1, stream), stream,
-            flush=flush),
-        "attn_dense_anchor": time_reps(lambda: sd.safedit_attn_subset(
+        "attn_subset_srsu": time_reps(lambda: tr.attn(
+            tr.q, tr.k_state, tr.v_state, tr.idx_s, tr.k, tr.o_state, 1, stream), stream, flush=flush),
+        "attn_dense_anchor": time_reps(lambda: tr.attn(
+            tr.q, tr.k_state, tr.v_state, None, 0, tr.o_state, 0, stream), stream, flush=flush),
+        "attn_dense_anchor_whole_units": time_reps(lambda: sd.safedit_attn_subset(
             tr.q, tr.k_state, tr.v_state, None, 0, None, None, 0.0, tr.o_state, 0, stream), stream, flush=flush),
         "pcsp_score": time_reps(lambda: sd.safedit_pcsp_score(
             tr.q_img, tr.k_txt, tr.valid, tr.content, 0, 0.0, tr.score, stream), stream, flush=flush),
@@ -582,7 +594,8 @@ def measure_1024(sd, dev, stream, flush):
         "sw_cfg": time_reps(lambda: sd.safedit_sw_cfg(
             tr.eps_c, tr.eps_u, tr.s, w.gamma_ctx, w.gamma_sens, tr.cfg_out, stream), stream, flush=flush),
     }
-    for name, flop in (("attn_subset_srsu", tr.flop_srsu), ("attn_dense_anchor", tr.flop_dense)):
+    for name, flop in (("attn_subset_srsu", tr.flop_srsu), ("attn_dense_anchor", tr.flop_dense),
+                       ("attn_dense_anchor_whole_units", tr.flop_dense)):
         tf = flop / (t[name]["p50"] * 1e-3) / 1e12
         t[name].update({"tflops": round(tf, 1), "frac_of_burst": round(tf / bf16_burst, 3)})
     for name, nbytes in tr.bytes.items():
@@ -803,11 +816,11 @@ def run_e2e(tr, stream, args):
                     sd.safedit_mask_is_row_constant(tr.mask, tr.verdict, None, stream)
                 if anchor:
                     eps_c, eps_u = a_c, a_u
-                    sd.safedit_attn_subset(aq, k_st, v_st, None, 0, None, None, 0.0, tr.o_state, 0, stream)
+                    tr.attn(aq, k_st, v_st, None, 0, tr.o_state, 0, stream)
                 else:
                     qs, ks, vs, eps_c, eps_u = sets[t % NSET][1]
                     sd.safedit_scatter_state([ks, vs], [k_st, v_st], tr.idx_s, tr.k, stream)
-                    sd.safedit_attn_subset(qs, k_st, v_st, None, 0, None, None, 0.0, o_s, 0, stream)
+                    tr.attn(qs, k_st, v_st, None, 0, o_s, 0, stream)
                     sd.safedit_scatter_state([o_s], [tr.o_state], tr.idx_s, tr.k, stream)
                 g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx
                 sd.safedit_sw_cfg(eps_c, eps_u, tr.s, w.gamma_ctx, g_sens, tr.cfg_out, stream)
@@ -958,9 +971,10 @@ def run_reference(args):
 def stress_srsu_cases(sd, dev, stream):
     """The SRSU launches of the mask-stress workload (B=1, H=32, N=16384,
     d=128, |S|=4915 from the clustered blob scores): mask elided (no mask
-    input), kept text-padding key mask (trailing 1/8 of the keys -inf), kept
-    non-uniform bias [1,1,N,N] in bf16, both, and the bias in f32.  Returns
-    the launch closures (name -> fn) and the flop of one call."""
+    input; whole units, and tail-balanced), kept text-padding key mask
+    (trailing 1/8 of the keys -inf), kept non-uniform bias [1,1,N,N] in bf16,
+    both, and the bias in f32.  Returns the launch closures (name -> fn) and
+    the flop of one call."""
     w = wl.STRESS
     q, k, v = wl.qkv(w, device=dev)
     o = torch.zeros_like(q)
@@ -972,8 +986,12 @@ def stress_srsu_cases(sd, dev, stream):
     bias = wl.mask(w, "bias", device=dev)            # [1,1,N,N] bf16
     bias32 = bias.float()                            # the same bias in f32 (1.07 GB)
     att = lambda kp, bb: (lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, kp, bb, 0.0, o, 1, stream))
+    nb = sd.safedit_attn_subset_workspace_size(w.B, w.H, w.k, w.N, w.d)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)  # 640 units = 4 waves + 48 split in 3
     cases = {
         "srsu_mask_elided": att(None, None),
+        "srsu_mask_elided_tail_split": lambda: sd.safedit_attn_subset_ws(q, k, v, idx, w.k, None, None, 0.0, o, 1,
+                                                                        ws, stream),
         "srsu_kept_padding": att(pad, None),
         "srsu_kept_bias": att(None, bias),
         "srsu_kept_padding_and_bias": att(pad, bias),

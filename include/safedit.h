@@ -209,6 +209,54 @@ safedit_status safedit_attn_subset(const safedit_tensor *q,
                                    int32_t out_scattered, void *stream);
 
 /* ------------------------------------------------------------------------
+ * The same attention with the tail of the launch balanced over the SMs (a
+ * scheduling choice of this library: the pages define only the result,
+ * the SRSU rows over all keys of [P1 방법론 3]).  The work is cut into
+ * units of 256 query rows of one (b, h) slice.  When the units do not fill
+ * the last wave of the GPU's SMs, each of those last units may run as
+ * s = 2..4 parts over the key tiles: the whole units run first as one
+ * launch (a whole number of waves), the parts as a second launch that may
+ * start while the first one's last wave drains (programmatic dependent
+ * launch; it completes only after the first), writing their unnormalised
+ * output rows, running max and row sum (f32) to d_workspace, and a merge
+ * kernel then combines them into the output rows (the online-softmax merge;
+ * the result equals safedit_attn_subset's within the attention tolerance,
+ * not bit for bit).  The plan takes a split only where a per-CTA cost model
+ * (set-up + per-key-tile time measured on B200) predicts a saving of at
+ * least 3% of the call; otherwise, and for launches with kept masks
+ * (key_pad or bias), the call is safedit_attn_subset.  All launches go on
+ * `stream`, in order, so the call is stream-ordered like the others.
+ *
+ * Arguments as safedit_attn_subset, plus d_workspace / workspace_bytes:
+ * device memory of at least safedit_attn_subset_workspace_size(...) bytes
+ * for this call on the current device, 16-byte aligned (else
+ * SAFEDIT_ERR_ALIGNMENT), owned by the caller, not read before it is
+ * written; NULL is allowed when that size is 0.  A smaller workspace returns
+ * SAFEDIT_ERR_INVALID_ARG before any launch.  Calls that share a workspace
+ * must not overlap on the GPU.
+ */
+safedit_status safedit_attn_subset_ws(const safedit_tensor *q,
+                                      const safedit_tensor *k,
+                                      const safedit_tensor *v,
+                                      const int32_t *d_idx, int32_t n_idx,
+                                      const safedit_tensor *key_pad,
+                                      const safedit_tensor *bias, float scale,
+                                      const safedit_tensor *out,
+                                      int32_t out_scattered,
+                                      void *d_workspace, size_t workspace_bytes,
+                                      void *stream);
+
+/* Workspace bytes safedit_attn_subset_ws needs on the current device (its
+ * SM count enters the plan) for batch x heads slices of n_rows query rows
+ * over n_keys keys of head_dim (64, 96 or 128): (split units) x s x 256 x
+ * (head_dim + 2) x 4.  kept_masks != 0 for a call with key_pad or bias
+ * (never split: 0 bytes); 0 also when the plan keeps whole units.  Host
+ * only, no launch; invalid sizes give 0. */
+size_t safedit_attn_subset_workspace_size(int64_t batch, int64_t heads,
+                                          int64_t n_rows, int64_t n_keys,
+                                          int32_t head_dim, int32_t kept_masks);
+
+/* ------------------------------------------------------------------------
  * State scatter.  [P1 방법론 3 / P4 Metodologia 3]: context states are cached
  * and reused between anchors; fresh sensitive rows replace their entries.
  *

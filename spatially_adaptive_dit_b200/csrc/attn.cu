@@ -82,6 +82,14 @@ struct AttnParams {
   int out_scattered;
   int* status;
   uint64_t wait_limit;
+  // Schedule: unit u = (row block u % n_rb, slice u / n_rb) of 256 query rows.
+  // Units below n_full run whole (one launch, a whole number of waves when
+  // split); every later unit runs as `split` CTAs of a second launch over
+  // consecutive parts of the key tiles, which write their unnormalised O,
+  // running max and row sum to `part` for attn_merge_kernel.
+  int n_rb, n_full, split;
+  float* part;  // [(unit - n_full) * split + part][256][D] O, then [..][256][2] (m, l)
+  int n_part_units;
 };
 
 // 12 warps: two softmax warpgroups (warps 0-7), then TMA producer (8), MMA
@@ -170,7 +178,7 @@ __device__ __forceinline__ void stage_bias(uint32_t buf, const T* base, int64_t 
   cp_async_commit();
 }
 
-template <int D, bool PAD, int BIAS>
+template <int D, bool PAD, int BIAS, bool SPLIT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_subset_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -193,10 +201,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
+  // whole units: 2D grid (x: row block, y: slice), units from n_full on left
+  // to the part launch; parts: CTA i runs part i % split of unit
+  // n_full + i / split (recomputed where needed rather than kept live
+  // through the main loop).  A whole-unit CTA lets a dependent launch (the
+  // parts, which read only what it reads) start as soon as it is resident,
+  // so the parts fill the SMs its last wave frees.
+  if constexpr (!SPLIT) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (!SPLIT && int(blockIdx.y) * p.n_rb + int(blockIdx.x) >= p.n_full) return;
+  auto decode = [&](int& unit_out, int& kpart_out) {
+    if (SPLIT) {
+      unit_out = p.n_full + int(blockIdx.x) / p.split;
+      kpart_out = int(blockIdx.x) - (int(blockIdx.x) / p.split) * p.split;
+    } else {
+      unit_out = int(blockIdx.y) * p.n_rb + int(blockIdx.x);
+      kpart_out = -1;
+    }
+  };
+  int unit, kpart;
+  decode(unit, kpart);
+  const int bh = SPLIT ? unit / p.n_rb : int(blockIdx.y);
   const int b = bh / p.H, h = bh - b * p.H;
-  const int row0 = blockIdx.x * 256;
+  const int row0 = SPLIT ? (unit - bh * p.n_rb) * 256 : int(blockIdx.x) * 256;
   const int nk = (p.Nk + C::BN - 1) / C::BN;
+  // this CTA's key tiles [k_lo, k_hi) (kept-padding launches are never split)
+  const int k_lo = !SPLIT || kpart < 0 ? 0 : int(int64_t(nk) * kpart / p.split);
+  const int k_hi = !SPLIT || kpart < 0 ? nk : int(int64_t(nk) * (kpart + 1) / p.split);
   // live key tiles (kept key padding): a tile whose pad entries are all -inf
   // adds nothing to any row (its weights are exactly zero) and is skipped by
   // every role; every role walks the same bitmask, so they agree on the
@@ -235,7 +265,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     return nk;
   };
   auto live_count = [&]() -> int {
-    if (!skip_tiles) return nk;
+    if (!skip_tiles) return k_hi - k_lo;
     int n = 0;
     for (int w = 0; w < (nk + 31) / 32; ++w) n += __popc(live_word(w));
     return n;
@@ -338,7 +368,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float* const pad_row = PAD ? p.pad + b * p.pad_sb : nullptr;
     float4 pad_next = make_float4(0.f, 0.f, 0.f, 0.f);
     const int n_live = live_count();
-    int j_first = next_live(0);
+    int j_first = next_live(k_lo);
     if constexpr (PAD) pad_next = load_pad4(pad_row, j_first * C::BN + 4 * lane, p.Nk);
     using BiasT = typename std::conditional<BIAS == kBiasF32, float, __nv_bfloat16>::type;
     const BiasT* const bias_bh =
@@ -579,17 +609,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       pad_slot = (pad_slot == 2) ? 0 : pad_slot + 1;
     }
     if constexpr (BIAS != kBiasNone) cp_async_wait_all();  // none in flight at exit
-    // ---- epilogue: O / l -> bf16 rows
+    // ---- epilogue: O / l -> bf16 rows; for a key-range part of a split
+    // unit, the unnormalised O, running max and row sum for the merge
     if (ok && wait_warp(BAR(O_FULL), 0u, ctl)) {
       tc_fence_after();
+      int e_unit, e_part;
+      decode(e_unit, e_part);
+      const bool partial = SPLIT && e_part >= 0;
       const bool live = my_q >= 0;
-      if (live && !(l_run > 0.f)) set_status(p.status, SAFEDIT_ERR_MASKED_ROW);
+      if (live && !partial && !(l_run > 0.f)) set_status(p.status, SAFEDIT_ERR_MASKED_ROW);
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
       // with skipped key tiles O may never have been written: a row with no
       // weight (fully masked: an error, reported above) is written as zeros
       const bool zero_row = PAD && !(l_run > 0.f);
+      const int64_t slot = int64_t(e_unit - p.n_full) * p.split + e_part;
+      const int rr = t * 128 + wr * 32 + lane;
       __nv_bfloat16* orow = nullptr;
-      if (live) {
+      float* po = nullptr;
+      if (live && partial) {
+        po = p.part + (slot * 256 + rr) * D;
+      } else if (live) {
         const int64_t orow_idx = p.out_scattered ? int64_t(my_q) : int64_t(my_row);
         orow = p.out + b * p.o_sb + h * p.o_sh + orow_idx * p.o_sr;
       }
@@ -598,7 +637,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t r[32];
         tmem_ld32(tO + uint32_t(c * 32), r);
         tmem_wait_ld();
-        if (live) {
+        if (live && partial) {
+          float4* dst = reinterpret_cast<float4*>(po + c * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                 __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+        } else if (live) {
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
@@ -611,6 +656,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
         }
       }
+      if (live && partial) {
+        float* const pml = p.part + int64_t(p.n_part_units) * p.split * 256 * D + (slot * 256 + rr) * 2;
+        pml[0] = m_run;
+        pml[1] = l_run;
+      }
     }
   } else {
     setmaxnreg_dec<MASKED ? kControlRegsMasked : kControlRegs>();
@@ -619,7 +669,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (lane == 0) {
         int issued_k = 0, issued_v = 0;
         const int n_live = live_count();
-        for (int it = 0, kt = next_live(0); it < n_live; ++it, kt = next_live(kt + 1)) {
+        for (int it = 0, kt = next_live(k_lo); it < n_live; ++it, kt = next_live(kt + 1)) {
           const int s = it % C::NS;
           const uint32_t ph = uint32_t((it / C::NS) & 1);
           if (!wait_bounded(BAR(K_EMPTY + s), ph ^ 1u, ctl)) break;
@@ -729,19 +779,143 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // the part launch may overlap the whole-unit launch before it: its last CTA
+  // leaves only once that launch has completed, so whatever follows in the
+  // stream (the merge, then the caller's work) runs after both
+  if constexpr (SPLIT) {
+    if (threadIdx.x == 0 && blockIdx.x == gridDim.x - 1) asm volatile("griddepcontrol.wait;" ::: "memory");
+  }
 }
 
-template <int D, bool PAD, int BIAS>
+// Combines the key-range parts of the split units: per query row,
+// m = max m_i, l = sum 2^(m_i - m) l_i, o = sum 2^(m_i - m) O_i / l (the same
+// online-softmax merge the kernel applies between key tiles), written as a
+// bf16 row where the whole unit would have written it.  One warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const AttnParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= int64_t(p.n_part_units) * 256) return;
+  const int pu = int(row >> 8), rr = int(row & 255);
+  const int unit = p.n_full + pu;
+  const int bh = unit / p.n_rb;
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int my_row = (unit - bh * p.n_rb) * 256 + rr;
+  if (my_row >= p.n_rows) return;
+  const int my_q = p.idx ? __ldg(p.idx + my_row) : my_row;
+  if (my_q < 0 || my_q >= p.Nq) return;  // reported by the attention kernel
+  const float* ml = p.part + int64_t(p.n_part_units) * p.split * 256 * D;
+  float m = -INFINITY;
+  for (int k = 0; k < p.split; ++k) m = fmaxf(m, ml[((int64_t(pu) * p.split + k) * 256 + rr) * 2]);
+  float l = 0.f, acc[D / 32];
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
+  for (int k = 0; k < p.split; ++k) {
+    const int64_t slot = int64_t(pu) * p.split + k;
+    const float w = exp2f(ml[(slot * 256 + rr) * 2] - m);
+    l = fmaf(w, ml[(slot * 256 + rr) * 2 + 1], l);
+    const float* po = p.part + (slot * 256 + rr) * D;
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(w, po[lane + 32 * e], acc[e]);
+  }
+  const float inv = 1.f / l;
+  const int64_t orow_idx = p.out_scattered ? int64_t(my_q) : int64_t(my_row);
+  __nv_bfloat16* orow = p.out + b * p.o_sb + h * p.o_sh + orow_idx * p.o_sr;
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) orow[lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
+}
+
+// Launch plan: units of 256 query rows, longest first.  When the units do
+// not fill the last wave of the SMs, those last units are each split into
+// s = 2..4 parts over the key tiles, run after the whole units (which then
+// fill a whole number of waves).  A CTA costs about kFixedUs (set-up, TMEM,
+// epilogue) plus kTileUs per key tile of 128 at d = 96 (measured on B200,
+// one full wave, 1280..25600 keys; scaled by d / 96 for other widths).  The
+// tail's ceil(tail s / SMs) rounds of 1/s units plus the merge must save 3%
+// of the whole launch (its rounds of whole units) for a split to be taken:
+// smaller predicted savings did not show on B200, where a power-capped
+// launch runs its other SMs faster while the last round leaves some idle.
+struct AttnPlan {
+  int n_rb = 0, n_units = 0, n_full = 0, split = 1, n_part_units = 0;
+  size_t ws_bytes = 0;
+};
+
+static int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    sms = 148;
+  return sms;
+}
+
+static AttnPlan plan_attn(int64_t n_rows, int64_t BH, int64_t Nk, int D, bool splittable, int sms) {
+  AttnPlan pl;
+  pl.n_rb = int((n_rows + 255) / 256);
+  pl.n_units = int(pl.n_rb * BH);
+  pl.n_full = pl.n_units;
+  const int64_t nk = (Nk + 127) / 128;
+  const int tail = pl.n_units % sms;
+  if (!splittable || tail == 0 || nk < 8) return pl;
+  constexpr double kFixedUs = 11.6, kTileUs = 1.83, kMergeUs = 8.0;
+  const double tile_us = kTileUs * D / 96.0;
+  const double unit_us = kFixedUs + double(nk) * tile_us;
+  const double rounds_whole = double((pl.n_units + sms - 1) / sms);
+  double best = unit_us - 0.03 * rounds_whole * unit_us;
+  for (int s = 2; s <= 4; ++s) {
+    const double rounds = double((int64_t(tail) * s + sms - 1) / sms);
+    const double cost = rounds * (kFixedUs + double(nk) * tile_us / s) + kMergeUs;
+    if (cost < best) {
+      best = cost;
+      pl.split = s;
+    }
+  }
+  if (pl.split == 1) return pl;
+  pl.n_part_units = tail;
+  pl.n_full = pl.n_units - tail;
+  pl.ws_bytes = size_t(tail) * size_t(pl.split) * 256u * size_t(D + 2) * sizeof(float);
+  return pl;
+}
+
+template <int D, bool PAD, int BIAS, bool SPLIT = false>
 static safedit_status launch_attn(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                   const AttnParams& p, int B, cudaStream_t stream) {
   using C = AttnCfg<D>;
-  auto kern = attn_subset_kernel<D, PAD, BIAS>;
+  auto kern = attn_subset_kernel<D, PAD, BIAS, SPLIT>;
   constexpr int smem_bytes =
       C::SMEM_BYTES + (BIAS != kBiasNone ? C::BIAS_BYTES : 0) + (PAD ? C::PAD_BYTES : 0);
   safedit_status st = set_smem(reinterpret_cast<const void*>(kern), smem_bytes);
   if (st != SAFEDIT_OK) return st;
-  dim3 grid((p.n_rows + 255) / 256, B * p.H);
-  kern<<<grid, kAttnThreads, smem_bytes, stream>>>(tmK, tmV, p);
+  if (SPLIT) {
+    // programmatic serialization after the whole-unit launch (when there is
+    // one): the parts may start while its last wave drains
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(p.n_part_units * p.split));
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.n_full > 0 ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, tmK, tmV, p) != cudaSuccess) return SAFEDIT_ERR_CUDA;
+  } else {
+    (void)B;
+    dim3 grid(p.n_rb, (p.n_full + p.n_rb - 1) / p.n_rb);
+    kern<<<grid, kAttnThreads, smem_bytes, stream>>>(tmK, tmV, p);
+  }
+  return after_launch(1);
+}
+
+// A split plan: the whole units (a whole number of waves), then the parts of
+// the last units, then their merge, in stream order.
+template <int D>
+static safedit_status launch_attn_split(const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                        const AttnParams& p, int B, cudaStream_t stream) {
+  safedit_status st = SAFEDIT_OK;
+  if (p.n_full > 0 && (st = launch_attn<D, false, kBiasNone>(tmK, tmV, p, B, stream)) != SAFEDIT_OK) return st;
+  if ((st = launch_attn<D, false, kBiasNone, true>(tmK, tmV, p, B, stream)) != SAFEDIT_OK) return st;
+  attn_merge_kernel<D><<<(p.n_part_units * 256 + 7) / 8, 256, 0, stream>>>(p);
   return after_launch(1);
 }
 
@@ -757,6 +931,7 @@ static safedit_status dispatch_attn(const CUtensorMap& tmK, const CUtensorMap& t
   }
   if (bias == kBiasBf16) return launch_attn<D, false, kBiasBf16>(tmK, tmV, p, B, s);
   if (bias == kBiasF32) return launch_attn<D, false, kBiasF32>(tmK, tmV, p, B, s);
+  if (p.n_part_units > 0) return launch_attn_split<D>(tmK, tmV, p, B, s);
   return launch_attn<D, false, kBiasNone>(tmK, tmV, p, B, s);
 }
 
@@ -786,12 +961,14 @@ static safedit_status make_kv_map(CUtensorMap* m, const safedit_tensor* t, int D
 
 using namespace sd;
 
-extern "C" safedit_status safedit_attn_subset(const safedit_tensor* q, const safedit_tensor* k,
-                                              const safedit_tensor* v, const int32_t* d_idx,
-                                              int32_t n_idx, const safedit_tensor* key_pad,
-                                              const safedit_tensor* bias, float scale,
-                                              const safedit_tensor* out, int32_t out_scattered,
-                                              void* stream) {
+// Shared body of safedit_attn_subset (ws == NULL: whole units only) and
+// safedit_attn_subset_ws (the tail of the launch split over the keys when
+// the plan asks for it and the workspace holds the partial results).
+static safedit_status attn_subset_impl(const safedit_tensor* q, const safedit_tensor* k,
+                                       const safedit_tensor* v, const int32_t* d_idx, int32_t n_idx,
+                                       const safedit_tensor* key_pad, const safedit_tensor* bias,
+                                       float scale, const safedit_tensor* out, int32_t out_scattered,
+                                       void* d_ws, size_t ws_bytes, bool use_ws, void* stream) {
   safedit_status st;
   if ((st = check_bhnd(q)) != SAFEDIT_OK) return st;
   if ((st = check_bhnd(k)) != SAFEDIT_OK) return st;
@@ -807,6 +984,7 @@ extern "C" safedit_status safedit_attn_subset(const safedit_tensor* q, const saf
   if (out_scattered != 0 && out_scattered != 1) return SAFEDIT_ERR_INVALID_ARG;
   if (d_idx && n_idx < 0) return SAFEDIT_ERR_INVALID_ARG;
   const int64_t n_rows = d_idx ? n_idx : Nq;
+  if ((n_rows + 255) / 256 * B * H > INT32_MAX) return SAFEDIT_ERR_SHAPE;  // units counted in int
   if (out->dims[0] != B || out->dims[1] != H || out->dims[3] != D) return SAFEDIT_ERR_SHAPE;
   if (out_scattered ? (out->dims[2] != Nq) : (out->dims[2] != n_rows)) return SAFEDIT_ERR_SHAPE;
   AttnParams p{};
@@ -835,7 +1013,17 @@ extern "C" safedit_status safedit_attn_subset(const safedit_tensor* q, const saf
     p.bias_sh = bias->dims[1] == 1 ? 0 : bias->strides[1];
     p.bias_sq = bias->strides[2];
   }
+  AttnPlan pl = plan_attn(n_rows, B * H, Nk, int(D), use_ws && !key_pad && !bias, sm_count());
+  if (use_ws && pl.ws_bytes > 0) {
+    if (!d_ws || ws_bytes < pl.ws_bytes) return SAFEDIT_ERR_INVALID_ARG;
+    if (!aligned16(d_ws)) return SAFEDIT_ERR_ALIGNMENT;
+  }
   if (n_rows == 0 || B * H == 0) return SAFEDIT_OK;
+  p.n_rb = pl.n_rb;
+  p.n_full = pl.n_full;
+  p.split = pl.split;
+  p.n_part_units = pl.n_part_units;
+  p.part = static_cast<float*>(d_ws);
   p.q = static_cast<const __nv_bfloat16*>(q->data);
   p.q_sb = q->strides[0];
   p.q_sh = q->strides[1];
@@ -868,4 +1056,35 @@ extern "C" safedit_status safedit_attn_subset(const safedit_tensor* q, const saf
     case 96: return dispatch_attn<96>(tmK, tmV, p, static_cast<int>(B), s);
     default: return dispatch_attn<128>(tmK, tmV, p, static_cast<int>(B), s);
   }
+}
+
+extern "C" safedit_status safedit_attn_subset(const safedit_tensor* q, const safedit_tensor* k,
+                                              const safedit_tensor* v, const int32_t* d_idx,
+                                              int32_t n_idx, const safedit_tensor* key_pad,
+                                              const safedit_tensor* bias, float scale,
+                                              const safedit_tensor* out, int32_t out_scattered,
+                                              void* stream) {
+  return attn_subset_impl(q, k, v, d_idx, n_idx, key_pad, bias, scale, out, out_scattered, nullptr, 0,
+                          false, stream);
+}
+
+extern "C" safedit_status safedit_attn_subset_ws(const safedit_tensor* q, const safedit_tensor* k,
+                                                 const safedit_tensor* v, const int32_t* d_idx,
+                                                 int32_t n_idx, const safedit_tensor* key_pad,
+                                                 const safedit_tensor* bias, float scale,
+                                                 const safedit_tensor* out, int32_t out_scattered,
+                                                 void* d_workspace, size_t workspace_bytes,
+                                                 void* stream) {
+  return attn_subset_impl(q, k, v, d_idx, n_idx, key_pad, bias, scale, out, out_scattered, d_workspace,
+                          workspace_bytes, true, stream);
+}
+
+extern "C" size_t safedit_attn_subset_workspace_size(int64_t batch, int64_t heads, int64_t n_rows,
+                                                     int64_t n_keys, int32_t head_dim, int32_t kept_masks) {
+  if (batch <= 0 || heads <= 0 || n_rows <= 0 || n_keys <= 0) return 0;
+  if (head_dim != 64 && head_dim != 96 && head_dim != 128) return 0;
+  if (batch * heads > 65535 || n_rows > INT32_MAX || n_keys > INT32_MAX ||
+      (n_rows + 255) / 256 * batch * heads > INT32_MAX)
+    return 0;
+  return plan_attn(n_rows, batch * heads, n_keys, head_dim, kept_masks == 0, sm_count()).ws_bytes;
 }

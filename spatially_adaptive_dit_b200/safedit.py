@@ -31,6 +31,7 @@ _DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16, torch.bo
 
 EXPORTED = ("safedit_cross_attn_probs", "safedit_partition_accumulate", "safedit_pcsp_score",
             "safedit_partition_finalize", "safedit_mask_is_row_constant", "safedit_attn_subset",
+            "safedit_attn_subset_ws", "safedit_attn_subset_workspace_size",
             "safedit_scatter_state", "safedit_gather_rows", "safedit_sw_cfg", "safedit_stepcache_sw_cfg",
             "safedit_gemm_bias_act", "safedit_get_device_status", "safedit_status_string", "safedit_kernel_launch_count",
             "safedit_debug_set_wait_limit_ns", "safedit_debug_set_index_check")
@@ -58,6 +59,10 @@ _lib.safedit_partition_finalize.argtypes = [_vp, _i32, _i32, _vp, _vp, _vp, _vp]
 _lib.safedit_pcsp_score.argtypes = [_T, _T, _vp, _vp, _i32, _f32, _vp, _vp]
 _lib.safedit_mask_is_row_constant.argtypes = [_T, _vp, _vp, _vp]
 _lib.safedit_attn_subset.argtypes = [_T, _T, _T, _vp, _i32, _T, _T, _f32, _T, _i32, _vp]
+_lib.safedit_attn_subset_ws.argtypes = [_T, _T, _T, _vp, _i32, _T, _T, _f32, _T, _i32, _vp, ctypes.c_size_t, _vp]
+_lib.safedit_attn_subset_workspace_size.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                                    _i32, _i32]
+_lib.safedit_attn_subset_workspace_size.restype = ctypes.c_size_t
 _lib.safedit_scatter_state.argtypes = [_T, _T, _i32, _vp, _i32, _vp]
 _lib.safedit_gather_rows.argtypes = [_T, _T, _i32, _vp, _i32, _vp]
 _lib.safedit_sw_cfg.argtypes = [_T, _T, _vp, _f32, _f32, _T, _vp]
@@ -73,7 +78,8 @@ _lib.safedit_debug_set_index_check.argtypes = [ctypes.c_int32]
 _lib.safedit_debug_set_index_check.restype = ctypes.c_int32
 for _n in EXPORTED:
     if _n not in ("safedit_status_string", "safedit_kernel_launch_count",
-                  "safedit_debug_set_wait_limit_ns", "safedit_debug_set_index_check"):
+                  "safedit_debug_set_wait_limit_ns", "safedit_debug_set_index_check",
+                  "safedit_attn_subset_workspace_size"):
         getattr(_lib, _n).restype = ctypes.c_int
 
 
@@ -163,6 +169,22 @@ def safedit_attn_subset(q, k, v, idx, n_idx, key_pad, bias, scale, out, out_scat
     _check(_lib.safedit_attn_subset(_ref(q), _ref(k), _ref(v), _idx_ptr(idx), int(n_idx), _ref(key_pad),
                                     _ref(bias), float(scale), _ref(out), int(out_scattered),
                                     _stream(stream)), "safedit_attn_subset")
+
+
+def safedit_attn_subset_ws(q, k, v, idx, n_idx, key_pad, bias, scale, out, out_scattered, workspace,
+                           stream=None):
+    """workspace: a device tensor of at least safedit_attn_subset_workspace_size(...)
+    bytes, or None when that size is 0."""
+    ptr = None if workspace is None else workspace.data_ptr()
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.safedit_attn_subset_ws(_ref(q), _ref(k), _ref(v), _idx_ptr(idx), int(n_idx), _ref(key_pad),
+                                       _ref(bias), float(scale), _ref(out), int(out_scattered), ptr, nbytes,
+                                       _stream(stream)), "safedit_attn_subset_ws")
+
+
+def safedit_attn_subset_workspace_size(batch, heads, n_rows, n_keys, head_dim, kept_masks=False) -> int:
+    return int(_lib.safedit_attn_subset_workspace_size(int(batch), int(heads), int(n_rows), int(n_keys),
+                                                       int(head_dim), 1 if kept_masks else 0))
 
 
 def _desc_array(ts):

@@ -179,3 +179,30 @@ def test_bandwidth_kernels_host_validation(sd):
     xp3 = _desc(sd, (2, 256, 30), (256 * 30, 30, 1), sd.F32)
     xk3 = _bhnd(sd, 2, 2, 30, 64)
     assert x(R(xq), R(xk3), ctypes.c_void_p(0x80000), 0, 0.0, R(xp3), None) == sd.ERR_ALIGNMENT
+
+
+def test_attention_tail_split_plan(sd):
+    """Workspace the tail-balanced attention needs (148 SMs): the units that do
+    not fill the last wave are split over the keys into the s in 2..4 that
+    ends the call soonest by the per-CTA cost model (11.6 us + 1.83 us per key
+    tile at d = 96), when that saves 3% of the whole launch; each split unit
+    keeps s x 256 rows of (d + 2) f32."""
+    ws = sd.safedit_attn_subset_workspace_size
+    row = lambda d: 256 * (d + 2) * 4
+    # 2560^2 SRSU: 30 x 48 = 1440 units = 9 waves + 108; 108 units x 4 parts
+    # (3 rounds of 1/4) would save 61 us of 10 rounds x 378 us: under 3%
+    assert ws(2, 24, 7680, 25600, 96) == 0
+    # 2560^2 anchor: 100 x 48 = 4800 = 32 waves + 64; 64 x 2 saves 1.4%
+    assert ws(2, 24, 25600, 25600, 96) == 0
+    # 1024^2 SRSU: 5 x 48 = 240 = 1 wave + 92 units of 32 key tiles: two
+    # rounds of 1/3 + the merge (70 us) do not beat one whole round (70 us)
+    assert ws(2, 24, 1229, 4096, 96) == 0
+    # 1024^2 anchor: 16 x 48 = 768 = 5 waves + 28 -> 28 x 4 (one round of 1/4)
+    assert ws(2, 24, 4096, 4096, 96) == 28 * 4 * row(96)
+    # stress SRSU: 20 x 32 = 640 = 4 waves + 48 -> 48 x 3 (one round of 1/3)
+    assert ws(1, 32, 4915, 16384, 128) == 48 * 3 * row(128)
+    # no tail, kept masks, or too few key tiles to split: nothing
+    assert ws(1, 148, 256, 25600, 96) == 0
+    assert ws(2, 24, 7680, 25600, 96, kept_masks=True) == 0
+    assert ws(1, 2, 64, 256, 64) == 0
+    assert ws(0, 2, 64, 256, 64) == 0 and ws(1, 2, 64, 4096, 80) == 0

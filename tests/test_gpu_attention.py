@@ -350,3 +350,105 @@ def test_config_2560_dense_anchor_as_benchmarked():
     for (b, h) in [(0, 3), (1, 20)]:
         ref = oracle.attn_dense(f64(q[b, h, rt]), f64(k[b, h]), f64(v[b, h]))
         check_attn(f64(out[b, h, rt]), ref, f"anchor b{b}h{h}")
+
+
+def run_ws(q, k, v, idx=None, out=None, scattered=False, pad=None, bias=None, status=0):
+    """safedit_attn_subset_ws with a workspace of exactly the size the plan asks for."""
+    B, H, Nq, D = q.shape
+    n = Nq if idx is None else idx.numel()
+    nbytes = sd().safedit_attn_subset_workspace_size(B, H, n, k.shape[2], D, pad is not None or bias is not None)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=DEV) if nbytes else None
+    if out is None:
+        out = torch.zeros(B, H, Nq if scattered else n, D, dtype=BF, device=DEV)
+    sd().safedit_attn_subset_ws(q, k, v, idx, n, pad, bias, 0.0, out, int(scattered), ws)
+    expect_status(status)
+    return out, nbytes
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,D,k_rows", [(1, 3, 2000, 2000, 96, 600),    # 9 units -> 4 key parts each
+                                                 (1, 2, 700, 4000, 64, 300),     # ragged last key tile in a part
+                                                 (2, 3, 900, 1100, 128, None),   # dense rows, d = 128
+                                                 (1, 20, 512, 8192, 96, 300),    # 40 units -> 3 parts each
+                                                 (1, 50, 700, 4096, 96, 700)])   # 148 whole units + 2 in 4 parts
+def test_tail_split_matches_oracle(B, H, Nq, Nk, D, k_rows):
+    """The tail-balanced launch: units of 256 query rows run as key-range parts
+    whose partial (O, m, l) the merge kernel combines; against the oracle, and
+    within the attention tolerance of the whole-unit launch."""
+    q, k, v = _qkv(B, H, Nq, Nk, D, seed=3 * Nq + Nk + D)
+    idx = None if k_rows is None else _rand_idx(Nq, k_rows, seed=Nk + D)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    idd = None if idx is None else idx.to(DEV)
+    out, nbytes = run_ws(qd, kd, vd, idd)
+    assert nbytes > 0, "the shape should give a split tail"
+    ix = np.arange(Nq, dtype=np.int32) if idx is None else idx.numpy()
+    for b in range(B):
+        for h in range(0, H, max(1, H // 4)):
+            ref = oracle_rows(q, k, v, ix, b, h)
+            check_attn(f64(out[b, h]), ref, f"b{b}h{h}")
+    whole = run(qd, kd, vd, idd)
+    check_attn(f64(out), f64(whole), "split vs whole units")
+
+
+def test_tail_split_scattered_state_and_errors():
+    """Scattered output: the merge writes the S rows at their token index and
+    leaves the context rows alone; a workspace smaller than asked for is
+    refused before any launch; kept masks are never split."""
+    B, H, N, D, kr = 1, 6, 1500, 96, 500
+    q, k, v = _qkv(B, H, N, N, D, seed=1234)
+    idx = _rand_idx(N, kr, seed=4321)
+    state = torch.randn(B, H, N, D, generator=_gen(99)).to(BF)
+    st_d = state.to(DEV)
+    _, nbytes = run_ws(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), out=st_d, scattered=True)
+    assert nbytes > 0
+    keep = torch.ones(N, dtype=torch.bool)
+    keep[idx.long()] = False
+    assert torch.equal(st_d.cpu()[:, :, keep].view(torch.int16), state[:, :, keep].view(torch.int16))
+    for h in (0, 5):
+        check_attn(f64(st_d[0, h, idx.long().to(DEV)]), oracle_rows(q, k, v, idx.numpy(), 0, h), f"h{h}")
+    small = torch.empty(nbytes - 16, dtype=torch.uint8, device=DEV)
+    out = torch.zeros(B, H, kr, D, dtype=BF, device=DEV)
+    with pytest.raises(sd().SafeditError) as e:
+        sd().safedit_attn_subset_ws(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), kr, None, None, 0.0, out, 0,
+                                    small)
+    assert e.value.code == sd().ERR_INVALID_ARG
+    pad = torch.zeros(B, N, device=DEV)
+    assert sd().safedit_attn_subset_workspace_size(B, H, kr, N, D, True) == 0
+    o2, _ = run_ws(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), pad=pad)
+    o3 = run(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), pad=pad)
+    assert torch.equal(o2, o3)
+
+
+def test_tail_split_as_benchmarked():
+    """The launches the plan splits at the benchmarked sizes: the 1024^2 dense
+    anchor (768 units = 5 waves + 28 units in 4 key parts) and the stress-case
+    SRSU (640 units = 4 waves + 48 in 3 parts); sampled rows of split units
+    and of whole units against the oracle.  The 2560^2 launches keep whole
+    units: their predicted saving is under 3% of the launch."""
+    w = wl.W1024
+    q, k, v = wl.qkv(w, device=DEV)
+    out = torch.zeros(w.B, w.H, w.N, w.d, dtype=BF, device=DEV)
+    _, nbytes = run_ws(q, k, v, None, out=out)
+    assert nbytes == 28 * 4 * 256 * (w.d + 2) * 4
+    # units are (row block, slice) with row blocks fastest: the last 28 are
+    # row blocks 4..15 of slice 46 (b = 1, h = 22) and all of slice 47
+    rows = np.linspace(0, w.N - 1, 48).astype(np.int64)
+    rt = torch.as_tensor(rows, device=DEV)
+    for (b, h) in [(1, 23), (1, 22), (0, 5)]:
+        ref = oracle.attn_dense(f64(q[b, h, rt]), f64(k[b, h]), f64(v[b, h]))
+        check_attn(f64(out[b, h, rt]), ref, f"anchor b{b}h{h}")
+    assert sd().safedit_attn_subset_workspace_size(wl.W2560.B, wl.W2560.H, wl.W2560.k, wl.W2560.N, 96) == 0
+    del q, k, v, out
+    w = wl.STRESS
+    q, k, v = wl.qkv(w, device=DEV)
+    idx = torch.empty(w.k, dtype=torch.int32, device=DEV)
+    sd().safedit_partition_finalize(wl.blob_scores(w, device=DEV).contiguous(), w.N, w.k, idx, None, None)
+    state = torch.zeros(w.B, w.H, w.N, w.d, dtype=BF, device=DEV)
+    _, nbytes = run_ws(q, k, v, idx, out=state, scattered=True)
+    assert nbytes == 48 * 3 * 256 * (w.d + 2) * 4
+    # the last 48 units: row blocks 12..19 of slice 29, all of slices 30 and 31
+    ic = idx.cpu().numpy()
+    rows = np.linspace(0, w.k - 1, 40).astype(np.int64)
+    for h in (31, 29, 3):
+        ref = oracle_rows(q, k, v, ic, 0, h, rows=rows)
+        got = state[0, h, torch.as_tensor(ic[rows].astype(np.int64), device=DEV)]
+        check_attn(f64(got), ref, f"stress h{h}")
