@@ -257,6 +257,36 @@ size_t safedit_attn_subset_workspace_size(int64_t batch, int64_t heads,
                                           int32_t head_dim, int32_t kept_masks);
 
 /* ------------------------------------------------------------------------
+ * safedit_attn_subset_ws without a caller workspace.  The pages have no
+ * counterpart: this is a deployment variant for callers that may not
+ * allocate device memory around the call, not a step of the method.
+ *
+ * Arguments and result as safedit_attn_subset_ws.  The workspace is a
+ * fixed array of SAFEDIT_ATTN_NOALLOC_SCRATCH_BYTES (24 MiB) per device
+ * inside the library, reserved when its device code is loaded; the call
+ * allocates nothing.  A call whose plan needs more
+ * (safedit_attn_subset_workspace_size(...) > the limit) returns
+ * SAFEDIT_ERR_UNSUPPORTED before any launch.  The first call on a device
+ * (with that device current) looks the array's address up
+ * (cudaGetSymbolAddress) and caches it: make that first call before any
+ * stream capture.  Nothing in the array needs to start at zero (the parts
+ * write their results in full before the merge reads them), so nothing is
+ * cleared.  All calls on one device share the array: calls that overlap
+ * on the GPU (other streams, other host threads) race on it.
+ */
+#define SAFEDIT_ATTN_NOALLOC_SCRATCH_BYTES ((size_t)24 << 20)
+
+safedit_status safedit_attn_subset_noalloc(const safedit_tensor *q,
+                                           const safedit_tensor *k,
+                                           const safedit_tensor *v,
+                                           const int32_t *d_idx, int32_t n_idx,
+                                           const safedit_tensor *key_pad,
+                                           const safedit_tensor *bias,
+                                           float scale,
+                                           const safedit_tensor *out,
+                                           int32_t out_scattered, void *stream);
+
+/* ------------------------------------------------------------------------
  * State scatter.  [P1 방법론 3 / P4 Metodologia 3]: context states are cached
  * and reused between anchors; fresh sensitive rows replace their entries.
  *

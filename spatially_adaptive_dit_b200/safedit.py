@@ -31,7 +31,7 @@ _DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16, torch.bo
 
 EXPORTED = ("safedit_cross_attn_probs", "safedit_partition_accumulate", "safedit_pcsp_score",
             "safedit_partition_finalize", "safedit_mask_is_row_constant", "safedit_attn_subset",
-            "safedit_attn_subset_ws", "safedit_attn_subset_workspace_size",
+            "safedit_attn_subset_ws", "safedit_attn_subset_workspace_size", "safedit_attn_subset_noalloc",
             "safedit_scatter_state", "safedit_gather_rows", "safedit_sw_cfg", "safedit_stepcache_sw_cfg",
             "safedit_gemm_bias_act", "safedit_get_device_status", "safedit_status_string", "safedit_kernel_launch_count",
             "safedit_debug_set_wait_limit_ns", "safedit_debug_set_index_check")
@@ -63,6 +63,7 @@ _lib.safedit_attn_subset_ws.argtypes = [_T, _T, _T, _vp, _i32, _T, _T, _f32, _T,
 _lib.safedit_attn_subset_workspace_size.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                                     _i32, _i32]
 _lib.safedit_attn_subset_workspace_size.restype = ctypes.c_size_t
+_lib.safedit_attn_subset_noalloc.argtypes = [_T, _T, _T, _vp, _i32, _T, _T, _f32, _T, _i32, _vp]
 _lib.safedit_scatter_state.argtypes = [_T, _T, _i32, _vp, _i32, _vp]
 _lib.safedit_gather_rows.argtypes = [_T, _T, _i32, _vp, _i32, _vp]
 _lib.safedit_sw_cfg.argtypes = [_T, _T, _vp, _f32, _f32, _T, _vp]
@@ -180,6 +181,15 @@ def safedit_attn_subset_ws(q, k, v, idx, n_idx, key_pad, bias, scale, out, out_s
     _check(_lib.safedit_attn_subset_ws(_ref(q), _ref(k), _ref(v), _idx_ptr(idx), int(n_idx), _ref(key_pad),
                                        _ref(bias), float(scale), _ref(out), int(out_scattered), ptr, nbytes,
                                        _stream(stream)), "safedit_attn_subset_ws")
+
+
+def safedit_attn_subset_noalloc(q, k, v, idx, n_idx, key_pad, bias, scale, out, out_scattered, stream=None):
+    _check(_lib.safedit_attn_subset_noalloc(_ref(q), _ref(k), _ref(v), _idx_ptr(idx), int(n_idx), _ref(key_pad),
+                                            _ref(bias), float(scale), _ref(out), int(out_scattered),
+                                            _stream(stream)), "safedit_attn_subset_noalloc")
+
+
+ATTN_NOALLOC_SCRATCH_BYTES = 24 << 20
 
 
 def safedit_attn_subset_workspace_size(batch, heads, n_rows, n_keys, head_dim, kept_masks=False) -> int:
