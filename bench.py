@@ -443,7 +443,8 @@ def run_ours(args):
                          "unit": "TFLOP/s", "frac": round(achieved / bf16_sust, 4),
                          "frac_of_burst": round(achieved / bf16_burst, 4), "traffic": traffic,
                          "algorithmic_bytes": algo_bytes,
-                         "traffic_over_algorithmic": None if traffic is None else round(traffic / algo_bytes, 3)},
+                         "traffic_over_algorithmic": None if traffic is None else round(traffic / algo_bytes, 3),
+                         "mufu_colimit": mufu_colimit(W.d, 0.75)},
             "gpu_launches": launches,
             "memory": {"peak_allocated_gb": round(peak_gb, 2),
                        "note": f"this device's buffers of the attention path ({tr.H} heads) incl. the "
@@ -468,6 +469,19 @@ def run_ours(args):
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def mufu_colimit(d, mufu_share):
+    """Ceiling the exponentials put on the attention, as a fraction of the
+    tensor peak: per (query, key) pair the MMAs do 4 d flop at 8192 dense bf16
+    flop per clock per SM, and the softmax one exponential, of which
+    `mufu_share` runs on the MUFU unit at 16 per clock per SM (measured on
+    B200) and the rest on the FMA pipe."""
+    tensor_clk, mufu_clk = 4 * d / 8192, mufu_share / 16
+    return {"flop_per_exponential": 4 * d, "tensor_flop_per_clk_sm": 8192, "ex2_per_clk_sm": 16,
+            "ceiling_all_on_mufu": round(min(1.0, tensor_clk / (1 / 16)), 3),
+            "mufu_share_as_built": mufu_share,
+            "ceiling_as_built": round(min(1.0, tensor_clk / mufu_clk), 3)}
 
 
 def _srsu_algorithmic_bytes(tr):

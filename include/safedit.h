@@ -104,7 +104,8 @@ safedit_status safedit_cross_attn_probs(const safedit_tensor *q_img,
  * accumulated in fp64.  Call it once per warm-up step (and layer) with the
  * same score buffer; zero the buffer before the first call.
  *
- * p [H,N,L] f32, inner stride 1.  d_content [L] u8.  d_score [N] f64.
+ * p [H,N,L] f32 or bf16 (widened exactly), inner stride 1.  d_content [L]
+ * u8.  d_score [N] f64.
  */
 safedit_status safedit_partition_accumulate(const safedit_tensor *p,
                                             const uint8_t *d_content,

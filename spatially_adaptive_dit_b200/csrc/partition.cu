@@ -1,8 +1,8 @@
 // partition.cu -- PCSP (SAFE-DiT summary, 방법론 2; AccelAes summary B.1):
-//   * partition_accumulate: score[i] += sum_h sum_{content j} P[h,i,j], one
-//     warp per image token, 128-bit streaming loads of the 16-byte groups of
-//     P that hold a content column (padding is never read), fp64
-//     accumulation and a warp-shuffle reduction;
+//   * partition_accumulate: score[i] += sum_h sum_{content j} P[h,i,j] (P in
+//     f32 or bf16), one warp per image token, 128-bit streaming loads of the
+//     16-byte groups of P that hold a content column (padding is never
+//     read), fp64 accumulation and a warp-shuffle reduction;
 //   * partition_finalize: the top-k split (ties to the lower index) by an
 //     8-pass radix select on order-preserving 64-bit keys, a stable
 //     block-scan compaction into ascending S / C index lists, and the
@@ -14,7 +14,7 @@ namespace sd {
 
 // ---------------------------------------------------------- accumulate ----
 struct AccParams {
-  const float* P;
+  const void* P;  // f32 or bf16 elements
   const uint8_t* content;
   double* score;
   int64_t H, N, L;
@@ -25,61 +25,78 @@ struct AccParams {
 constexpr int kAccWarps = 8;
 constexpr int kAccHeads = 4;  // heads whose loads a lane keeps in flight at once (8 measured slower)
 
-// Vector path: L % 4 == 0, strides % 4 == 0, 16-byte aligned base,
-// L <= 128 * NCH (NCH passes of 128 columns per warp).
-template <int NCH>
+// element e of a 16-byte group of P as f32 (bf16 widens exactly)
+template <typename T>
+__device__ __forceinline__ float acc_elem(const uint4& v, int e);
+template <>
+__device__ __forceinline__ float acc_elem<float>(const uint4& v, int e) {
+  const uint32_t w = e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
+  return __uint_as_float(w);
+}
+template <>
+__device__ __forceinline__ float acc_elem<__nv_bfloat16>(const uint4& v, int e) {
+  const int q = e >> 1;
+  const uint32_t w = q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+  return __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
+}
+
+// Vector path: 16-byte groups of VEC = 16 / sizeof(T) columns, L % VEC == 0,
+// strides % VEC == 0, 16-byte aligned base, L <= 32 VEC NCH (NCH passes of
+// 32 groups per warp).
+template <typename T, int NCH>
 __global__ void __launch_bounds__(kAccWarps * 32) accumulate_vec_kernel(AccParams p) {
+  constexpr int VEC = 16 / int(sizeof(T));
+  constexpr int CH = 32 * VEC;  // columns per pass of the warp
+  static_assert(VEC * NCH <= 32, "content flags of a lane fit one word");
+  const T* const P = static_cast<const T*>(p.P);
   const int lane = threadIdx.x & 31;
   const int64_t warp = blockIdx.x * int64_t(kAccWarps) + (threadIdx.x >> 5);
   const int64_t nwarps = int64_t(gridDim.x) * kAccWarps;
-  const int nchunk = NCH;
-  // content flags of this lane's columns: 4 bits per chunk
+  constexpr uint32_t kGroup = (1u << VEC) - 1u;
+  // content flags of this lane's columns: VEC bits per pass
   uint32_t cmask = 0;
-  for (int c = 0; c < nchunk; ++c)
-    for (int e = 0; e < 4; ++e) {
-      const int64_t j = int64_t(c) * 128 + lane * 4 + e;
-      if (j < p.L && p.content[j]) cmask |= 1u << (c * 4 + e);
+  for (int c = 0; c < NCH; ++c)
+    for (int e = 0; e < VEC; ++e) {
+      const int64_t j = int64_t(c) * CH + lane * VEC + e;
+      if (j < p.L && p.content[j]) cmask |= 1u << (c * VEC + e);
     }
   for (int64_t i = warp; i < p.N; i += nwarps) {
     double acc = 0.0;
-    const float* row0 = p.P + i * p.sN;
+    const T* row0 = P + i * p.sN;
     int64_t h = 0;
     for (; h + kAccHeads <= p.H; h += kAccHeads) {
-      float4 v[kAccHeads][NCH];
+      uint4 v[kAccHeads][NCH];
 #pragma unroll
       for (int hh = 0; hh < kAccHeads; ++hh)
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
           // only 16-byte groups holding a content column are read (text
           // padding and the non-content tokens never leave HBM)
-          if ((cmask >> (c * 4)) & 0xFu)
-            v[hh][c] = __ldcs(reinterpret_cast<const float4*>(row0 + (h + hh) * p.sH +
-                                                              int64_t(c) * 128 + lane * 4));
+          if ((cmask >> (c * VEC)) & kGroup)
+            v[hh][c] = __ldcs(reinterpret_cast<const uint4*>(row0 + (h + hh) * p.sH + int64_t(c) * CH +
+                                                             lane * VEC));
           else
-            v[hh][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            v[hh][c] = make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
       for (int hh = 0; hh < kAccHeads; ++hh)
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
-          const uint32_t m = cmask >> (c * 4);
-          if (m & 1u) acc += static_cast<double>(v[hh][c].x);
-          if (m & 2u) acc += static_cast<double>(v[hh][c].y);
-          if (m & 4u) acc += static_cast<double>(v[hh][c].z);
-          if (m & 8u) acc += static_cast<double>(v[hh][c].w);
+          const uint32_t m = cmask >> (c * VEC);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e)
+            if ((m >> e) & 1u) acc += static_cast<double>(acc_elem<T>(v[hh][c], e));
         }
     }
     for (; h < p.H; ++h) {
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
-        const int64_t j = int64_t(c) * 128 + lane * 4;
-        if ((cmask >> (c * 4)) & 0xFu) {
-          const float4 v = __ldcs(reinterpret_cast<const float4*>(row0 + h * p.sH + j));
-          const uint32_t m = cmask >> (c * 4);
-          if (m & 1u) acc += static_cast<double>(v.x);
-          if (m & 2u) acc += static_cast<double>(v.y);
-          if (m & 4u) acc += static_cast<double>(v.z);
-          if (m & 8u) acc += static_cast<double>(v.w);
+        const uint32_t m = cmask >> (c * VEC);
+        if (m & kGroup) {
+          const uint4 v = __ldcs(reinterpret_cast<const uint4*>(row0 + h * p.sH + int64_t(c) * CH + lane * VEC));
+#pragma unroll
+          for (int e = 0; e < VEC; ++e)
+            if ((m >> e) & 1u) acc += static_cast<double>(acc_elem<T>(v, e));
         }
       }
     }
@@ -90,16 +107,18 @@ __global__ void __launch_bounds__(kAccWarps * 32) accumulate_vec_kernel(AccParam
 }
 
 // General path: any L and strides (inner stride 1).
+template <typename T>
 __global__ void __launch_bounds__(kAccWarps * 32) accumulate_scalar_kernel(AccParams p) {
+  const T* const P = static_cast<const T*>(p.P);
   const int lane = threadIdx.x & 31;
   const int64_t warp = blockIdx.x * int64_t(kAccWarps) + (threadIdx.x >> 5);
   const int64_t nwarps = int64_t(gridDim.x) * kAccWarps;
   for (int64_t i = warp; i < p.N; i += nwarps) {
     double acc = 0.0;
     for (int64_t h = 0; h < p.H; ++h) {
-      const float* row = p.P + h * p.sH + i * p.sN;
+      const T* row = P + h * p.sH + i * p.sN;
       for (int64_t j = lane; j < p.L; j += 32)
-        if (p.content[j]) acc += static_cast<double>(row[j]);
+        if (p.content[j]) acc += static_cast<double>(static_cast<float>(row[j]));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -281,10 +300,11 @@ safedit_status safedit_partition_accumulate(const safedit_tensor* p, const uint8
   if ((st = check_tensor(p, 3)) != SAFEDIT_OK) return st;
   if ((p->dims[2] > 0 && !d_content) || (p->dims[1] > 0 && !d_score))
     return SAFEDIT_ERR_INVALID_ARG;
-  if (p->dtype != SAFEDIT_F32) return SAFEDIT_ERR_DTYPE;
+  if (p->dtype != SAFEDIT_F32 && p->dtype != SAFEDIT_BF16) return SAFEDIT_ERR_DTYPE;
   if (p->strides[2] != 1) return SAFEDIT_ERR_ALIGNMENT;
+  const bool bf16 = p->dtype == SAFEDIT_BF16;
   AccParams a;
-  a.P = static_cast<const float*>(p->data);
+  a.P = p->data;
   a.content = d_content;
   a.score = d_score;
   a.H = p->dims[0];
@@ -295,7 +315,8 @@ safedit_status safedit_partition_accumulate(const safedit_tensor* p, const uint8
   if (a.N == 0) return SAFEDIT_OK;
   a.status = status_ptr();
   if (!a.status) return SAFEDIT_ERR_CUDA;
-  const bool vec = (a.L % 4 == 0) && (a.sH % 4 == 0) && (a.sN % 4 == 0) && aligned16(a.P) &&
+  const int vec_w = bf16 ? 8 : 4;  // elements per 16-byte group
+  const bool vec = (a.L % vec_w == 0) && (a.sH % vec_w == 0) && (a.sN % vec_w == 0) && aligned16(a.P) &&
                    a.L <= 1024;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -304,18 +325,30 @@ safedit_status safedit_partition_accumulate(const safedit_tensor* p, const uint8
   const int64_t cap = int64_t(sms) * 16;
   if (blocks > cap) blocks = cap;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int nch = static_cast<int>((a.L + 127) / 128);
+  const int nch = static_cast<int>((a.L + 32 * vec_w - 1) / (32 * vec_w));  // passes of 32 groups
   const dim3 grid(static_cast<unsigned>(blocks)), block(kAccWarps * 32);
-  if (vec && nch <= 1)
-    accumulate_vec_kernel<1><<<grid, block, 0, s>>>(a);
-  else if (vec && nch <= 2)
-    accumulate_vec_kernel<2><<<grid, block, 0, s>>>(a);
-  else if (vec && nch <= 4)
-    accumulate_vec_kernel<4><<<grid, block, 0, s>>>(a);
-  else if (vec)
-    accumulate_vec_kernel<8><<<grid, block, 0, s>>>(a);
-  else
-    accumulate_scalar_kernel<<<static_cast<unsigned>(blocks), kAccWarps * 32, 0, s>>>(a);
+  if (!vec) {
+    if (bf16)
+      accumulate_scalar_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(a);
+    else
+      accumulate_scalar_kernel<float><<<grid, block, 0, s>>>(a);
+  } else if (bf16) {
+    if (nch <= 1)
+      accumulate_vec_kernel<__nv_bfloat16, 1><<<grid, block, 0, s>>>(a);
+    else if (nch <= 2)
+      accumulate_vec_kernel<__nv_bfloat16, 2><<<grid, block, 0, s>>>(a);
+    else
+      accumulate_vec_kernel<__nv_bfloat16, 4><<<grid, block, 0, s>>>(a);
+  } else {
+    if (nch <= 1)
+      accumulate_vec_kernel<float, 1><<<grid, block, 0, s>>>(a);
+    else if (nch <= 2)
+      accumulate_vec_kernel<float, 2><<<grid, block, 0, s>>>(a);
+    else if (nch <= 4)
+      accumulate_vec_kernel<float, 4><<<grid, block, 0, s>>>(a);
+    else
+      accumulate_vec_kernel<float, 8><<<grid, block, 0, s>>>(a);
+  }
   return after_launch(1);
 }
 

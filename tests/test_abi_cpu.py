@@ -153,7 +153,7 @@ def test_bandwidth_kernels_host_validation(sd):
     assert fin(ctypes.c_void_p(0x40000), 10, 11, None, None, None, None) == sd.ERR_INVALID_ARG
     assert fin(ctypes.c_void_p(0x40000), 10, -1, None, None, None, None) == sd.ERR_INVALID_ARG
 
-    P = _desc(sd, (2, 16, 32), (512, 32, 1), sd.BF16)
+    P = _desc(sd, (2, 16, 32), (512, 32, 1), sd.F16)  # P in f32 or bf16 only
     acc = lambda *a: sd.raw_call("safedit_partition_accumulate", *a)  # noqa: E731
     assert acc(R(P), ctypes.c_void_p(0x50000), ctypes.c_void_p(0x60000), None) == sd.ERR_DTYPE
     Pf = _desc(sd, (2, 16, 32), (512, 32, 2), sd.F32)

@@ -38,3 +38,14 @@ def test_source_hash_ignores_comments_and_whitespace(tmp_path):
 def test_committed_traffic_matches_current_attention_source():
     import bench
     assert bench._ncu_traffic() is not None, "profiles/attn_subset_srsu_2560.traffic.json is stale"
+
+
+def test_mufu_colimit_at_the_head_dims():
+    import bench
+    # d = 96: 384 flop per exponential take 384 / 8192 clock of tensor time,
+    # an exponential on MUFU 1 / 16: all on MUFU caps the tensor pipe at 75%;
+    # with a quarter on the FMA pipe the two times are equal
+    c = bench.mufu_colimit(96, 0.75)
+    assert c["ceiling_all_on_mufu"] == 0.75 and c["ceiling_as_built"] == 1.0
+    assert bench.mufu_colimit(128, 1.0)["ceiling_as_built"] == 1.0
+    assert bench.mufu_colimit(64, 1.0)["ceiling_as_built"] == 0.5

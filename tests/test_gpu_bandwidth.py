@@ -164,6 +164,31 @@ def test_partition_accumulate_and_finalize(H, N, L, nvalid):
     assert a == b
 
 
+@pytest.mark.parametrize("H,N,L,nvalid", [(24, 4096, 256, 128), (3, 1000, 30, 25), (4, 300, 512, 400),
+                                          (2, 700, 1024, 900)])
+def test_partition_accumulate_bf16_probabilities(H, N, L, nvalid):
+    """P stored in bf16 (vector path when L % 8 == 0, the scalar path at
+    L = 30), widened exactly: against the oracle on the same bf16 values."""
+    g = _gen(7 * H * N + L)
+    logits = torch.randn(H, N, L, generator=g)
+    logits[:, :, nvalid:] = float("-inf")
+    P = torch.softmax(logits, dim=-1).to(torch.bfloat16)
+    content = torch.zeros(L, dtype=torch.uint8)
+    content[1:nvalid - 1] = 1
+    score = torch.zeros(N, dtype=torch.float64, device=DEV)
+    sd().safedit_partition_accumulate(P.to(DEV), content.to(DEV), score)
+    expect_status(0)
+    ref = oracle.partition_accumulate(P.double(), content)
+    assert np.abs(score.cpu().numpy() - ref).max() <= 1e-12 * np.abs(ref).max()
+    # a strided view (every other head of a larger tensor) takes the same path
+    big = torch.zeros(2 * H, N, L, dtype=torch.bfloat16, device=DEV)
+    big[::2] = P.to(DEV)
+    score.zero_()
+    sd().safedit_partition_accumulate(big[::2], content.to(DEV), score)
+    expect_status(0)
+    assert np.abs(score.cpu().numpy() - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
 def test_partition_finalize_ties_and_signed_zero():
     N = 5000
     g = _gen(99)
