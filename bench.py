@@ -751,12 +751,14 @@ def run_e2e(tr, stream, args):
     compact Q_S over all N keys, scatter O_S into O_state.  Each step's inputs
     sit back to back in one pinned block and cross the link as one copy (large
     copies reach the link's rate, 70 MB ones do not).  A copy stream runs
-    ahead of the compute stream: three SRSU input blocks, and two anchor blocks
+    ahead of the compute stream: four SRSU input blocks, and two anchor blocks
     (Q, K, V, predictions) whose K and V then serve as the cached state until
     the next anchor, so an anchor's upload never waits for the step before it;
-    events order every buffer reuse."""
+    events order every buffer reuse.  With three SRSU blocks the upload of the
+    fourth step after an anchor waited for the first one's compute, which
+    starts only after the anchor's 12 ms: the link idled ~5 ms per anchor."""
     w = tr.w
-    NSET = 3
+    NSET = 4
     q_s = tr.q[:, :, : tr.k].contiguous()
     o_s = torch.empty_like(q_s)
     srsu_src = [q_s, tr.k_s, tr.v_s, tr.eps_c, tr.eps_u]
