@@ -557,11 +557,14 @@ def measure_extensions(tr, stream, dev, unfused_pcsp_ms):
     ms = time_reps_interleaved(cases, stream)
     base = ms["srsu_mask_elided"]["p50"]
     out["kept_mask_stress"] = {
-        name: {**t, "tflops": round(flop / (t["p50"] * 1e-3) / 1e12, 1), "vs_elided": round(t["p50"] / base, 3)}
+        name: {**t, "tflops": round(flop / (t["p50"] * 1e-3) / 1e12, 1), "vs_elided": round(t["p50"] / base, 3),
+               **({"vs_whole_units": round(t["p50"] / ms[name[:-len("_tail_split")]]["p50"], 3)}
+                  if name.endswith("_tail_split") else {})}
         for name, t in ms.items()}
     out["kept_mask_stress"]["workload"] = (
         f"B=1, H=32, N={wl.STRESS.N}, d=128, |S|={wl.STRESS.k} (blob scores); padding = trailing 1/8 of the keys "
-        "at -inf; bias = [1,1,N,N] N(0,1) in bf16 or f32; the six launches taken in turn within every rep")
+        "at -inf; bias = [1,1,N,N] N(0,1) in bf16 or f32; each as whole units and tail-balanced; the ten launches "
+        "taken in turn within every rep")
     del cases
     torch.cuda.empty_cache()
     out["config_1024"] = measure_1024(sd, dev, stream, flush)
@@ -987,9 +990,10 @@ def run_reference(args):
 def stress_srsu_cases(sd, dev, stream):
     """The SRSU launches of the mask-stress workload (B=1, H=32, N=16384,
     d=128, |S|=4915 from the clustered blob scores): mask elided (no mask
-    input; whole units, and tail-balanced), kept text-padding key mask
-    (trailing 1/8 of the keys -inf), kept non-uniform bias [1,1,N,N] in bf16,
-    both, and the bias in f32.  Returns the launch closures (name -> fn) and
+    input), kept text-padding key mask (trailing 1/8 of the keys -inf), kept
+    non-uniform bias [1,1,N,N] in bf16, both, and the bias in f32; each as
+    whole units and tail-balanced (`_tail_split`: 640 units = 4 waves + 48,
+    those 48 in 3 key parts).  Returns the launch closures (name -> fn) and
     the flop of one call."""
     w = wl.STRESS
     q, k, v = wl.qkv(w, device=dev)
@@ -1004,15 +1008,13 @@ def stress_srsu_cases(sd, dev, stream):
     att = lambda kp, bb: (lambda: sd.safedit_attn_subset(q, k, v, idx, w.k, kp, bb, 0.0, o, 1, stream))
     nb = sd.safedit_attn_subset_workspace_size(w.B, w.H, w.k, w.N, w.d)
     ws = torch.empty(nb, dtype=torch.uint8, device=dev)  # 640 units = 4 waves + 48 split in 3
-    cases = {
-        "srsu_mask_elided": att(None, None),
-        "srsu_mask_elided_tail_split": lambda: sd.safedit_attn_subset_ws(q, k, v, idx, w.k, None, None, 0.0, o, 1,
-                                                                        ws, stream),
-        "srsu_kept_padding": att(pad, None),
-        "srsu_kept_bias": att(None, bias),
-        "srsu_kept_padding_and_bias": att(pad, bias),
-        "srsu_kept_bias_f32": att(None, bias32),
-    }
+    att_ws = lambda kp, bb: (lambda: sd.safedit_attn_subset_ws(q, k, v, idx, w.k, kp, bb, 0.0, o, 1, ws, stream))
+    cases = {}
+    for name, kp, bb in (("srsu_mask_elided", None, None), ("srsu_kept_padding", pad, None),
+                         ("srsu_kept_bias", None, bias), ("srsu_kept_padding_and_bias", pad, bias),
+                         ("srsu_kept_bias_f32", None, bias32)):
+        cases[name] = att(kp, bb)
+        cases[name + "_tail_split"] = att_ws(kp, bb)
     return cases, 4.0 * w.k * w.N * w.d * w.B * w.H
 
 

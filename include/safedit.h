@@ -222,11 +222,15 @@ safedit_status safedit_attn_subset(const safedit_tensor *q,
  * output rows, running max and row sum (f32) to d_workspace, and a merge
  * kernel then combines them into the output rows (the online-softmax merge;
  * the result equals safedit_attn_subset's within the attention tolerance,
- * not bit for bit).  The plan takes a split only where a per-CTA cost model
- * (set-up + per-key-tile time measured on B200) predicts a saving of at
- * least 3% of the call; otherwise, and for launches with kept masks
- * (key_pad or bias), the call is safedit_attn_subset.  All launches go on
- * `stream`, in order, so the call is stream-ordered like the others.
+ * not bit for bit).  Kept masks (key_pad, bias) are split like the rest;
+ * a part whose key range holds no admissible key for a row leaves it to
+ * the merge, which reports a row with none in any part as
+ * SAFEDIT_ERR_MASKED_ROW and writes zeros, as safedit_attn_subset does.
+ * The plan takes a split only where a per-CTA cost model (set-up +
+ * per-key-tile time of the mask-free kernel, measured on B200) predicts a
+ * saving of at least 3% of the call; otherwise the call is
+ * safedit_attn_subset.  All launches go on `stream`, in order, so the call
+ * is stream-ordered like the others.
  *
  * Arguments as safedit_attn_subset, plus d_workspace / workspace_bytes:
  * device memory of at least safedit_attn_subset_workspace_size(...) bytes
@@ -250,12 +254,11 @@ safedit_status safedit_attn_subset_ws(const safedit_tensor *q,
 /* Workspace bytes safedit_attn_subset_ws needs on the current device (its
  * SM count enters the plan) for batch x heads slices of n_rows query rows
  * over n_keys keys of head_dim (64, 96 or 128): (split units) x s x 256 x
- * (head_dim + 2) x 4.  kept_masks != 0 for a call with key_pad or bias
- * (never split: 0 bytes); 0 also when the plan keeps whole units.  Host
- * only, no launch; invalid sizes give 0. */
+ * (head_dim + 2) x 4, with or without kept masks; 0 when the plan keeps
+ * whole units.  Host only, no launch; invalid sizes give 0. */
 size_t safedit_attn_subset_workspace_size(int64_t batch, int64_t heads,
                                           int64_t n_rows, int64_t n_keys,
-                                          int32_t head_dim, int32_t kept_masks);
+                                          int32_t head_dim);
 
 /* ------------------------------------------------------------------------
  * safedit_attn_subset_ws without a caller workspace.  The pages have no

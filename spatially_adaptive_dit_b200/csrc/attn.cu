@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int b = bh / p.H, h = bh - b * p.H;
   const int row0 = SPLIT ? (unit - bh * p.n_rb) * 256 : int(blockIdx.x) * 256;
   const int nk = (p.Nk + C::BN - 1) / C::BN;
-  // this CTA's key tiles [k_lo, k_hi) (kept-padding launches are never split)
+  // this CTA's key tiles [k_lo, k_hi)
   const int k_lo = !SPLIT || kpart < 0 ? 0 : int(int64_t(nk) * kpart / p.split);
   const int k_hi = !SPLIT || kpart < 0 ? nk : int(int64_t(nk) * (kpart + 1) / p.split);
   // live key tiles (kept key padding): a tile whose pad entries are all -inf
@@ -264,10 +264,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     return nk;
   };
+  // live tiles in [k_lo, k_hi)
   auto live_count = [&]() -> int {
     if (!skip_tiles) return k_hi - k_lo;
     int n = 0;
-    for (int w = 0; w < (nk + 31) / 32; ++w) n += __popc(live_word(w));
+    for (int w = k_lo >> 5; w <= (k_hi - 1) >> 5; ++w) {
+      uint32_t bits = live_word(w);
+      if (w == (k_lo >> 5)) bits &= ~0u << (k_lo & 31);
+      if (w == ((k_hi - 1) >> 5) && (k_hi & 31)) bits &= ~(~0u << (k_hi & 31));
+      n += __popc(bits);
+    }
     return n;
   };
 
@@ -620,7 +626,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (live && !partial && !(l_run > 0.f)) set_status(p.status, SAFEDIT_ERR_MASKED_ROW);
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
       // with skipped key tiles O may never have been written: a row with no
-      // weight (fully masked: an error, reported above) is written as zeros
+      // weight (fully masked: an error, reported above; for a part, a key
+      // range with no admissible key, left to the merge) is written as zeros
       const bool zero_row = PAD && !(l_run > 0.f);
       const int64_t slot = int64_t(e_unit - p.n_full) * p.split + e_part;
       const int rr = t * 128 + wr * 32 + lane;
@@ -641,8 +648,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           float4* dst = reinterpret_cast<float4*>(po + c * 32);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                                 __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+            dst[e] = zero_row ? make_float4(0.f, 0.f, 0.f, 0.f)
+                              : make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                            __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
         } else if (live) {
           uint32_t w[16];
 #pragma unroll
@@ -807,6 +815,14 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnParams p) {
   const float* ml = p.part + int64_t(p.n_part_units) * p.split * 256 * D;
   float m = -INFINITY;
   for (int k = 0; k < p.split; ++k) m = fmaxf(m, ml[((int64_t(pu) * p.split + k) * 256 + rr) * 2]);
+  const int64_t orow_idx = p.out_scattered ? int64_t(my_q) : int64_t(my_row);
+  __nv_bfloat16* orow = p.out + b * p.o_sb + h * p.o_sh + orow_idx * p.o_sr;
+  if (m == -INFINITY) {  // no part has an admissible key: a fully masked row
+    if (lane == 0) set_status(p.status, SAFEDIT_ERR_MASKED_ROW);
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) orow[lane + 32 * e] = __float2bfloat16_rn(0.f);
+    return;
+  }
   float l = 0.f, acc[D / 32];
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
@@ -819,8 +835,6 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnParams p) {
     for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(w, po[lane + 32 * e], acc[e]);
   }
   const float inv = 1.f / l;
-  const int64_t orow_idx = p.out_scattered ? int64_t(my_q) : int64_t(my_row);
-  __nv_bfloat16* orow = p.out + b * p.o_sb + h * p.o_sh + orow_idx * p.o_sr;
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) orow[lane + 32 * e] = __float2bfloat16_rn(acc[e] * inv);
 }
@@ -909,14 +923,21 @@ static safedit_status launch_attn(const CUtensorMap& tmK, const CUtensorMap& tmV
 
 // A split plan: the whole units (a whole number of waves), then the parts of
 // the last units, then their merge, in stream order.
-template <int D>
+template <int D, bool PAD, int BIAS>
 static safedit_status launch_attn_split(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                         const AttnParams& p, int B, cudaStream_t stream) {
   safedit_status st = SAFEDIT_OK;
-  if (p.n_full > 0 && (st = launch_attn<D, false, kBiasNone>(tmK, tmV, p, B, stream)) != SAFEDIT_OK) return st;
-  if ((st = launch_attn<D, false, kBiasNone, true>(tmK, tmV, p, B, stream)) != SAFEDIT_OK) return st;
+  if (p.n_full > 0 && (st = launch_attn<D, PAD, BIAS>(tmK, tmV, p, B, stream)) != SAFEDIT_OK) return st;
+  if ((st = launch_attn<D, PAD, BIAS, true>(tmK, tmV, p, B, stream)) != SAFEDIT_OK) return st;
   attn_merge_kernel<D><<<(p.n_part_units * 256 + 7) / 8, 256, 0, stream>>>(p);
   return after_launch(1);
+}
+
+template <int D, bool PAD, int BIAS>
+static safedit_status launch_planned(const CUtensorMap& tmK, const CUtensorMap& tmV, const AttnParams& p,
+                                     int B, cudaStream_t s) {
+  if (p.n_part_units > 0) return launch_attn_split<D, PAD, BIAS>(tmK, tmV, p, B, s);
+  return launch_attn<D, PAD, BIAS>(tmK, tmV, p, B, s);
 }
 
 template <int D>
@@ -925,14 +946,13 @@ static safedit_status dispatch_attn(const CUtensorMap& tmK, const CUtensorMap& t
   const bool pad = p.pad != nullptr;
   const int bias = p.bias == nullptr ? kBiasNone : (p.bias_f32 ? kBiasF32 : kBiasBf16);
   if (pad) {
-    if (bias == kBiasBf16) return launch_attn<D, true, kBiasBf16>(tmK, tmV, p, B, s);
-    if (bias == kBiasF32) return launch_attn<D, true, kBiasF32>(tmK, tmV, p, B, s);
-    return launch_attn<D, true, kBiasNone>(tmK, tmV, p, B, s);
+    if (bias == kBiasBf16) return launch_planned<D, true, kBiasBf16>(tmK, tmV, p, B, s);
+    if (bias == kBiasF32) return launch_planned<D, true, kBiasF32>(tmK, tmV, p, B, s);
+    return launch_planned<D, true, kBiasNone>(tmK, tmV, p, B, s);
   }
-  if (bias == kBiasBf16) return launch_attn<D, false, kBiasBf16>(tmK, tmV, p, B, s);
-  if (bias == kBiasF32) return launch_attn<D, false, kBiasF32>(tmK, tmV, p, B, s);
-  if (p.n_part_units > 0) return launch_attn_split<D>(tmK, tmV, p, B, s);
-  return launch_attn<D, false, kBiasNone>(tmK, tmV, p, B, s);
+  if (bias == kBiasBf16) return launch_planned<D, false, kBiasBf16>(tmK, tmV, p, B, s);
+  if (bias == kBiasF32) return launch_planned<D, false, kBiasF32>(tmK, tmV, p, B, s);
+  return launch_planned<D, false, kBiasNone>(tmK, tmV, p, B, s);
 }
 
 static safedit_status check_bhnd(const safedit_tensor* t) {
@@ -1013,7 +1033,7 @@ static safedit_status attn_subset_impl(const safedit_tensor* q, const safedit_te
     p.bias_sh = bias->dims[1] == 1 ? 0 : bias->strides[1];
     p.bias_sq = bias->strides[2];
   }
-  AttnPlan pl = plan_attn(n_rows, B * H, Nk, int(D), use_ws && !key_pad && !bias, sm_count());
+  AttnPlan pl = plan_attn(n_rows, B * H, Nk, int(D), use_ws, sm_count());
   if (use_ws && pl.ws_bytes > 0) {
     if (!d_ws || ws_bytes < pl.ws_bytes) return SAFEDIT_ERR_INVALID_ARG;
     if (!aligned16(d_ws)) return SAFEDIT_ERR_ALIGNMENT;
@@ -1080,11 +1100,11 @@ extern "C" safedit_status safedit_attn_subset_ws(const safedit_tensor* q, const 
 }
 
 extern "C" size_t safedit_attn_subset_workspace_size(int64_t batch, int64_t heads, int64_t n_rows,
-                                                     int64_t n_keys, int32_t head_dim, int32_t kept_masks) {
+                                                     int64_t n_keys, int32_t head_dim) {
   if (batch <= 0 || heads <= 0 || n_rows <= 0 || n_keys <= 0) return 0;
   if (head_dim != 64 && head_dim != 96 && head_dim != 128) return 0;
   if (batch * heads > 65535 || n_rows > INT32_MAX || n_keys > INT32_MAX ||
       (n_rows + 255) / 256 * batch * heads > INT32_MAX)
     return 0;
-  return plan_attn(n_rows, batch * heads, n_keys, head_dim, kept_masks == 0, sm_count()).ws_bytes;
+  return plan_attn(n_rows, batch * heads, n_keys, head_dim, true, sm_count()).ws_bytes;
 }

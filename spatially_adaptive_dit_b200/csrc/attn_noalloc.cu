@@ -53,7 +53,7 @@ extern "C" safedit_status safedit_attn_subset_noalloc(const safedit_tensor* q, c
   if (!q || !k || q->ndim != 4 || k->ndim != 4) return SAFEDIT_ERR_INVALID_ARG;
   const int64_t n_rows = d_idx ? int64_t(n_idx) : q->dims[2];
   const size_t need = safedit_attn_subset_workspace_size(q->dims[0], q->dims[1], n_rows, k->dims[2],
-                                                         int32_t(q->dims[3]), key_pad || bias ? 1 : 0);
+                                                         int32_t(q->dims[3]));
   if (need > kAttnScratchBytes) return SAFEDIT_ERR_UNSUPPORTED;  // before any launch
   void* scratch = nullptr;
   const safedit_status st = scratch_address(&scratch);

@@ -61,7 +61,7 @@ _lib.safedit_mask_is_row_constant.argtypes = [_T, _vp, _vp, _vp]
 _lib.safedit_attn_subset.argtypes = [_T, _T, _T, _vp, _i32, _T, _T, _f32, _T, _i32, _vp]
 _lib.safedit_attn_subset_ws.argtypes = [_T, _T, _T, _vp, _i32, _T, _T, _f32, _T, _i32, _vp, ctypes.c_size_t, _vp]
 _lib.safedit_attn_subset_workspace_size.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
-                                                    _i32, _i32]
+                                                    _i32]
 _lib.safedit_attn_subset_workspace_size.restype = ctypes.c_size_t
 _lib.safedit_attn_subset_noalloc.argtypes = [_T, _T, _T, _vp, _i32, _T, _T, _f32, _T, _i32, _vp]
 _lib.safedit_scatter_state.argtypes = [_T, _T, _i32, _vp, _i32, _vp]
@@ -192,9 +192,9 @@ def safedit_attn_subset_noalloc(q, k, v, idx, n_idx, key_pad, bias, scale, out, 
 ATTN_NOALLOC_SCRATCH_BYTES = 24 << 20
 
 
-def safedit_attn_subset_workspace_size(batch, heads, n_rows, n_keys, head_dim, kept_masks=False) -> int:
+def safedit_attn_subset_workspace_size(batch, heads, n_rows, n_keys, head_dim) -> int:
     return int(_lib.safedit_attn_subset_workspace_size(int(batch), int(heads), int(n_rows), int(n_keys),
-                                                       int(head_dim), 1 if kept_masks else 0))
+                                                       int(head_dim)))
 
 
 def _desc_array(ts):

@@ -199,10 +199,10 @@ def test_attention_tail_split_plan(sd):
     assert ws(2, 24, 1229, 4096, 96) == 0
     # 1024^2 anchor: 16 x 48 = 768 = 5 waves + 28 -> 28 x 4 (one round of 1/4)
     assert ws(2, 24, 4096, 4096, 96) == 28 * 4 * row(96)
-    # stress SRSU: 20 x 32 = 640 = 4 waves + 48 -> 48 x 3 (one round of 1/3)
+    # stress SRSU (with kept masks or not: the same plan): 20 x 32 = 640 =
+    # 4 waves + 48 -> 48 x 3 (one round of 1/3)
     assert ws(1, 32, 4915, 16384, 128) == 48 * 3 * row(128)
-    # no tail, kept masks, or too few key tiles to split: nothing
+    # no tail, or too few key tiles to split: nothing
     assert ws(1, 148, 256, 25600, 96) == 0
-    assert ws(2, 24, 7680, 25600, 96, kept_masks=True) == 0
     assert ws(1, 2, 64, 256, 64) == 0
     assert ws(0, 2, 64, 256, 64) == 0 and ws(1, 2, 64, 4096, 80) == 0

@@ -356,7 +356,7 @@ def run_ws(q, k, v, idx=None, out=None, scattered=False, pad=None, bias=None, st
     """safedit_attn_subset_ws with a workspace of exactly the size the plan asks for."""
     B, H, Nq, D = q.shape
     n = Nq if idx is None else idx.numel()
-    nbytes = sd().safedit_attn_subset_workspace_size(B, H, n, k.shape[2], D, pad is not None or bias is not None)
+    nbytes = sd().safedit_attn_subset_workspace_size(B, H, n, k.shape[2], D)
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=DEV) if nbytes else None
     if out is None:
         out = torch.zeros(B, H, Nq if scattered else n, D, dtype=BF, device=DEV)
@@ -392,7 +392,7 @@ def test_tail_split_matches_oracle(B, H, Nq, Nk, D, k_rows):
 def test_tail_split_scattered_state_and_errors():
     """Scattered output: the merge writes the S rows at their token index and
     leaves the context rows alone; a workspace smaller than asked for is
-    refused before any launch; kept masks are never split."""
+    refused before any launch."""
     B, H, N, D, kr = 1, 6, 1500, 96, 500
     q, k, v = _qkv(B, H, N, N, D, seed=1234)
     idx = _rand_idx(N, kr, seed=4321)
@@ -411,11 +411,59 @@ def test_tail_split_scattered_state_and_errors():
         sd().safedit_attn_subset_ws(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), kr, None, None, 0.0, out, 0,
                                     small)
     assert e.value.code == sd().ERR_INVALID_ARG
-    pad = torch.zeros(B, N, device=DEV)
-    assert sd().safedit_attn_subset_workspace_size(B, H, kr, N, D, True) == 0
-    o2, _ = run_ws(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), pad=pad)
-    o3 = run(q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV), pad=pad)
-    assert torch.equal(o2, o3)
+
+
+@pytest.mark.parametrize("D", [96, 128])
+@pytest.mark.parametrize("kind", ["pad", "bias_bf16", "pad_bias_bf16", "bias_f32"])
+def test_tail_split_with_kept_masks(D, kind):
+    """Kept masks through the tail-balanced launch (9 units of 16 key tiles,
+    each in 4 parts of 4 tiles): dead key tiles inside a part and one part
+    whose whole key range is padding (its rows leave nothing to the merge),
+    max jumps past the lazy-rescale threshold, a ragged last tile; against the
+    oracle and within tolerance of the whole-unit launch."""
+    B, H, N, kr = 1, 3, 2000, 600          # 16 key tiles, the last one 80 keys
+    q, k, v = _qkv(B, H, N, N, D, seed=3000 + D)
+    idx = _rand_idx(N, kr, seed=3001)
+    pad = bias = None
+    if "pad" in kind:
+        pad = torch.zeros(B, N)
+        pad[:, 512:1024] = float("-inf")    # tiles 4..7: all of part 1
+        pad[:, 1536:1664] = float("-inf")   # tile 12: the first tile of part 3
+        pad[:, 3::11] = float("-inf")
+        pad[:, 1100:1110] += 15.0           # a max jump in part 2
+    if "bias" in kind:
+        g = _gen(3002 + D)
+        bias = torch.randn(B, 1 if "bf16" in kind else H, N, N, generator=g) * 0.5
+        bias[..., ::2, 300:310] += 12.0     # part 0
+        bias[..., 1::2, 1900:1905] += 14.0  # the ragged tile, part 3
+        if "bf16" in kind:
+            bias = bias.to(BF)
+    dv = lambda t: None if t is None else t.to(DEV)  # noqa: E731
+    qd, kd, vd, idd = q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV)
+    out, nbytes = run_ws(qd, kd, vd, idd, pad=dv(pad), bias=dv(bias))
+    assert nbytes == 9 * 4 * 256 * (D + 2) * 4
+    for h in range(H):
+        ref = oracle_rows(q, k, v, idx.numpy(), 0, h, pad=pad, bias=bias)
+        check_attn(f64(out[0, h]), ref, f"{kind} D={D} h{h}")
+    whole = run(qd, kd, vd, idd, pad=dv(pad), bias=dv(bias))
+    check_attn(f64(out), f64(whole), "split vs whole units")
+
+
+def test_tail_split_fully_masked_rows():
+    """A batch whose every key is padding: no part has an admissible key, so
+    the merge reports SAFEDIT_ERR_MASKED_ROW and writes zeros, as the
+    whole-unit launch does; the other batch is unaffected."""
+    B, H, N, D, kr = 2, 2, 2000, 96, 700   # 3 x 4 = 12 units of 16 key tiles
+    q, k, v = _qkv(B, H, N, N, D, seed=4000)
+    idx = _rand_idx(N, kr, seed=4001)
+    pad = torch.zeros(B, N)
+    pad[1] = float("-inf")
+    qd, kd, vd, idd = q.to(DEV), k.to(DEV), v.to(DEV), idx.to(DEV)
+    out, nbytes = run_ws(qd, kd, vd, idd, pad=pad.to(DEV), status=sd().ERR_MASKED_ROW)
+    assert nbytes > 0
+    assert not out[1].any()
+    for h in range(H):
+        check_attn(f64(out[0, h]), oracle_rows(q, k, v, idx.numpy(), 0, h, pad=pad), f"h{h}")
 
 
 def test_tail_split_as_benchmarked():
