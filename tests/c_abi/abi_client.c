@@ -1,10 +1,11 @@
 /* A plain C client of libsafedit.so (include/safedit.h), with no Python in
  * the loop: device memory from the CUDA runtime, seeded inputs from a small
  * LCG, one SRSU subset-attention call (gathered rows over all keys, output
- * scattered into a state), the same rows with kept masks (key padding and an
- * f32 bias, compact output), one row-constant mask check and one SW-CFG
- * call, each compared with the fp64 oracle (test infrastructure,
- * liboracle.so).
+ * scattered into a state), the same rows through the tail-balanced entry
+ * points (a caller workspace, and the library's fixed array), the same rows
+ * with kept masks (key padding and an f32 bias, compact output), one
+ * row-constant mask check and one SW-CFG call, each compared with the fp64
+ * oracle (test infrastructure, liboracle.so).
  *
  *   abi_client          run the checks on the current CUDA device (exit 0 = pass)
  *   abi_client --abi    only the host-side argument checks (no GPU needed)
@@ -102,8 +103,9 @@ int main(int argc, char **argv) {
   if (argc > 1 && strcmp(argv[1], "--abi") == 0) return abi_checks();
   if (abi_checks()) return 1;
 
-  /* one (b, h) slice: N = 700 keys and queries, d = 96, 210 gathered rows */
-  const int64_t N = 700, d = 96, n_idx = 210;
+  /* one (b, h) slice: N = 1100 keys and queries (9 key tiles), d = 96, 330
+   * gathered rows (2 units of 256 rows) */
+  const int64_t N = 1100, d = 96, n_idx = 330;
   const size_t nel = (size_t)(N * d);
   uint16_t *hq = malloc(nel * 2), *hk = malloc(nel * 2), *hv = malloc(nel * 2), *ho = malloc(nel * 2);
   double *q = malloc(nel * 8), *k = malloc(nel * 8), *v = malloc(nel * 8);
@@ -165,6 +167,40 @@ int main(int argc, char **argv) {
   printf("attn_subset: relFro %.3e  max|err| %.3e  untouched rows %s\n", rel, mx,
          kept ? "ok" : "CHANGED");
   if (!(rel <= 5e-3 && mx <= 2e-2 && kept)) return 6;
+
+  /* the same call through the tail-balanced entry points: both units run as
+   * key-range parts merged afterwards, the partial results first in a
+   * caller workspace, then in the library's fixed array */
+  const size_t ws_bytes = safedit_attn_subset_workspace_size(1, 1, n_idx, N, (int32_t)d);
+  if (ws_bytes == 0) return 11;
+  void *dws;
+  CHECK_CUDA(cudaMalloc(&dws, ws_bytes));
+  for (int variant = 0; variant < 2; ++variant) {
+    CHECK_CUDA(cudaMemset(dout, 0, nel * 2));
+    if (variant == 0)
+      CHECK_SD(safedit_attn_subset_ws(&tq, &tk, &tv, (const int32_t *)didx, (int32_t)n_idx, NULL, NULL,
+                                      0.f, &to, 1, dws, ws_bytes, NULL));
+    else
+      CHECK_SD(safedit_attn_subset_noalloc(&tq, &tk, &tv, (const int32_t *)didx, (int32_t)n_idx, NULL,
+                                           NULL, 0.f, &to, 1, NULL));
+    CHECK_SD(safedit_get_device_status(&status, NULL));
+    if (status != SAFEDIT_OK) {
+      fprintf(stderr, "device status %s\n", safedit_status_string((safedit_status)status));
+      return 4;
+    }
+    CHECK_CUDA(cudaMemcpy(ho, dout, nel * 2, cudaMemcpyDeviceToHost));
+    double n2 = 0.0, d2 = 0.0, m2 = 0.0;
+    for (int64_t r = 0; r < n_idx; ++r)
+      for (int64_t c = 0; c < d; ++c) {
+        const double g = from_bf16(ho[(size_t)idx[r] * d + c]), e = ref[r * d + c];
+        n2 += (g - e) * (g - e), d2 += e * e;
+        if (fabs(g - e) > m2) m2 = fabs(g - e);
+      }
+    printf("%s (%zu-byte partials): relFro %.3e  max|err| %.3e\n",
+           variant == 0 ? "attn_subset_ws" : "attn_subset_noalloc", ws_bytes, sqrt(n2 / d2), m2);
+    if (!(sqrt(n2 / d2) <= 5e-3 && m2 <= 2e-2)) return 12;
+  }
+  CHECK_CUDA(cudaFree(dws));
 
   /* the same rows with kept masks, compact output: a key-padding vector (key
    * tile 2 -inf throughout, so it is skipped, plus scattered -inf keys) and a

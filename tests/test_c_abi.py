@@ -2,7 +2,8 @@
 is compiled with gcc against include/safedit.h and linked with libsafedit.so,
 the CUDA runtime and the oracle library (test infrastructure).  On the CPU it
 runs the host-side argument checks; on a GPU it also runs one SRSU attention
-(without and with kept masks), one mask check and one SW-CFG call against the
+(plain, tail-balanced with a caller workspace and with the library's fixed
+array, and with kept masks), one mask check and one SW-CFG call against the
 oracle."""
 import os
 import subprocess
