@@ -15,7 +15,9 @@
  * - Memory.  Every pointer named d_* and every safedit_tensor.data is DEVICE
  *   memory on the current CUDA device; host_* pointers are host memory.  The
  *   caller owns and allocates every buffer.  The library allocates nothing
- *   except one static device status word per device.  A pointer to an array
+ *   except one static device status word per device and the static scratch
+ *   array of safedit_attn_subset_noalloc (both reserved when the library's
+ *   device code loads, never at call time).  A pointer to an array
  *   with no elements (an empty tensor, a zero-length vector) may be NULL.
  * - Empty work.  A call whose work is empty (no rows, no tokens, no
  *   columns) checks its arguments, launches nothing and returns SAFEDIT_OK.
