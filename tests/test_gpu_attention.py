@@ -280,11 +280,14 @@ def test_config_2560_srsu_launch_as_benchmarked():
         check_attn(f64(got), ref, f"b{b}h{h}")
 
 
+@pytest.mark.parametrize("split", [False, True])
 @pytest.mark.parametrize("kind", ["pad", "bias_bf16", "pad+bias_bf16", "bias_f32"])
-def test_config_stress_kept_masks_sampled(kind):
-    """The mask-stress shape in the launch configuration the benchmark times
-    (blob-score rows scattered into the state), for every kept-mask variant;
-    sampled rows of two heads against the oracle."""
+def test_config_stress_kept_masks_sampled(kind, split):
+    """The mask-stress shape in the launch configurations the benchmark times
+    (blob-score rows scattered into the state; whole units, and tail-balanced:
+    the last 48 units, slices 29..31 from row block 12 of slice 29 on, in 3
+    key parts), for every kept-mask variant; sampled rows of a whole-unit head
+    and of a split one against the oracle."""
     w = wl.STRESS
     q, k, v = wl.qkv(w, device=DEV)
     score = wl.blob_scores(w).to(DEV)
@@ -299,7 +302,11 @@ def test_config_stress_kept_masks_sampled(kind):
         if kind.endswith("f32"):
             bias = bias.float()
     state = torch.zeros(w.B, w.H, w.N, w.d, dtype=BF, device=DEV)
-    run(q, k, v, idx, pad=pad, bias=bias, out=state, scattered=True)
+    if split:
+        _, nbytes = run_ws(q, k, v, idx, pad=pad, bias=bias, out=state, scattered=True)
+        assert nbytes == 48 * 3 * 256 * (w.d + 2) * 4
+    else:
+        run(q, k, v, idx, pad=pad, bias=bias, out=state, scattered=True)
     rows = np.linspace(0, w.k - 1, 24).astype(np.int64)
     ic = idx.cpu().numpy()
     for h in (0, 31):
