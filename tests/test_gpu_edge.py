@@ -33,6 +33,11 @@ def test_attention_without_rows():
     # no query rows at all
     q0 = torch.empty(1, 2, 0, 96, dtype=BF, device=DEV)
     _no_launch(lambda: sd().safedit_attn_subset(q0, k, k, None, 0, None, None, 0.0, out, 0))
+    # the tail-balanced entry points: no workspace needed, nothing launched
+    assert sd().safedit_attn_subset_workspace_size(1, 2, 0, 64, 96) == 0
+    _no_launch(lambda: sd().safedit_attn_subset_ws(q, k, k, idx, 0, None, None, 0.0, state, 1, None))
+    _no_launch(lambda: sd().safedit_attn_subset_noalloc(q, k, k, idx, 0, None, None, 0.0, state, 1))
+    assert torch.equal(state.view(torch.int16), before.view(torch.int16))
 
 
 def test_row_copies_without_rows():

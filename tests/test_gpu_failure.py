@@ -72,6 +72,37 @@ def test_bounded_wait_timeout_is_reported_and_context_survives():
     assert torch.equal(again_g, ref_g)
 
 
+def test_tail_split_timeout_is_reported_and_context_survives():
+    """The tail-balanced launch (whole units, key-range parts that may overlap
+    them, the merge) with the wait limit at 0: every CTA of both attention
+    launches gives up, the part launch still completes after the whole-unit
+    one, the status word reports SAFEDIT_ERR_TIMEOUT, and the next call
+    reproduces the reference bit for bit."""
+    g = torch.Generator().manual_seed(8)
+    q, k, v = (torch.randn(1, 50, 2000, 96, generator=g).to(torch.bfloat16).to(DEV) for _ in range(3))
+    idx = torch.arange(0, 2000, 3, dtype=torch.int32, device=DEV)[:600]
+    nb = sd().safedit_attn_subset_workspace_size(1, 50, 600, 2000, 96)
+    assert nb > 0  # 150 units: 148 whole, 2 in key parts
+    ws = torch.empty(nb, dtype=torch.uint8, device=DEV)
+
+    def run():
+        out = torch.zeros(1, 50, 600, 96, dtype=torch.bfloat16, device=DEV)
+        sd().safedit_attn_subset_ws(q, k, v, idx, 600, None, None, 0.0, out, 0, ws)
+        return out
+
+    ref = run()
+    expect_status(0)
+    old = sd().safedit_debug_set_wait_limit_ns(0)
+    try:
+        run()
+        expect_status(sd().ERR_TIMEOUT)
+    finally:
+        sd().safedit_debug_set_wait_limit_ns(old)
+    again = run()
+    expect_status(0)
+    assert torch.equal(again, ref)
+
+
 def test_device_errors_do_not_poison_later_calls():
     q, k, v, idx = _attn_case()
     ref = _run_attn(q, k, v, idx)
