@@ -25,7 +25,8 @@
  *   Every call only enqueues work on that stream and returns without
  *   synchronising, except safedit_get_device_status.
  * - Errors.  Argument errors are detected on the host and returned before
- *   any CUDA call is made (no launch happens).  Errors found on the device
+ *   any launch (at most the current device and its attributes are read).
+ *   Errors found on the device
  *   (an index out of range, a fully masked row, a pipeline wait that timed
  *   out) set the device status word, which safedit_get_device_status reads
  *   and clears; the outputs of the failing call are then unspecified.
@@ -34,7 +35,9 @@
  *   (strides[3] == 1) and every other stride a multiple of 8 elements
  *   (16 bytes); data must be 16-byte aligned.
  * - Threading.  Stateless and reentrant apart from the status word, the
- *   launch counter and the debug wait limit.
+ *   launch counter, the debug settings (wait limit, index check) and the
+ *   scratch array of safedit_attn_subset_noalloc, which calls that overlap
+ *   on one device share.
  */
 #ifndef SAFEDIT_H_
 #define SAFEDIT_H_
