@@ -200,21 +200,45 @@ def score_all_reduce(score):
     torch.distributed.all_reduce(score, op=torch.distributed.ReduceOp.SUM)
 
 
+def split_broadcast(tr):
+    """CFG-parallel generation: the S/C split and the sensitivity score are
+    made on the cond-branch rank (0), which alone has a prompt to score
+    against, and sent to the uncond-branch rank."""
+    for t in (tr.idx_s, tr.idx_c, tr.s):
+        torch.distributed.broadcast(t, src=0)
+
+
+def eps_all_gather(tr):
+    """CFG-parallel generation: each rank's branch prediction (rank 0 the
+    conditional, rank 1 the unconditional one) to both ranks, before the
+    guidance combine that needs the two."""
+    torch.distributed.all_gather([tr.eps_c, tr.eps_u], tr.eps_own)
+
+
 class Trajectory:
     """Device-resident buffers and the launch sequence of one trajectory.
     heads=(h0, h1) keeps only those heads of the (same, globally seeded)
     generation on this device; reduce_score then completes the PCSP score
-    over the other devices' heads before the split."""
+    over the other devices' heads before the split.  branch=b keeps only
+    batch entry b (0 = cond, 1 = uncond) of the self-attention tensors and of
+    the prediction; only the cond branch scores the tokens, share_split then
+    hands the split to the other branch's device, and exchange_eps gathers
+    both branches' predictions before every guidance combine."""
 
-    def __init__(self, w, dev, seed_step=0, heads=None, reduce_score=None, pcsp="fused"):
+    def __init__(self, w, dev, seed_step=0, heads=None, reduce_score=None, pcsp="fused", branch=None,
+                 share_split=None, exchange_eps=None):
         from spatially_adaptive_dit_b200 import safedit as sd
         self.sd, self.w, self.dev = sd, w, dev
         self.pcsp = pcsp  # "fused": one pcsp_score launch; "unfused": probabilities, then aggregation
-        B, N, d, L, k = w.B, w.N, w.d, w.L, w.k
+        N, d, L, k = w.N, w.d, w.L, w.k
         h0, h1 = (0, w.H) if heads is None else heads
-        H = h1 - h0
-        sl = (lambda t: t) if heads is None else (lambda t: t[:, h0:h1].contiguous())
+        b0, b1 = (0, w.B) if branch is None else (branch, branch + 1)
+        H, B = h1 - h0, b1 - b0
+        slh = (lambda t: t) if heads is None else (lambda t: t[:, h0:h1].contiguous())
+        sl = (lambda t: slh(t)) if branch is None else (lambda t: slh(t)[b0:b1].contiguous())
         self.reduce_score = reduce_score
+        self.branch, self.share_split, self.exchange_eps = branch, share_split, exchange_eps
+        self.pcsp_here = branch in (None, 0)  # the score comes from the cond branch
         self.k = k
         self.q, self.k_full, self.v_full = (sl(t) for t in wl.qkv(w, step=seed_step, device=dev))
         self.k_s, self.v_s = (sl(t) for t in wl.fresh_sensitive_kv(w, k, step=seed_step, device=dev))
@@ -224,7 +248,7 @@ class Trajectory:
         self.v_state.copy_(self.v_full)
         self.o_state = torch.zeros_like(self.q)
         self.q_img, self.k_txt, self.valid, self.content = wl.text(w, step=seed_step, device=dev)
-        self.q_img, self.k_txt = sl(self.q_img), sl(self.k_txt)
+        self.q_img, self.k_txt = slh(self.q_img), slh(self.k_txt)
         self.P = torch.empty(H, N, L, device=dev)
         self.score = torch.zeros(N, dtype=torch.float64, device=dev)
         self.idx_s = torch.empty(k, dtype=torch.int32, device=dev)
@@ -235,8 +259,9 @@ class Trajectory:
         self.mask = torch.zeros(B, 1, 1, N, dtype=torch.bfloat16, device=dev).expand(B, 1, N, N)
         self.verdict = torch.zeros(1, dtype=torch.int32, device=dev)
         self.eps_c, self.eps_u = wl.cfg_preds(w, step=seed_step, device=dev)
+        self.eps_own = None if branch is None else (self.eps_c, self.eps_u)[branch].clone()
         self.cfg_out = torch.empty_like(self.eps_c)
-        self.H = H
+        self.H, self.B = H, B
         # tail-balanced attention: one workspace per launch shape (S rows,
         # all rows), as large as the launch plan asks (none where it keeps
         # whole units, as at 2560^2)
@@ -285,19 +310,21 @@ class Trajectory:
         self.score.zero_()
         for t in range(w.steps):
             anchor = (t % w.period == 0)
-            if t < w.warmup and self.pcsp == "fused":  # PCSP warm-up on the cond branch
+            if t < w.warmup and self.pcsp_here and self.pcsp == "fused":  # PCSP warm-up on the cond branch
                 timed("pcsp_score", lambda: sd.safedit_pcsp_score(
                     self.q_img, self.k_txt, self.valid, self.content, 0, 0.0, self.score, stream))
-            elif t < w.warmup:
+            elif t < w.warmup and self.pcsp_here:
                 timed("cross_attn_probs", lambda: sd.safedit_cross_attn_probs(
                     self.q_img, self.k_txt, self.valid, 0, 0.0, self.P, stream))
                 timed("partition_accumulate", lambda: sd.safedit_partition_accumulate(
                     self.P, self.content, self.score, stream))
             if t == w.warmup - 1 and self.reduce_score is not None:
                 timed("score_all_reduce", lambda: self.reduce_score(self.score))
-            if t == w.warmup - 1:
+            if t == w.warmup - 1 and self.pcsp_here:
                 timed("partition_finalize", lambda: sd.safedit_partition_finalize(
                     self.score, w.N, self.k, self.idx_s, self.idx_c, self.s, stream))
+            if t == w.warmup - 1 and self.share_split is not None:
+                timed("split_broadcast", lambda: self.share_split(self))
             if t == 0:
                 timed("mask_is_row_constant", lambda: sd.safedit_mask_is_row_constant(
                     self.mask, self.verdict, None, stream))
@@ -314,6 +341,8 @@ class Trajectory:
                     self.q, self.k_state, self.v_state, self.idx_s, self.k, self.o_state, 1, stream))
             g_ctx = w.gamma_ctx
             g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx  # global CFG before the split
+            if self.exchange_eps is not None:
+                timed("eps_exchange", lambda: self.exchange_eps(self))
             timed("sw_cfg", lambda: sd.safedit_sw_cfg(self.eps_c, self.eps_u, self.s, g_ctx, g_sens,
                                                        self.cfg_out, stream))
 
@@ -326,8 +355,15 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     from spatially_adaptive_dit_b200 import safedit as sd
-    sharded = args.shard == "heads" and ws > 1
-    if sharded:  # one generation, H / ws heads per GPU, one score all-reduce
+    sharded = args.shard in ("heads", "cfg") and ws > 1
+    if sharded and args.shard == "cfg":
+        # one generation, its cond / uncond branches on two GPUs: the split
+        # broadcast once, the branch predictions gathered every step
+        if ws != 2:
+            raise SystemExit("--shard cfg puts the two guidance branches on exactly 2 GPUs")
+        tr = Trajectory(W, dev, seed_step=0, branch=rank, share_split=split_broadcast,
+                        exchange_eps=eps_all_gather, pcsp=args.pcsp)
+    elif sharded:  # one generation, H / ws heads per GPU, one score all-reduce
         tr = Trajectory(W, dev, seed_step=0, heads=head_range(W.H, ws, rank), reduce_score=score_all_reduce,
                         pcsp=args.pcsp)
     else:  # independent replicas
@@ -339,7 +375,7 @@ def run_ours(args):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     state_bytes = tr.k_state.numel() * tr.k_state.element_size()
     flush = L2Flush(dev) if 2 * state_bytes < 2 * l2 else None
-    l2_note = (f"per-device K/V state {2 * state_bytes / 1e6:.0f} MB fits in L2 ({l2 / 1e6:.0f} MB): L2 flushed "
+    l2_note = (f"per-device K/V state {2 * state_bytes / 1e6:.0f} MB under twice the L2 ({l2 / 1e6:.0f} MB): L2 flushed "
                f"({4 * l2 / 1e6:.0f} MB write) before every attention and scatter launch, outside their events"
                if flush is not None else
                f"inputs larger than L2 (Q/K/V/state {state_bytes / 1e6:.0f} MB each per device, L2 "
@@ -429,7 +465,11 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": W.B if sharded else W.B * ws, "seq_len": W.N,
-                       "parallelism": (f"heads x{ws} (one generation, {W.H // ws} heads per GPU; one all-reduce "
+                       "parallelism": ("cfg x2 (one generation, its cond and uncond branches on one GPU each; "
+                                       "the S/C split and s broadcast once from the cond branch, the two "
+                                       "branch predictions all-gathered before every guidance combine)")
+                                      if sharded and args.shard == "cfg" else
+                                      (f"heads x{ws} (one generation, {W.H // ws} heads per GPU; one all-reduce "
                                        "of the fp64 score vector after the warm-up)") if sharded else
                                       f"replicas x{ws} (independent trajectories, no collective)",
                        "l2": l2_note,
@@ -450,7 +490,7 @@ def run_ours(args):
                        "note": f"this device's buffers of the attention path ({tr.H} heads) incl. the "
                                f"{tr.P.numel() * 4 / 1e9:.2f} GB probability tensor; a dense masked path that "
                                "materialises bf16 scores [B,H,N,N] would need "
-                               f"{W.B * tr.H * W.N * W.N * 2 / 1e9:.1f} GB for them alone"},
+                               f"{tr.B * tr.H * W.N * W.N * 2 / 1e9:.1f} GB for them alone"},
             "device_status": status,
             "extensions": ext,
             "e2e": {"value": round(whole_job_tflops(tr.flop_srsu * n_srsu / args.steps, ws, e2e["ms"]), 3),
@@ -488,7 +528,7 @@ def _srsu_algorithmic_bytes(tr):
     """Bytes one SRSU launch must move at least: K and V of every slice read
     once, the gathered Q rows read and the output rows written."""
     w = tr.w
-    return (2 * w.N + 2 * tr.k) * w.d * 2 * w.B * tr.H + 4 * tr.k
+    return (2 * w.N + 2 * tr.k) * w.d * 2 * tr.B * tr.H + 4 * tr.k
 
 
 def measure_extensions(tr, stream, dev, unfused_pcsp_ms):
@@ -764,8 +804,11 @@ def run_e2e(tr, stream, args):
     NSET = 4
     q_s = tr.q[:, :, : tr.k].contiguous()
     o_s = torch.empty_like(q_s)
-    srsu_src = [q_s, tr.k_s, tr.v_s, tr.eps_c, tr.eps_u]
-    anchor_src = [tr.q, tr.k_full, tr.v_full, tr.eps_c, tr.eps_u]
+    # each step's predictions: both, or (one branch per device) this branch's,
+    # gathered with the other device's before the guidance combine
+    eps_src = [tr.eps_c, tr.eps_u] if tr.branch is None else [tr.eps_own]
+    srsu_src = [q_s, tr.k_s, tr.v_s] + eps_src
+    anchor_src = [tr.q, tr.k_full, tr.v_full] + eps_src
     text_src = [tr.q_img, tr.k_txt]
     h_srsu, hv = _packed(srsu_src, pin=True)
     for v, t in zip(hv, srsu_src):
@@ -776,8 +819,8 @@ def run_e2e(tr, stream, args):
     h_text, hv = _packed(text_src, pin=True)
     for v, t in zip(hv, text_src):
         v.copy_(t)
-    sets = [_packed(srsu_src, device=tr.dev) for _ in range(NSET)]      # (block, [q_s, k_s, v_s, c, u])
-    states = [_packed(anchor_src, device=tr.dev) for _ in range(2)]    # (block, [q, k, v, c, u])
+    sets = [_packed(srsu_src, device=tr.dev) for _ in range(NSET)]      # (block, [q_s, k_s, v_s, eps...])
+    states = [_packed(anchor_src, device=tr.dev) for _ in range(2)]    # (block, [q, k, v, eps...])
     d_text = _packed(text_src, device=tr.dev)
     out_h = [torch.empty(tr.cfg_out.shape, dtype=tr.cfg_out.dtype, pin_memory=True) for _ in range(NSET)]
     copy_stream = torch.cuda.Stream(device=tr.dev)
@@ -795,7 +838,7 @@ def run_e2e(tr, stream, args):
             anchor = (t % w.period == 0)
             ready = torch.cuda.Event()
             with torch.cuda.stream(copy_stream):
-                if t < w.warmup:
+                if t < w.warmup and tr.pcsp_here:
                     if text_freed[0] is not None:
                         copy_stream.wait_event(text_freed[0])
                     d_text[0].copy_(h_text, non_blocking=True)
@@ -814,10 +857,10 @@ def run_e2e(tr, stream, args):
                 if count:
                     counts["h2d"] += src.numel()
                 ready.record(copy_stream)
-            aq, k_st, v_st, a_c, a_u = states[cur_state[0]][1]
+            aq, k_st, v_st, *a_eps = states[cur_state[0]][1]
             stream.wait_event(ready)
             with torch.cuda.stream(stream):
-                if t < w.warmup:
+                if t < w.warmup and tr.pcsp_here:
                     q_img, k_txt = d_text[1]
                     if tr.pcsp == "fused":
                         sd.safedit_pcsp_score(q_img, k_txt, tr.valid, tr.content, 0, 0.0, tr.score, stream)
@@ -829,18 +872,26 @@ def run_e2e(tr, stream, args):
                     text_freed[0] = ev
                 if t == w.warmup - 1 and tr.reduce_score is not None:
                     tr.reduce_score(tr.score)
-                if t == w.warmup - 1:
+                if t == w.warmup - 1 and tr.pcsp_here:
                     sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s, stream)
+                if t == w.warmup - 1 and tr.share_split is not None:
+                    tr.share_split(tr)
                 if t == 0:
                     sd.safedit_mask_is_row_constant(tr.mask, tr.verdict, None, stream)
                 if anchor:
-                    eps_c, eps_u = a_c, a_u
+                    eps = a_eps
                     tr.attn(aq, k_st, v_st, None, 0, tr.o_state, 0, stream)
                 else:
-                    qs, ks, vs, eps_c, eps_u = sets[t % NSET][1]
+                    qs, ks, vs, *eps = sets[t % NSET][1]
                     sd.safedit_scatter_state([ks, vs], [k_st, v_st], tr.idx_s, tr.k, stream)
                     tr.attn(qs, k_st, v_st, None, 0, o_s, 0, stream)
                     sd.safedit_scatter_state([o_s], [tr.o_state], tr.idx_s, tr.k, stream)
+                if tr.branch is None:
+                    eps_c, eps_u = eps
+                else:  # this branch's prediction as uploaded, the other one from its device
+                    tr.eps_own.copy_(eps[0])
+                    tr.exchange_eps(tr)
+                    eps_c, eps_u = tr.eps_c, tr.eps_u
                 g_sens = w.gamma_sens if t >= w.warmup else w.gamma_ctx
                 sd.safedit_sw_cfg(eps_c, eps_u, tr.s, w.gamma_ctx, g_sens, tr.cfg_out, stream)
                 out_h[t % NSET].copy_(tr.cfg_out, non_blocking=True)
@@ -1222,9 +1273,10 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
-                    help="N > 1: independent replicas (default, weak scaling) or one generation split by heads "
-                         "(strong scaling; the PCSP score is all-reduced once)")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads", "cfg"],
+                    help="N > 1: independent replicas (default, weak scaling), one generation split by heads "
+                         "(strong scaling; the PCSP score is all-reduced once), or, on 2 GPUs, one generation "
+                         "split by guidance branch (the split broadcast once, the predictions gathered every step)")
     ap.add_argument("--pcsp", default="fused", choices=["fused", "unfused"],
                     help="PCSP warm-up in the timed trajectory: the fused score kernel (default) or the "
                          "probabilities kernel followed by the aggregation")

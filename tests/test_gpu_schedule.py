@@ -124,3 +124,46 @@ def test_head_sharded_trajectory_split_matches_unsharded(pcsp):
     if not near:
         assert torch.equal(lo.idx_s, full.idx_s)
         assert torch.equal(lo.o_state, full.o_state[:, :12])
+
+
+def test_guidance_branch_sharded_trajectory_matches_unsharded():
+    """The benchmark's guidance-branch split on one GPU: two trajectories of
+    the 1024^2 workload keep batch entry 0 (cond) and 1 (uncond) of the same
+    seeded generation; only the cond one scores the tokens, the uncond one
+    takes its split through the share hook, and each takes the other's
+    branch prediction through the exchange hook (standing in for the
+    broadcast and the all-gather).  Split and guided output must equal the
+    unsharded trajectory's exactly, each branch's state rows bit for bit, and
+    its attention output within the attention tolerance (the two launch
+    shapes may take different tail-balancing plans)."""
+    import bench
+    w = wl.W1024
+    dev = torch.device(DEV)
+    stream = torch.cuda.Stream()
+    full = bench.Trajectory(w, dev)
+    with torch.cuda.stream(stream):
+        full.run(stream)
+    stream.synchronize()
+    br = {}
+
+    def share(tr):
+        if tr.branch == 1:
+            for name in ("idx_s", "idx_c", "s"):
+                getattr(tr, name).copy_(getattr(br[0], name))
+
+    def exchange(tr):
+        tr.eps_c.copy_(br[0].eps_own)
+        tr.eps_u.copy_(br[1].eps_own)
+
+    for b in (0, 1):
+        br[b] = bench.Trajectory(w, dev, branch=b, share_split=share, exchange_eps=exchange)
+    for b in (0, 1):
+        with torch.cuda.stream(stream):
+            br[b].run(stream)
+        stream.synchronize()
+    expect_status(0)
+    for b in (0, 1):
+        assert torch.equal(br[b].idx_s, full.idx_s) and torch.equal(br[b].s, full.s)
+        assert torch.equal(br[b].cfg_out, full.cfg_out)
+        assert torch.equal(br[b].k_state, full.k_state[b:b + 1])
+        check_attn(br[b].o_state.double().cpu().numpy(), full.o_state[b:b + 1].double().cpu().numpy(), f"branch {b}")

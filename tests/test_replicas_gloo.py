@@ -107,3 +107,61 @@ def test_two_gloo_ranks_head_sharded_split_matches_one_process():
         assert err <= 1e-14
         assert idx_rank == idx_full
     assert res[0][1] == res[1][1]
+
+
+def _cfg_rank(rank, world, port, out):
+    """One rank of a generation split by guidance branch: rank 0 (cond)
+    makes the split from its scores, the benchmark's broadcast hands it to
+    rank 1 (uncond); the two branch predictions are then gathered on both
+    ranks for the guidance combine."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+    import types
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    import numpy as np
+    import bench
+    import oracle
+    H, N, L, k, F = 4, 96, 16, 29, 8
+    g = torch.Generator()
+    g.manual_seed(11)
+    P = torch.rand(H, N, L, generator=g)
+    eps = [torch.randn(N, F, generator=g), torch.randn(N, F, generator=g)]  # cond, uncond
+    content = torch.zeros(L, dtype=torch.uint8)
+    content[1:L - 1] = 1
+    tr = types.SimpleNamespace(idx_s=torch.zeros(k, dtype=torch.int32), idx_c=torch.zeros(N - k, dtype=torch.int32),
+                               s=torch.zeros(N), eps_c=torch.zeros(N, F), eps_u=torch.zeros(N, F),
+                               eps_own=eps[rank].clone())
+    if rank == 0:  # only the cond branch has a prompt to score the tokens against
+        s_idx, c_idx, sv = oracle.partition_select(oracle.partition_accumulate(P, content), k)
+        tr.idx_s.copy_(torch.from_numpy(s_idx))
+        tr.idx_c.copy_(torch.from_numpy(c_idx))
+        tr.s.copy_(torch.from_numpy(sv))
+    bench.split_broadcast(tr)
+    bench.eps_all_gather(tr)
+    cfg = oracle.sw_cfg(tr.eps_c.double(), tr.eps_u.double(), tr.s, 3.0, 5.0)
+    ref_split = oracle.partition_select(oracle.partition_accumulate(P, content), k)
+    ref_cfg = oracle.sw_cfg(eps[0].double(), eps[1].double(), torch.from_numpy(ref_split[2]), 3.0, 5.0)
+    dist.barrier()
+    out[rank] = (tr.idx_s.tolist() == ref_split[0].tolist() and tr.idx_c.tolist() == ref_split[1].tolist()
+                 and bool(np.array_equal(tr.s.numpy(), ref_split[2])),
+                 bool(torch.equal(tr.eps_c, eps[0]) and torch.equal(tr.eps_u, eps[1])),
+                 bool(np.array_equal(cfg, ref_cfg)))
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_two_gloo_ranks_guidance_branch_split():
+    """Guidance-branch sharding of one generation: the uncond rank receives
+    the cond rank's split and sensitivity score exactly, both ranks end up
+    with both branch predictions, and their guidance combine equals the
+    single-process one."""
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_cfg_rank, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+        res = dict(out)
+    for r in range(world):
+        assert res[r] == (True, True, True), (r, res[r])
