@@ -14,7 +14,9 @@ launches of the timed steps, timed with CUDA events on the launching stream;
 whole-job aggregate over ranks (sum of flop / max of per-rank time).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-(for N > 1 launch under torchrun; each rank runs its own independent replica).
+(for N > 1 launch under torchrun; by default each rank runs its own independent
+replica; --shard heads splits one generation by heads, --shard cfg on 2 GPUs by
+guidance branch).
 """
 import argparse
 import json
