@@ -4,8 +4,10 @@
 //     16-byte groups of P that hold a content column (padding is never
 //     read), fp64 accumulation and a warp-shuffle reduction;
 //   * partition_finalize: the top-k split (ties to the lower index) by an
-//     8-pass radix select on order-preserving 64-bit keys, a stable
-//     block-scan compaction into ascending S / C index lists, and the
+//     8-pass radix select on order-preserving 64-bit keys (held in shared
+//     memory up to 28800 tokens; warp-aggregated histogram), a stable
+//     compaction into ascending S / C index lists (a contiguous token range
+//     per warp, ballots within it, one scan over the warps), and the
 //     min-max sensitivity score s -- one CTA, once per trajectory.
 #include "common.cuh"
 #include "internal.h"
@@ -136,66 +138,65 @@ __device__ __forceinline__ uint64_t score_key(double x) {
   const uint64_t u = static_cast<uint64_t>(__double_as_longlong(x));
   return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
-
-// Exclusive block scan of one int per thread (kFinThreads threads); returns
-// the exclusive prefix and writes the block total to *total.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_sums[wid] = x;
-  __syncthreads();
-  if (wid == 0) {
-    int w = warp_sums[lane];
-    int s = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    warp_sums[lane] = s - w;  // exclusive prefix of warp totals
-    if (lane == 31) *total = s;
-  }
-  __syncthreads();
-  const int r = warp_sums[wid] + x - v;
-  __syncthreads();
-  return r;
+// Its inverse (a -0 score comes back as +0, which s treats alike).
+__device__ __forceinline__ double key_score(uint64_t key) {
+  const uint64_t u = (key >> 63) ? (key & 0x7FFFFFFFFFFFFFFFull) : ~key;
+  return __longlong_as_double(static_cast<long long>(u));
 }
+
+
+// Keys kept in shared memory for n up to this many tokens (224 KB, with the
+// kernel's static 2 KB under the 227 KB a CTA may hold); larger calls read
+// the scores from global memory in every pass.
+constexpr int kFinCacheKeys = 28672;
 
 __global__ void __launch_bounds__(kFinThreads, 1)
     finalize_kernel(const double* __restrict__ score, int n, int k, int* __restrict__ idx_s,
                     int* __restrict__ idx_c, float* __restrict__ s_out, int* status) {
+  extern __shared__ uint64_t skeys[];  // the n order-preserving keys, when cached
   __shared__ unsigned int hist[256];
-  __shared__ int warp_sums[32];
-  __shared__ int total;
+  __shared__ int wcount[2][32];        // per warp: keys equal to T, keys selected
+  __shared__ int wbase[2][32];         // exclusive prefixes of the same over warps
   __shared__ uint64_t sh_prefix;
   __shared__ int sh_need;
   __shared__ double red_lo[32], red_hi[32];
   __shared__ int sh_nan;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const bool cached = n <= kFinCacheKeys;
+  auto key_at = [&](int i) -> uint64_t { return cached ? skeys[i] : score_key(score[i]); };
   if (tid == 0) sh_nan = 0;
   __syncthreads();
 
-  // min / max (exact, order independent) and the NaN check
+  // min / max (exact, order independent), the NaN check, the key cache
   double lo = INFINITY, hi = -INFINITY;
-  for (int i = tid; i < n; i += kFinThreads) {
-    const double x = score[i];
-    if (isnan(x)) sh_nan = 1;
-    lo = fmin(lo, x);
-    hi = fmax(hi, x);
+  bool nan_seen = false;
+  for (int base = tid; base < n; base += 4 * kFinThreads) {
+    double x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * kFinThreads;
+      x[u] = i < n ? score[i] : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * kFinThreads;
+      if (i < n) {
+        nan_seen |= isnan(x[u]);
+        lo = fmin(lo, x[u]);
+        hi = fmax(hi, x[u]);
+        if (cached) skeys[i] = score_key(x[u]);
+      }
+    }
   }
+  if (nan_seen) sh_nan = 1;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lo = fmin(lo, __shfl_xor_sync(0xffffffffu, lo, o));
     hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
-  if ((tid & 31) == 0) {
-    red_lo[tid >> 5] = lo;
-    red_hi[tid >> 5] = hi;
+  if (lane == 0) {
+    red_lo[wid] = lo;
+    red_hi[wid] = hi;
   }
   __syncthreads();
   if (tid < 32) {
@@ -220,27 +221,57 @@ __global__ void __launch_bounds__(kFinThreads, 1)
   uint64_t prefix = 0, pmask = 0;
   int remaining = k;
   if (k > 0 && k < n) {
+    constexpr int U = 4;  // keys of a thread in flight per round
+    const int n_up = (n + U * kFinThreads - 1) / (U * kFinThreads) * (U * kFinThreads);
     for (int pass = 0; pass < 8; ++pass) {
       const int shift = 56 - 8 * pass;
       for (int b = tid; b < 256; b += kFinThreads) hist[b] = 0;
       __syncthreads();
-      for (int i = tid; i < n; i += kFinThreads) {
-        const uint64_t key = score_key(score[i]);
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFF], 1u);
+      for (int base = tid; base < n_up; base += U * kFinThreads) {
+        uint64_t kk[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int i = base + u * kFinThreads;
+          kk[u] = i < n ? key_at(i) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int i = base + u * kFinThreads;
+          const uint32_t bin = (i < n && (kk[u] & pmask) == prefix) ? uint32_t(kk[u] >> shift) & 0xFFu : 256u;
+          // one shared-memory atomic per distinct byte in the warp (the keys
+          // of a pass share a few leading bytes: per-lane atomics serialise)
+          const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+          if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], uint32_t(__popc(peers)));
+        }
       }
       __syncthreads();
-      if (tid == 0) {
-        int cum = 0, sel = 0;
-        for (int b = 255; b >= 0; --b) {
-          const int c = static_cast<int>(hist[b]);
-          if (cum + c >= remaining) {
-            sel = b;
-            break;
-          }
-          cum += c;
+      if (tid < 32) {
+        // lane l holds bins 255 - 8 l down to 248 - 8 l (larger keys first)
+        uint32_t c[8], sum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          c[e] = hist[255 - 8 * lane - e];
+          sum += c[e];
         }
-        sh_prefix = prefix | (uint64_t(sel) << shift);
-        sh_need = remaining - cum;
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        // the candidates of this pass number at least `remaining`, so some lane hits
+        const uint32_t hit = __ballot_sync(0xffffffffu, incl >= uint32_t(remaining));
+        if (lane == __ffs(hit) - 1) {
+          uint32_t cum = incl - sum;
+          int sel = -1;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (sel < 0 && cum + c[e] >= uint32_t(remaining)) sel = 255 - 8 * lane - e;
+            if (sel < 0) cum += c[e];
+          }
+          sh_prefix = prefix | (uint64_t(sel) << shift);
+          sh_need = remaining - int(cum);
+        }
       }
       __syncthreads();
       prefix = sh_prefix;
@@ -254,37 +285,79 @@ __global__ void __launch_bounds__(kFinThreads, 1)
   const uint64_t T = prefix;
   const int need_eq = remaining;
 
-  int eq_before = 0, sel_before = 0;
-  for (int base = 0; base < n; base += kFinThreads) {
-    const int i = base + tid;
-    const bool in = i < n;
-    uint64_t key = 0;
-    double x = 0.0;
-    if (in) {
-      x = score[i];
-      key = score_key(x);
+  // stable compaction in token order: warp w owns the contiguous range
+  // [w0, w1), walked 32 tokens at a time (coalesced); per-warp counts, one
+  // scan over the 32 warps, then every token's place from ballots
+  const int per_warp = ((n + 31) / 32 + 31) / 32 * 32;
+  const int w0 = min(n, wid * per_warp), w1 = min(n, w0 + per_warp);
+  const uint32_t lt = (1u << lane) - 1u;
+  auto classify = [&](int i, bool& eq, bool& gt) {
+    eq = gt = false;
+    if (i >= w1) return;
+    if (k >= n) {
+      gt = true;
+    } else if (k > 0) {
+      const uint64_t key = key_at(i);
+      eq = key == T;
+      gt = key > T;
     }
-    bool sel;
-    if (k == 0)
-      sel = false;
-    else if (k >= n)
-      sel = in;
-    else {
-      const int eq = (in && key == T) ? 1 : 0;
-      const int eq_rank = eq_before + block_exclusive_scan(eq, warp_sums, &total);
-      eq_before += total;
-      sel = in && (key > T || (eq && eq_rank < need_eq));
+  };
+  int n_eq = 0, n_gt = 0;
+  for (int b0 = w0; b0 < w1; b0 += 32) {
+    bool eq, gt;
+    classify(b0 + lane, eq, gt);
+    n_eq += __popc(__ballot_sync(0xffffffffu, eq));
+    n_gt += __popc(__ballot_sync(0xffffffffu, gt));
+  }
+  if (lane == 0) {
+    wcount[0][wid] = n_eq;
+    wcount[1][wid] = n_gt;
+  }
+  __syncthreads();
+  if (tid < 32) {
+    // exclusive scan of the equal counts, then of the selected counts (the
+    // keys greater than T, plus the equal ones whose rank is below need_eq)
+    const int e = wcount[0][lane];
+    int incl = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    const int pos_s = sel_before + block_exclusive_scan(sel ? 1 : 0, warp_sums, &total);
-    sel_before += total;
-    if (in) {
+    const int eb = incl - e;
+    const int sel = wcount[1][lane] + max(0, min(e, need_eq - eb));
+    int incl_s = sel;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl_s, o);
+      if (lane >= o) incl_s += y;
+    }
+    wbase[0][lane] = eb;
+    wbase[1][lane] = incl_s - sel;
+  }
+  __syncthreads();
+  int eq_rank = wbase[0][wid], pos_s = wbase[1][wid];
+  for (int b0 = w0; b0 < w1; b0 += 32) {
+    const int i = b0 + lane;
+    bool eq, gt;
+    classify(i, eq, gt);
+    const uint32_t eq_bits = __ballot_sync(0xffffffffu, eq);
+    const bool sel = gt || (eq && eq_rank + __popc(eq_bits & lt) < need_eq);
+    const uint32_t sel_bits = __ballot_sync(0xffffffffu, sel);
+    const int pos = pos_s + __popc(sel_bits & lt);
+    if (i < w1) {
       if (sel) {
-        if (idx_s && pos_s < k) idx_s[pos_s] = i;
+        if (idx_s && pos < k) idx_s[pos] = i;
       } else {
-        if (idx_c && i - pos_s < n - k) idx_c[i - pos_s] = i;
+        if (idx_c && i - pos < n - k) idx_c[i - pos] = i;
       }
-      if (s_out) s_out[i] = (hi == lo) ? 0.0f : __double2float_rn((x - lo) / (hi - lo));
+      if (s_out) {
+        const double x = cached ? key_score(skeys[i]) : score[i];
+        s_out[i] = (hi == lo) ? 0.0f : __double2float_rn((x - lo) / (hi - lo));
+      }
     }
+    eq_rank += __popc(eq_bits);
+    pos_s += __popc(sel_bits);
   }
 }
 
@@ -360,8 +433,11 @@ safedit_status safedit_partition_finalize(const double* d_score, int32_t n, int3
   if (!d_score) return SAFEDIT_ERR_INVALID_ARG;
   int* status = status_ptr();
   if (!status) return SAFEDIT_ERR_CUDA;
-  finalize_kernel<<<1, kFinThreads, 0, static_cast<cudaStream_t>(stream)>>>(d_score, n, k, d_idx_s,
-                                                                            d_idx_c, d_s, status);
+  const int cache_bytes = n <= kFinCacheKeys ? n * 8 : 0;
+  safedit_status st = set_smem(reinterpret_cast<const void*>(finalize_kernel), kFinCacheKeys * 8);
+  if (st != SAFEDIT_OK) return st;
+  finalize_kernel<<<1, kFinThreads, cache_bytes, static_cast<cudaStream_t>(stream)>>>(d_score, n, k, d_idx_s,
+                                                                                      d_idx_c, d_s, status);
   return after_launch(1);
 }
 

@@ -331,3 +331,38 @@ def test_stepcache_sw_cfg_large_sampled():
     mag = (1 + abs(w)) * sum(t.abs() for t in sub).double().numpy()
     err = np.abs(out[rows].cpu().double().numpy() - ref)
     assert np.all(err <= CFG_REL * (1 + gam) * mag + 1e-30)
+
+
+@pytest.mark.parametrize("n", [1, 3, 1000, 1024, 1025, 36864])
+def test_partition_finalize_sizes_and_degenerate_scores(n):
+    """Sizes below, at and above one token per thread (the compaction gives
+    each of the 1024 threads a contiguous run of tokens) and the 3072^2 token
+    count; all-equal scores (every token ties: the lowest indices win,
+    s = 0) and scores in a few distinct values.  (The oracle's selection is
+    quadratic: the large size takes one k.)"""
+    g = _gen(n + 5)
+    for kind in ("random", "equal", "few"):
+        if kind == "random":
+            score = torch.randn(n, generator=g, dtype=torch.float64)
+        elif kind == "equal":
+            score = torch.full((n,), 0.25, dtype=torch.float64)
+        else:
+            score = torch.randint(-3, 4, (n,), generator=g).double() * 0.5
+        for k in (sorted({0, 1, n // 3, n - 1, n}) if n <= 1025 else [n // 3]):
+            idx_s = torch.full((max(k, 1),), -7, dtype=torch.int32, device=DEV)
+            idx_c = torch.full((max(n - k, 1),), -7, dtype=torch.int32, device=DEV)
+            s = torch.empty(n, device=DEV)
+            sd().safedit_partition_finalize(score.to(DEV), n, k, idx_s, idx_c, s)
+            expect_status(0)
+            r_s, r_c, r_sv = oracle.partition_select(score.numpy(), k)
+            assert np.array_equal(idx_s.cpu().numpy()[:k], r_s), (kind, k)
+            assert np.array_equal(idx_c.cpu().numpy()[:n - k], r_c), (kind, k)
+            assert np.array_equal(s.cpu().numpy(), r_sv), (kind, k)
+
+
+def test_partition_finalize_nan_score_is_reported():
+    score = torch.randn(5000, dtype=torch.float64)
+    score[1234] = float("nan")
+    idx_s = torch.empty(100, dtype=torch.int32, device=DEV)
+    sd().safedit_partition_finalize(score.to(DEV), 5000, 100, idx_s, None, None)
+    expect_status(sd().ERR_INVALID_ARG)
