@@ -33,6 +33,12 @@
 //     ring, the bias one pass ahead through per-warp cp.async staging; each
 //     key tile in passes of 64 (f32 bias: 32) columns; key tiles whose pad is
 //     -inf throughout are skipped by every role; every exponential on MUFU.
+//   * schedule: units of 256 query rows of one (b, h) slice.  A plain call
+//     runs every unit whole; the tail-balanced call runs the units that fill
+//     whole waves in one launch and cuts the last wave's units into key-range
+//     parts (a second launch, SPLIT, overlapping the first one's drain by
+//     programmatic dependent launch) whose partial O, max and sum
+//     attn_merge_kernel combines.
 // Every mbarrier wait is bounded; an expired wait raises the CTA's abort
 // flag, drains in-flight TMA loads and MMAs, frees TMEM and returns.
 #include <cmath>
