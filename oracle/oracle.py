@@ -11,7 +11,6 @@ int32), following the definitions cited in oracle.c.
 """
 import ctypes
 import math
-import os
 
 import numpy as np
 
