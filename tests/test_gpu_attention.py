@@ -456,6 +456,32 @@ def test_tail_split_with_kept_masks(D, kind):
     check_attn(f64(out), f64(whole), "split vs whole units")
 
 
+def test_tail_split_bad_index_and_explicit_scale():
+    """Through the key-range parts and the merge: an out-of-range index sets
+    SAFEDIT_ERR_INDEX and its row is skipped (neither written by a part nor
+    by the merge); an explicit scale reaches every part."""
+    B, H, N, D, kr = 1, 3, 2000, 96, 600     # 9 units in 4 key parts
+    q, k, v = _qkv(B, H, N, N, D, seed=5000)
+    idx = _rand_idx(N, kr, seed=5001)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    nbytes = sd().safedit_attn_subset_workspace_size(B, H, kr, N, D)
+    assert nbytes > 0
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+    out = torch.zeros(B, H, kr, D, dtype=BF, device=DEV)
+    sd().safedit_attn_subset_ws(qd, kd, vd, idx.to(DEV), kr, None, None, 0.3, out, 0, ws)
+    expect_status(0)
+    for h in (0, 2):
+        check_attn(f64(out[0, h]), oracle_rows(q, k, v, idx.numpy(), 0, h, scale=0.3), f"scale h{h}")
+    bad = idx.clone()
+    bad[300] = N + 5
+    out = torch.full((B, H, kr, D), 7.0, dtype=BF, device=DEV)
+    sd().safedit_attn_subset_ws(qd, kd, vd, bad.to(DEV), kr, None, None, 0.0, out, 0, ws)
+    expect_status(sd().ERR_INDEX)
+    assert torch.all(out[:, :, 300] == 7.0)
+    keep = [r for r in range(kr) if r != 300]
+    check_attn(f64(out[0, 1, keep]), oracle_rows(q, k, v, idx.numpy(), 0, 1, rows=keep), "other rows")
+
+
 def test_tail_split_fully_masked_rows():
     """A batch whose every key is padding: no part has an admissible key, so
     the merge reports SAFEDIT_ERR_MASKED_ROW and writes zeros, as the
