@@ -483,7 +483,13 @@ def run_ours(args):
             "roofline": {"kernel": "attn_subset (SRSU)", "bound": "tensor", "achieved": round(achieved, 1),
                          "peak": bf16_sust, "peak_kind": f"bf16_tflops_sustained ({src})",
                          "unit": "TFLOP/s", "frac": round(achieved / bf16_sust, 4),
-                         "frac_of_burst": round(achieved / bf16_burst, 4), "traffic": traffic,
+                         "frac_of_burst": round(achieved / bf16_burst, 4),
+                         # the same call at the SM clock the burst peak runs at: the power cap's
+                         # clock (median under load) against the maximum
+                         "frac_of_burst_at_max_clock": (round(achieved * clk["sm_max_mhz"] / clk["sm_mhz"] /
+                                                              bf16_burst, 4)
+                                                        if clk and clk.get("sm_mhz") else None),
+                         "traffic": traffic,
                          "algorithmic_bytes": algo_bytes,
                          "traffic_over_algorithmic": None if traffic is None else round(traffic / algo_bytes, 3),
                          "mufu_colimit": mufu_colimit(W.d, 0.75)},
