@@ -1174,14 +1174,15 @@ def run_sweep(args):
 
 def run_only(args):
     """One kernel of the path in isolation, `--reps` times on the bench
-    workload's buffers (the target of ncu captures and quick timing).  Prints
-    per-launch CUDA-event times; not a bench line."""
+    workload's buffers (`--config` picks another configuration's; the target
+    of ncu captures and quick timing).  Prints per-launch CUDA-event times;
+    not a bench line."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     from spatially_adaptive_dit_b200 import safedit as sd
-    tr = Trajectory(W, dev)
+    w = {"2560": W, "1024": wl.W1024, "3072": wl.W3072}[args.config]
+    tr = Trajectory(w, dev)
     stream = torch.cuda.Stream(device=dev)
-    w = W
     with torch.cuda.stream(stream):
         sd.safedit_cross_attn_probs(tr.q_img, tr.k_txt, tr.valid, 0, 0.0, tr.P, stream)
         sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream)
@@ -1227,7 +1228,7 @@ def run_only(args):
         "accumulate": (lambda: sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream), None,
                        tr.bytes["partition_accumulate"]),
         "pcsp": (lambda: sd.safedit_pcsp_score(tr.q_img, tr.k_txt, tr.valid, tr.content, 0, 0.0, tr.score,
-                                               stream), None, W.H * W.N * W.d * 2 + W.H * W.L * W.d * 2),
+                                               stream), None, w.H * w.N * w.d * 2 + w.H * w.L * w.d * 2),
         "finalize": (lambda: sd.safedit_partition_finalize(tr.score, w.N, tr.k, tr.idx_s, tr.idx_c, tr.s,
                                                            stream), None, None),
         "scatter": (lambda: sd.safedit_scatter_state([tr.k_s, tr.v_s], [tr.k_state, tr.v_state], tr.idx_s,
@@ -1295,6 +1296,8 @@ def main():
                              "stepcache", "mask", "ffn1", "ffn2", "ffn", "qkv", "sweep", "stress"],
                     help="run one kernel of the path in isolation (profiling target)")
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--config", default="2560", choices=["2560", "1024", "3072"],
+                    help="with --only: the configuration whose buffers the kernel runs on (3072: rho = 0.3)")
     ap.add_argument("--flush", action="store_true", help="--only: flush L2 before every rep (outside the events)")
     ap.add_argument("--cfg-f", type=int, default=W.F, help="prediction width for --only cfg")
     args = ap.parse_args()
