@@ -513,6 +513,8 @@ def run_ours(args):
                         "qkv_projection_gathered": ext["qkv_projection_gathered"]["p50"],
                         "stepcache_sw_cfg": ext["stepcache_sw_cfg"]["p50"]})
             line["oracle_rows"] = oracle_rows(gms)
+            g1024 = {n: e["p50"] for n, e in ext["config_1024"].items() if isinstance(e, dict) and "p50" in e}
+            line["oracle_1024"] = oracle_full_1024(g1024)
         print(json.dumps(line), flush=True)
     if ws > 1:
         torch.distributed.barrier()
@@ -987,6 +989,49 @@ def oracle_rows(gpu_ms):
     row("qkv_projection_gathered", lambda: oracle.linear_act(x, wq, bq, act=0), w.B * w.k / rf,
         f"{rf} focus rows (x{w.B * w.k // rf})")
     return {"cores": oracle.num_threads(), "kind": "oracle", "rows": out}
+
+
+def oracle_full_1024(gpu_ms):
+    """The 1024^2 configuration's calls run in full (no sampling) by the fp64
+    oracle, as it stands, on the host cores, beside the GPU's per-call p50 of
+    this run (`gpu_ms`): probabilities and aggregation of the cond branch, the
+    split, the SRSU rows and the dense anchor over all 48 slices, the K and V
+    scatter of every slice, and the guidance combine."""
+    import numpy as np
+    import oracle
+    w = wl.W1024
+    out = {}
+
+    def row(name, fn, what):
+        t0 = time.perf_counter()
+        r = fn()
+        dt = (time.perf_counter() - t0) * 1e3
+        g = gpu_ms.get(name)
+        out[name] = {"oracle_ms": round(dt, 1), "gpu_ms": None if g is None else round(g, 4),
+                     "oracle_over_gpu": None if not g else round(dt / g, 1), "call": what}
+        return r
+
+    q_img, k_txt, valid, content = wl.text(w)
+    P = row("cross_attn_probs", lambda: oracle.cross_attn_probs(q_img[0], k_txt[0], valid[0]),
+            f"[{w.H}, {w.N}, {w.L}] probabilities")
+    score = row("partition_accumulate", lambda: oracle.partition_accumulate(P, content), "their aggregation")
+    idx_s = row("partition_finalize", lambda: oracle.partition_select(score, w.k), f"the split of N={w.N}")[0]
+    q, k, v = (t.double().numpy() for t in wl.qkv(w))
+    slices = [(b, h) for b in range(w.B) for h in range(w.H)]
+    row("attn_subset_srsu", lambda: [oracle.attn_subset(q[b, h], k[b, h], v[b, h], idx_s) for b, h in slices],
+        f"{w.k} rows x {len(slices)} slices over {w.N} keys")
+    row("attn_dense_anchor", lambda: [oracle.attn_subset(q[b, h], k[b, h], v[b, h]) for b, h in slices],
+        f"all {w.N} rows x {len(slices)} slices (the row-loop routine)")
+    ks, vs = (t.view(torch.int16).numpy() for t in wl.fresh_sensitive_kv(w, w.k, step=1))
+    kst, vst = (t.view(torch.int16).numpy() for t in wl.qkv(w)[1:])
+    row("scatter_state", lambda: [oracle.scatter_rows(src[b, h], dst[b, h], idx_s)
+                                  for src, dst in ((ks, kst), (vs, vst)) for b, h in slices],
+        f"K and V rows of {len(slices)} slices")
+    ec, eu = wl.cfg_preds(w)
+    sv = torch.rand(w.N).numpy()
+    row("sw_cfg", lambda: oracle.sw_cfg(ec, eu, sv, w.gamma_ctx, w.gamma_sens), f"[{w.N}, {w.F}]")
+    return {"cores": oracle.num_threads(), "kind": "oracle", "workload": "1024^2-equivalent, full calls",
+            "rows": out}
 
 
 def cpu_baseline(seconds=12.0, rows=None):
