@@ -38,6 +38,18 @@ def _run_xattn():
     return P
 
 
+def _run_pcsp():
+    g = torch.Generator().manual_seed(9)
+    qi = torch.randn(1, 4, 2048, 96, generator=g).to(torch.bfloat16).to(DEV)
+    kt = torch.randn(1, 4, 256, 96, generator=g).to(torch.bfloat16).to(DEV)
+    valid = torch.ones(1, 256, dtype=torch.uint8, device=DEV)
+    content = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    content[1:200] = 1
+    score = torch.zeros(2048, dtype=torch.float64, device=DEV)
+    sd().safedit_pcsp_score(qi, kt, valid, content, 0, 0.0, score)
+    return score
+
+
 def _run_gemm():
     g = torch.Generator().manual_seed(7)
     a = torch.randn(1000, 512, generator=g).to(torch.bfloat16).to(DEV)
@@ -52,6 +64,7 @@ def test_bounded_wait_timeout_is_reported_and_context_survives():
     ref = _run_attn(q, k, v, idx)
     ref_p = _run_xattn()
     ref_g = _run_gemm()
+    ref_s = _run_pcsp()
     expect_status(0)
     old = sd().safedit_debug_set_wait_limit_ns(0)
     try:
@@ -61,15 +74,19 @@ def test_bounded_wait_timeout_is_reported_and_context_survives():
         expect_status(sd().ERR_TIMEOUT)
         _run_gemm()
         expect_status(sd().ERR_TIMEOUT)
+        _run_pcsp()
+        expect_status(sd().ERR_TIMEOUT)
     finally:
         sd().safedit_debug_set_wait_limit_ns(old)
     again = _run_attn(q, k, v, idx)
     again_p = _run_xattn()
     again_g = _run_gemm()
+    again_s = _run_pcsp()
     expect_status(0)
     assert torch.equal(again, ref)
     assert torch.equal(again_p, ref_p)
     assert torch.equal(again_g, ref_g)
+    assert torch.equal(again_s, ref_s)
 
 
 def test_tail_split_timeout_is_reported_and_context_survives():
