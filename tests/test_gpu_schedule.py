@@ -167,3 +167,45 @@ def test_guidance_branch_sharded_trajectory_matches_unsharded():
         assert torch.equal(br[b].cfg_out, full.cfg_out)
         assert torch.equal(br[b].k_state, full.k_state[b:b + 1])
         check_attn(br[b].o_state.double().cpu().numpy(), full.o_state[b:b + 1].double().cpu().numpy(), f"branch {b}")
+
+
+def test_guidance_branch_sharded_e2e_leg_matches_unsharded():
+    """The benchmark's end-to-end leg (inputs uploaded every step from pinned
+    host memory) in the guidance-branch split, on one GPU: each branch
+    uploads only its own prediction and takes the other's through the
+    exchange hook; the uncond branch uploads no text and takes the split
+    through the share hook.  The guided output and the split must equal
+    those of the unsharded end-to-end leg exactly, and each branch uploads
+    less than the unsharded leg."""
+    import types
+    import bench
+    w = wl.W1024
+    dev = torch.device(DEV)
+    stream = torch.cuda.Stream()
+    args = types.SimpleNamespace(steps=1)
+    full = bench.Trajectory(w, dev)
+    r_full = bench.run_e2e(full, stream, args)
+    torch.cuda.synchronize()
+    br = {}
+
+    def share(tr):
+        if tr.branch == 1:
+            for name in ("idx_s", "idx_c", "s"):
+                getattr(tr, name).copy_(getattr(br[0], name))
+
+    def exchange(tr):
+        tr.eps_c.copy_(br[0].eps_own)
+        tr.eps_u.copy_(br[1].eps_own)
+
+    for b in (0, 1):
+        br[b] = bench.Trajectory(w, dev, branch=b, share_split=share, exchange_eps=exchange)
+    res = {}
+    for b in (0, 1):
+        res[b] = bench.run_e2e(br[b], stream, args)
+        torch.cuda.synchronize()
+    expect_status(0)
+    for b in (0, 1):
+        assert torch.equal(br[b].idx_s, full.idx_s) and torch.equal(br[b].s, full.s)
+        assert torch.equal(br[b].cfg_out, full.cfg_out)
+        assert res[b]["h2d"] < r_full["h2d"]
+    assert res[1]["h2d"] < res[0]["h2d"]  # no text upload on the uncond branch
