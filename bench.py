@@ -1268,6 +1268,12 @@ def run_only(args):
                                                 0.0, tr.o_state, 1, stream), tr.flop_srsu, None),
         "anchor": (lambda: sd.safedit_attn_subset(tr.q, tr.k_state, tr.v_state, None, 0, None, None, 0.0,
                                                   tr.o_state, 0, stream), tr.flop_dense, None),
+        # the tail-balanced entry point as the trajectory calls it (whole units,
+        # key-range parts and their merge where the plan splits)
+        "srsu_ws": (lambda: tr.attn(tr.q, tr.k_state, tr.v_state, tr.idx_s, tr.k, tr.o_state, 1, stream),
+                    tr.flop_srsu, None),
+        "anchor_ws": (lambda: tr.attn(tr.q, tr.k_state, tr.v_state, None, 0, tr.o_state, 0, stream),
+                      tr.flop_dense, None),
         "xattn": (lambda: sd.safedit_cross_attn_probs(tr.q_img, tr.k_txt, tr.valid, 0, 0.0, tr.P, stream),
                   None, tr.bytes["cross_attn_probs"]),
         "accumulate": (lambda: sd.safedit_partition_accumulate(tr.P, tr.content, tr.score, stream), None,
@@ -1337,7 +1343,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,
-                    choices=["srsu", "anchor", "xattn", "accumulate", "pcsp", "finalize", "scatter", "cfg",
+                    choices=["srsu", "anchor", "srsu_ws", "anchor_ws", "xattn", "accumulate", "pcsp", "finalize", "scatter", "cfg",
                              "stepcache", "mask", "ffn1", "ffn2", "ffn", "qkv", "sweep", "stress"],
                     help="run one kernel of the path in isolation (profiling target)")
     ap.add_argument("--reps", type=int, default=5)
