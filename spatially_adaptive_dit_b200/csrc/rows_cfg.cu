@@ -39,6 +39,7 @@ constexpr int kRowIters = 4;  // independent 16-byte copies in flight per thread
 // grid: x = row blocks x column slices, y = b*H + h, z = tensor.  A row of
 // at most kRowThreads 16-byte units is one slice, and a block copies several
 // such rows per pass; a wider row is cut into slices of kRowThreads units.
+// Scattering, a thread's compact-row loads go out before its index loads.
 __global__ void __launch_bounds__(kRowThreads) row_copy_kernel(RowCopyParams p) {
   const int t = blockIdx.z;
   const int bh = blockIdx.y;
@@ -60,28 +61,42 @@ __global__ void __launch_bounds__(kRowThreads) row_copy_kernel(RowCopyParams p) 
   uint4 v[kRowIters];
   int64_t dst_off[kRowIters];
   bool ok[kRowIters];
+  if (p.scatter) {
+    // the compact rows do not depend on the index: their loads go out first
 #pragma unroll
-  for (int it = 0; it < kRowIters; ++it) {
-    const int r = r_base + it * rpp;
-    ok[it] = r < p.n_idx;
-    if (!ok[it]) continue;
-    const int i = __ldg(p.idx + r);
-    if (i < 0 || i >= p.n_rows_x) {
-      set_status(p.status, SAFEDIT_ERR_INDEX);
-      ok[it] = false;
-      continue;
+    for (int it = 0; it < kRowIters; ++it) {
+      const int r = r_base + it * rpp;
+      ok[it] = r < p.n_idx;
+      if (ok[it]) v[it] = __ldcs(reinterpret_cast<const uint4*>(p.src[t] + c_off + int64_t(r) * p.c_sr[t]));
     }
-    int64_t s_off, d_off;
-    if (p.scatter) {
-      s_off = c_off + int64_t(r) * p.c_sr[t];
-      d_off = x_off + int64_t(i) * p.x_sr[t];
-    } else {
-      s_off = x_off + int64_t(i) * p.x_sr[t];
-      d_off = c_off + int64_t(r) * p.c_sr[t];
+#pragma unroll
+    for (int it = 0; it < kRowIters; ++it) {
+      if (!ok[it]) continue;
+      const int r = r_base + it * rpp;
+      const int i = __ldg(p.idx + r);
+      if (i < 0 || i >= p.n_rows_x) {
+        set_status(p.status, SAFEDIT_ERR_INDEX);
+        ok[it] = false;
+        continue;
+      }
+      dst_off[it] = x_off + int64_t(i) * p.x_sr[t];
     }
-    cb_src = p.src[t] + s_off;
-    v[it] = __ldcs(reinterpret_cast<const uint4*>(cb_src));
-    dst_off[it] = d_off;
+  } else {
+#pragma unroll
+    for (int it = 0; it < kRowIters; ++it) {
+      const int r = r_base + it * rpp;
+      ok[it] = r < p.n_idx;
+      if (!ok[it]) continue;
+      const int i = __ldg(p.idx + r);
+      if (i < 0 || i >= p.n_rows_x) {
+        set_status(p.status, SAFEDIT_ERR_INDEX);
+        ok[it] = false;
+        continue;
+      }
+      cb_src = p.src[t] + x_off + int64_t(i) * p.x_sr[t];
+      v[it] = __ldcs(reinterpret_cast<const uint4*>(cb_src));
+      dst_off[it] = c_off + int64_t(r) * p.c_sr[t];
+    }
   }
 #pragma unroll
   for (int it = 0; it < kRowIters; ++it) {
