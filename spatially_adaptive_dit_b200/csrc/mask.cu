@@ -1,8 +1,7 @@
 // mask.cu -- the exact mask-elision criterion (SAFE-DiT summary, 방법론 1;
 // Italian page, Metodologia 1): an additive mask row may be dropped iff it
 // is a constant shift c_i of the logits, i.e. all entries equal entry 0 under
-// IEEE == and that entry is finite.  One warp per row, 128-bit loads (the
-// first element taken from lane 0's first word, so no load waits on it), an
+// IEEE == and that entry is finite.  One warp per row, 128-bit loads, an
 // integer fast path (bit-identical words) with an IEEE fallback (+0 vs -0),
 // a warp vote per row, and an early exit once any row is kept (when per-row
 // flags are not requested).
@@ -84,44 +83,32 @@ __global__ void __launch_bounds__(kMaskWarps * 32) mask_rows_kernel(MaskParams p
   const int es = p.dtype == SAFEDIT_F32 ? 4 : (p.dtype == SAFEDIT_BOOL ? 1 : 2);
   for (int64_t row = blockIdx.x * int64_t(kMaskWarps) + (threadIdx.x >> 5); row < nrows;
        row += nwarps) {
+    // warp-uniform exit once another row has been found kept
+    if (!p.row_flags &&
+        __any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(p.verdict) == 0))
+      return;
     const int64_t q = row % p.Nq;
     const int64_t bh = row / p.Nq;
     const int64_t h = bh % p.Hm, b = bh / p.Hm;
     const char* rp = p.base + (b * p.sb + h * p.sh + q * p.sq) * es;
-    bool ok;
-    if (p.vec) {
-      // the row's first element arrives with lane 0's first word: no load
-      // waits on another before the row streams
-      const int64_t nv = (p.Nk * es) >> 4;  // 16-byte words in the row
-      const uint4* w = reinterpret_cast<const uint4*>(rp);
-      uint4 first = lane < nv ? __ldcs(w + lane) : make_uint4(0u, 0u, 0u, 0u);
-      // warp-uniform exit once another row has been found kept (read while
-      // the row's first words are in flight)
-      if (!p.row_flags &&
-          __any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(p.verdict) == 0))
-        return;
-      uint32_t v0 = __shfl_sync(0xffffffffu, first.x, 0);
-      if (es == 2) v0 &= 0xFFFFu;
-      else if (es == 1) v0 &= 0xFFu;
-      ok = finite_bits(v0, p.dtype);
-      if (lane < nv) ok &= vec_equal(first, v0, p.dtype);
-      int64_t j = lane + 32;
-      for (; j + 96 < nv; j += 128) {
-        const uint4 a = __ldcs(w + j), b2 = __ldcs(w + j + 32), c = __ldcs(w + j + 64),
-                    d = __ldcs(w + j + 96);
-        ok &= vec_equal(a, v0, p.dtype) & vec_equal(b2, v0, p.dtype) &
-              vec_equal(c, v0, p.dtype) & vec_equal(d, v0, p.dtype);
-      }
-      for (; j < nv; j += 32) ok &= vec_equal(__ldcs(w + j), v0, p.dtype);
-    } else {
-      if (!p.row_flags &&
-          __any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(p.verdict) == 0))
-        return;
-      const uint32_t v0 = load_elt(rp, p.dtype);
-      ok = finite_bits(v0, p.dtype);
-      if (ok)
+    const uint32_t v0 = load_elt(rp, p.dtype);
+    bool ok = finite_bits(v0, p.dtype);
+    if (ok) {
+      if (p.vec) {
+        const int64_t nv = (p.Nk * es) >> 4;  // 16-byte words in the row
+        const uint4* w = reinterpret_cast<const uint4*>(rp);
+        int64_t j = lane;
+        for (; j + 96 < nv; j += 128) {
+          const uint4 a = __ldcs(w + j), b2 = __ldcs(w + j + 32), c = __ldcs(w + j + 64),
+                      d = __ldcs(w + j + 96);
+          ok &= vec_equal(a, v0, p.dtype) & vec_equal(b2, v0, p.dtype) &
+                vec_equal(c, v0, p.dtype) & vec_equal(d, v0, p.dtype);
+        }
+        for (; j < nv; j += 32) ok &= vec_equal(__ldcs(w + j), v0, p.dtype);
+      } else {
         for (int64_t j = lane; j < p.Nk; j += 32)
           ok &= elt_equal(load_elt(rp + j * p.sk * es, p.dtype), v0, p.dtype);
+      }
     }
     ok = __all_sync(0xffffffffu, ok);
     if (lane == 0) {
